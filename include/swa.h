@@ -1,0 +1,191 @@
+/*
+ * swa.h -- C ABI of libswa.so: sliding-window attention (SWA) forward and
+ * ring-buffer decode on NVIDIA B200 (sm_100a).
+ *
+ * Every call is asynchronous on the CUDA stream passed as `stream` (a
+ * cudaStream_t as void*; NULL = the legacy default stream).  All pointers
+ * to tensors are DEVICE pointers owned by the caller; the library reads the
+ * inputs and writes the outputs and keeps no reference after the call
+ * returns.  Arguments are validated on the host before anything is
+ * launched: on failure the call returns a negative swa_status and launches
+ * nothing.  No call synchronises the stream; swa_device_error() does.
+ *
+ * Definitions (page title, section):
+ *  - Window and output: "滑动窗口注意力" (bmjup.com/post/11897), section
+ *    "滑动窗口注意力的核心原理" 1: query i attends only the keys of its
+ *    window, y_i = sum_j softmax(q_i . k_j * scale) v_j; keys outside the
+ *    window are not computed at all ("别再只加Mask了", §1: real SWA skips
+ *    them physically instead of masking an n x n matrix).
+ *  - Causal window: "滑动窗口注意力：Mistral 的长文本“接力跑”智慧"
+ *    (aiqz.cc), "Python 演示": the last window_size keys including the
+ *    current token.
+ *  - Dilation: "空洞滑窗机制" (mhpn.cn/news/940557), §二.1: j = i + k*d,
+ *    k in [-w, w]; §四: dilation at the level of 64-token blocks, dense
+ *    inside each block.
+ *  - Global tokens: aiqz.cc page, "全局注意力token": a global token attends
+ *    to all keys and all queries attend to it.
+ *  - Ring cache: "大模型窗口扩展技术" (intelliparadigm.com), §3.1: the
+ *    stream item with index t is stored in slot t % window_size.
+ *
+ * Key set of query i (token-level; win_left = L, win_right = R, dilation d):
+ *     K(i) = { i + k*d : -L <= k <= R, 0 <= i + k*d < N }
+ *            U { global keys }  U { 0 .. N-1 if i is global }
+ *     and, when R == 0 (causal), only keys j <= i are kept.
+ *  L < 0 (R < 0) means unbounded on the left (right).  A key is counted once
+ *  even when it is both in the band and global.
+ *  Block-level dilation (dilation_block = Bs > 1): with b_i = i / Bs,
+ *     K(i) = union over m in [-(L / Bs), R / Bs] of the block
+ *            [(b_i + m*d)*Bs, (b_i + m*d + 1)*Bs) cut to [0, N),
+ *     then globals and the causal clip as above.
+ *
+ * Layouts (row-major, contiguous, "[batch_size, seq_len, num_heads,
+ * head_dim]" as on page "别再只加Mask了", §3):
+ *     q, out            [B, N, H, D]
+ *     k, v              [B, N, Hkv, D]       query head h reads kv head
+ *                                            h / (H / Hkv)  (GQA)
+ *     lse               [B, H, N]  fp32, natural log of the softmax
+ *                                  denominator: ln sum_j exp(s_ij)
+ *     global_idx        [n_global] int32, sorted ascending, unique, in
+ *                                  [0, N); shared by all batches and heads
+ *     decode q, out     [B, H, D]
+ *     k_ring, v_ring    [B, W, Hkv, D]
+ *     pos               [B] int64 (device)
+ */
+#ifndef SWA_H_
+#define SWA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define SWA_API __attribute__((visibility("default")))
+#else
+#define SWA_API
+#endif
+
+typedef enum {
+  SWA_OK = 0,
+  SWA_ERR_ARG = -1,         /* null pointer, bad size, H % Hkv != 0, d < 1 ... */
+  SWA_ERR_ALIGN = -2,       /* a tensor pointer is not 16-byte aligned         */
+  SWA_ERR_UNSUPPORTED = -3, /* valid but not implemented (e.g. D not 64/128)   */
+  SWA_ERR_CUDA = -4,        /* a CUDA runtime/driver call failed               */
+  SWA_ERR_TIMEOUT = -5,     /* a device-side wait gave up (see swa_device_error) */
+  SWA_ERR_NOMEM = -6        /* library workspace could not be allocated        */
+} swa_status;
+
+/*
+ * swa_forward -- bf16 SWA prefill (the fused tcgen05 kernel).
+ *
+ * q, k, v: bf16 device tensors (layouts above).  out: bf16 [B,N,H,D].
+ * lse: fp32 [B,H,N] or NULL.  D must be 64 or 128.  win_left, win_right:
+ * window half-widths in dilation steps (negative = unbounded; win_right ==
+ * 0 = causal).  dilation >= 1.  global_idx: device int32 array of n_global
+ * entries (NULL iff n_global == 0).  scale <= 0 selects 1/sqrt(D) (the
+ * "softmax_scale None" default on page "别再只加Mask了", §3).
+ * B == 0 or N == 0 is a no-op returning SWA_OK.  The call allocates no
+ * device memory.  Entries of global_idx outside [0, N) are clamped when
+ * read (no out-of-bounds access) but then the result is unspecified.
+ */
+SWA_API int swa_forward(const void* q, const void* k, const void* v, void* out,
+                        float* lse, int B, int H, int Hkv, int N, int D,
+                        int win_left, int win_right, int dilation,
+                        const int32_t* global_idx, int n_global, float scale,
+                        void* stream);
+
+/*
+ * swa_forward_ex -- swa_forward with block-level dilation.
+ * dilation_block <= 1 is token-level dilation (identical to swa_forward);
+ * dilation_block = Bs > 1 applies the dilation to whole Bs-token blocks
+ * ("空洞滑窗机制" §四).  The fused kernel supports Bs = 64 (its tile is two
+ * 64-row blocks); other Bs > 1 return SWA_ERR_UNSUPPORTED.
+ */
+SWA_API int swa_forward_ex(const void* q, const void* k, const void* v, void* out,
+                           float* lse, int B, int H, int Hkv, int N, int D,
+                           int win_left, int win_right, int dilation,
+                           int dilation_block, const int32_t* global_idx,
+                           int n_global, float scale, void* stream);
+
+/*
+ * swa_forward_f32 -- the same operation in fp32 (q, k, v, out are float*),
+ * computed with fp32 FFMA on CUDA cores (no TF32), for callers that need
+ * fp32 accuracy.  D in {32, 64, 96, 128}; any dilation_block >= 0.
+ */
+SWA_API int swa_forward_f32(const float* q, const float* k, const float* v,
+                            float* out, float* lse, int B, int H, int Hkv, int N,
+                            int D, int win_left, int win_right, int dilation,
+                            int dilation_block, const int32_t* global_idx,
+                            int n_global, float scale, void* stream);
+
+/*
+ * swa_decode -- one new query token per sequence against a ring-buffer KV
+ * cache of W slots (bf16).  Sequence b's token is at position pos[b] >= 0;
+ * the caller has already written its k/v into slot pos[b] % W.  The query
+ * attends positions max(0, pos-W+1) .. pos, i.e. ring slots
+ * 0 .. min(pos, W-1) (all W slots once pos >= W-1).  scale is 1/sqrt(D).
+ * D must be 128 or 64; H % Hkv == 0 and H / Hkv <= 8.
+ * The first call on a device allocates a small library-owned workspace
+ * (split partials and counters, kept until swa_release); make that first
+ * call before capturing a CUDA graph.  Calls on different streams of one
+ * device share that workspace and must not overlap.
+ */
+SWA_API int swa_decode(const void* q, const void* k_ring, const void* v_ring,
+                       void* out, const int64_t* pos, int B, int H, int Hkv,
+                       int D, int W, void* stream);
+
+/* swa_decode_ex -- swa_decode that also writes lse [B,H] (fp32, may be NULL)
+   and takes a scale (<= 0: 1/sqrt(D)). */
+SWA_API int swa_decode_ex(const void* q, const void* k_ring, const void* v_ring,
+                          void* out, float* lse, const int64_t* pos, int B, int H,
+                          int Hkv, int D, int W, float scale, void* stream);
+
+/*
+ * swa_device_error -- synchronises `stream`, then reports (and clears) a
+ * device-side timeout: every wait inside the kernels is bounded, and a wait
+ * that gives up records an error word instead of hanging.  Returns SWA_OK,
+ * SWA_ERR_TIMEOUT or SWA_ERR_CUDA.
+ */
+SWA_API int swa_device_error(void* stream);
+
+/*
+ * swa_selftest_timeout -- launches one tiny kernel that waits on an mbarrier
+ * nobody arrives at, with a limit of `limit_us` microseconds, so the bounded
+ * wait expires and records its error.  Used by the failure-detection test;
+ * follow with swa_device_error(), which then returns SWA_ERR_TIMEOUT.
+ */
+SWA_API int swa_selftest_timeout(int limit_us, void* stream);
+
+/*
+ * swa_schedule -- host-only query of the band-aware tile scheduler (no GPU
+ * needed).  For the forward problem (N, win_left, win_right, dilation,
+ * dilation_block, n_global), writes one record of 6 int32 per query tile:
+ *   { residue_class, q_tile, first_row, kv_tile_begin, kv_tile_end, n_edge }
+ * where the 128-row query tile covers virtual rows [first_row,
+ * first_row+128) of its residue class, it visits kv tiles [begin, end) of
+ * 128 keys of the same class, and n_edge of those need the element mask
+ * (the rest lie wholly inside every row's window).  Rows of residue class c
+ * are the positions c, c+d, c+2d, ... (token-level) or the blocks
+ * c, c+d, ... (block-level).  The global-key tiles, if any, follow the band
+ * tiles and are not counted.  Returns the number of query tiles (the
+ * records written are min(that, cap)), or a negative swa_status.
+ * tile_out may be NULL to count only.
+ */
+SWA_API int swa_schedule(int N, int win_left, int win_right, int dilation,
+                         int dilation_block, int32_t* tile_out, int cap);
+
+/* swa_release -- frees library-owned workspaces on the current device. */
+SWA_API int swa_release(void);
+
+/* swa_status_string -- static text for a status code. */
+SWA_API const char* swa_status_string(int status);
+
+/* swa_version -- library version, major * 10000 + minor * 100 + patch. */
+SWA_API int swa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SWA_H_ */

@@ -1,0 +1,195 @@
+"""ctypes marshalling between torch tensors and the C ABI of libswa.so."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libswa.so")
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"libswa.so not found at {_LIB_PATH}: build it with "
+        "`python -m sliding_window_attention_fwd_b200.build` (nvcc, sm_100a)")
+
+_lib = ctypes.CDLL(_LIB_PATH)
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+
+_lib.swa_forward.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _F, _P]
+_lib.swa_forward_ex.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I,
+                                _F, _P]
+_lib.swa_forward_f32.argtypes = _lib.swa_forward_ex.argtypes
+_lib.swa_decode.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
+_lib.swa_decode_ex.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
+_lib.swa_device_error.argtypes = [_P]
+_lib.swa_selftest_timeout.argtypes = [_I, _P]
+_lib.swa_schedule.argtypes = [_I, _I, _I, _I, _I, _P, _I]
+_lib.swa_release.argtypes = []
+_lib.swa_status_string.argtypes = [_I]
+_lib.swa_status_string.restype = ctypes.c_char_p
+_lib.swa_version.argtypes = []
+for _fn in ("swa_forward", "swa_forward_ex", "swa_forward_f32", "swa_decode", "swa_decode_ex",
+            "swa_device_error", "swa_selftest_timeout", "swa_schedule", "swa_release",
+            "swa_version"):
+    getattr(_lib, _fn).restype = _I
+
+
+class SwaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {swa_status_string(status)} ({status})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def swa_status_string(status: int) -> str:
+    return _lib.swa_status_string(int(status)).decode()
+
+
+def swa_version() -> int:
+    return _lib.swa_version()
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise SwaError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t, name, dtype, ndim):
+    if t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name}: expected {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name}: must be a contiguous CUDA tensor")
+
+
+def _fwd_common(q, k, v, out, lse, global_idx, dtype):
+    _need(q, "q", dtype, 4)
+    _need(k, "k", dtype, 4)
+    _need(v, "v", dtype, 4)
+    B, N, H, D = q.shape
+    Hkv = k.shape[2]
+    if k.shape != (B, N, Hkv, D) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, N, Hkv, D] matching q [B, N, H, D]")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", dtype, 4)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 3)
+    ng = 0
+    if global_idx is not None and global_idx.numel() > 0:
+        _need(global_idx, "global_idx", torch.int32, 1)
+        ng = global_idx.numel()
+    else:
+        global_idx = None
+    return B, N, H, Hkv, D, out, global_idx, ng
+
+
+def swa_forward(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dilation=1,
+                global_idx=None, scale=0.0, stream=None):
+    """bf16 SWA forward (C: swa_forward).  Returns out."""
+    B, N, H, Hkv, D, out, gi, ng = _fwd_common(q, k, v, out, lse, global_idx, torch.bfloat16)
+    _check(_lib.swa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N, D,
+                            int(win_left), int(win_right), int(dilation), _ptr(gi), ng,
+                            float(scale), _stream(stream)), "swa_forward")
+    return out
+
+
+def swa_forward_ex(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dilation=1,
+                   dilation_block=0, global_idx=None, scale=0.0, stream=None):
+    """bf16 SWA forward with block-level dilation (C: swa_forward_ex)."""
+    B, N, H, Hkv, D, out, gi, ng = _fwd_common(q, k, v, out, lse, global_idx, torch.bfloat16)
+    _check(_lib.swa_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N, D,
+                               int(win_left), int(win_right), int(dilation), int(dilation_block),
+                               _ptr(gi), ng, float(scale), _stream(stream)), "swa_forward_ex")
+    return out
+
+
+def swa_forward_f32(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dilation=1,
+                    dilation_block=0, global_idx=None, scale=0.0, stream=None):
+    """fp32 SWA forward on CUDA cores (C: swa_forward_f32)."""
+    B, N, H, Hkv, D, out, gi, ng = _fwd_common(q, k, v, out, lse, global_idx, torch.float32)
+    _check(_lib.swa_forward_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N,
+                                D, int(win_left), int(win_right), int(dilation),
+                                int(dilation_block), _ptr(gi), ng, float(scale),
+                                _stream(stream)), "swa_forward_f32")
+    return out
+
+
+def _dec_common(q, k_ring, v_ring, out, pos):
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_ring, "k_ring", torch.bfloat16, 4)
+    _need(v_ring, "v_ring", torch.bfloat16, 4)
+    _need(pos, "pos", torch.int64, 1)
+    B, H, D = q.shape
+    W, Hkv = k_ring.shape[1], k_ring.shape[2]
+    if k_ring.shape != (B, W, Hkv, D) or v_ring.shape != k_ring.shape or pos.shape != (B,):
+        raise ValueError("k_ring/v_ring must be [B, W, Hkv, D] and pos [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 3)
+    return B, H, Hkv, D, W, out
+
+
+def swa_decode(q, k_ring, v_ring, pos, out=None, stream=None):
+    """Ring-buffer decode (C: swa_decode).  Returns out [B, H, D]."""
+    B, H, Hkv, D, W, out = _dec_common(q, k_ring, v_ring, out, pos)
+    _check(_lib.swa_decode(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(out), _ptr(pos), B, H, Hkv,
+                           D, W, _stream(stream)), "swa_decode")
+    return out
+
+
+def swa_decode_ex(q, k_ring, v_ring, pos, out=None, lse=None, scale=0.0, stream=None):
+    """Ring-buffer decode that also writes lse [B, H] (C: swa_decode_ex)."""
+    B, H, Hkv, D, W, out = _dec_common(q, k_ring, v_ring, out, pos)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    _check(_lib.swa_decode_ex(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(out), _ptr(lse),
+                              _ptr(pos), B, H, Hkv, D, W, float(scale), _stream(stream)),
+           "swa_decode_ex")
+    return out
+
+
+def swa_device_error(stream=None) -> int:
+    """Synchronises the stream; returns 0 or the (negative) status of a device timeout."""
+    return _lib.swa_device_error(_stream(stream))
+
+
+def swa_selftest_timeout(limit_us: int, stream=None) -> None:
+    _check(_lib.swa_selftest_timeout(int(limit_us), _stream(stream)), "swa_selftest_timeout")
+
+
+def swa_schedule(N, win_left, win_right, dilation=1, dilation_block=0):
+    """Host-only scheduler query: list of (class, q_tile, first_row, kv_begin, kv_end, n_edge)."""
+    n = _lib.swa_schedule(int(N), int(win_left), int(win_right), int(dilation),
+                          int(dilation_block), None, 0)
+    if n < 0:
+        raise SwaError(n, "swa_schedule")
+    buf = (ctypes.c_int32 * (6 * max(n, 1)))()
+    n2 = _lib.swa_schedule(int(N), int(win_left), int(win_right), int(dilation),
+                           int(dilation_block), ctypes.cast(buf, ctypes.c_void_p), n)
+    if n2 < 0:
+        raise SwaError(n2, "swa_schedule")
+    return [tuple(buf[6 * t: 6 * t + 6]) for t in range(n)]
+
+
+def swa_release() -> None:
+    _check(_lib.swa_release(), "swa_release")

@@ -1,0 +1,264 @@
+// swa_capi.cu -- the extern "C" boundary of libswa.so: argument checks,
+// dispatch to the kernels, device error word, host-side scheduler query.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "swa.h"
+#include "swa_internal.h"
+#include "swa_ptx.cuh"
+#include "swa_sched.cuh"
+
+namespace swa {
+
+__device__ int g_device_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices] = {};
+std::mutex g_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+__global__ void timeout_selftest_kernel(int* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nobody arrives on `bar`: the bounded wait must give up and report.
+    mbar_wait(&bar, 0, err, &abort_flag, limit_ns);
+  }
+  __syncthreads();
+}
+
+}  // namespace
+
+int* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<int*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+CUresult encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* base,
+                      const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                      CUtensorMapSwizzle swizzle) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return CUDA_ERROR_NOT_FOUND;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+  }
+  cuuint64_t d[5], s[4];
+  cuuint32_t b[5], e[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    b[i] = box[i];
+    e[i] = 1;
+    if (i < rank - 1) s[i] = strides_bytes[i];
+  }
+  return g_encode(map, dtype, (cuuint32_t)rank, base, d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+int launch_timeout_selftest(int limit_us, cudaStream_t stream) {
+  int* err = device_error_word();
+  if (!err) return SWA_ERR_CUDA;
+  timeout_selftest_kernel<<<1, 32, 0, stream>>>(err, (uint64_t)limit_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+}  // namespace swa
+
+using namespace swa;
+
+namespace {
+
+int check_forward_args(const void* q, const void* k, const void* v, const void* out,
+                       const float* lse, int B, int H, int Hkv, int N, int D, int dilation,
+                       int dilation_block, const int32_t* global_idx, int n_global) {
+  if (B < 0 || N < 0 || H <= 0 || Hkv <= 0 || D <= 0) return SWA_ERR_ARG;
+  if (H % Hkv != 0) return SWA_ERR_ARG;
+  if (dilation < 1 || dilation_block < 0) return SWA_ERR_ARG;
+  if (n_global < 0 || n_global > N || (n_global > 0 && !global_idx)) return SWA_ERR_ARG;
+  if (!q || !k || !v || !out) return SWA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SWA_ERR_ALIGN;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SWA_ERR_ALIGN;
+  if (global_idx && (reinterpret_cast<uintptr_t>(global_idx) & 3u)) return SWA_ERR_ALIGN;
+  return SWA_OK;
+}
+
+float resolve_scale(float scale, int D) {
+  return scale > 0.f ? scale : 1.0f / std::sqrt((float)D);
+}
+
+}  // namespace
+
+extern "C" {
+
+SWA_API int swa_forward_ex(const void* q, const void* k, const void* v, void* out, float* lse,
+                           int B, int H, int Hkv, int N, int D, int win_left, int win_right,
+                           int dilation, int dilation_block, const int32_t* global_idx,
+                           int n_global, float scale, void* stream) {
+  int st = check_forward_args(q, k, v, out, lse, B, H, Hkv, N, D, dilation, dilation_block,
+                              global_idx, n_global);
+  if (st != SWA_OK) return st;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (dilation_block > 1 && dilation_block != kBlockRows) return SWA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return SWA_OK;
+  const float sc = resolve_scale(scale, D);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  st = launch_fwd_sm100(q, k, v, out, lse, B, H, Hkv, N, D, win_left, win_right, dilation,
+                        dilation_block, global_idx, n_global, sc, s);
+  if (st != SWA_OK) return st;
+  if (n_global > 0)
+    st = launch_global_rows(q, k, v, out, lse, B, H, Hkv, N, D, win_right == 0, global_idx,
+                            n_global, sc, s);
+  return st;
+}
+
+SWA_API int swa_forward(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int B, int H, int Hkv, int N, int D, int win_left, int win_right,
+                        int dilation, const int32_t* global_idx, int n_global, float scale,
+                        void* stream) {
+  return swa_forward_ex(q, k, v, out, lse, B, H, Hkv, N, D, win_left, win_right, dilation, 0,
+                        global_idx, n_global, scale, stream);
+}
+
+SWA_API int swa_forward_f32(const float* q, const float* k, const float* v, float* out,
+                            float* lse, int B, int H, int Hkv, int N, int D, int win_left,
+                            int win_right, int dilation, int dilation_block,
+                            const int32_t* global_idx, int n_global, float scale,
+                            void* stream) {
+  int st = check_forward_args(q, k, v, out, lse, B, H, Hkv, N, D, dilation, dilation_block,
+                              global_idx, n_global);
+  if (st != SWA_OK) return st;
+  if (D != 32 && D != 64 && D != 96 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return SWA_OK;
+  return launch_fwd_f32(q, k, v, out, lse, B, H, Hkv, N, D, win_left, win_right, dilation,
+                        dilation_block, global_idx, n_global, resolve_scale(scale, D),
+                        static_cast<cudaStream_t>(stream));
+}
+
+SWA_API int swa_decode_ex(const void* q, const void* k_ring, const void* v_ring, void* out,
+                          float* lse, const int64_t* pos, int B, int H, int Hkv, int D, int W,
+                          float scale, void* stream) {
+  if (B < 0 || H <= 0 || Hkv <= 0 || D <= 0 || W <= 0) return SWA_ERR_ARG;
+  if (H % Hkv != 0) return SWA_ERR_ARG;
+  if (!q || !k_ring || !v_ring || !out || !pos) return SWA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_ring) || !aligned16(v_ring) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(pos) & 7u))
+    return SWA_ERR_ALIGN;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SWA_ERR_ALIGN;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (H / Hkv > 8) return SWA_ERR_UNSUPPORTED;
+  if (B == 0) return SWA_OK;
+  return launch_decode(q, k_ring, v_ring, out, lse, pos, B, H, Hkv, D, W,
+                       resolve_scale(scale, D), static_cast<cudaStream_t>(stream));
+}
+
+SWA_API int swa_decode(const void* q, const void* k_ring, const void* v_ring, void* out,
+                       const int64_t* pos, int B, int H, int Hkv, int D, int W, void* stream) {
+  return swa_decode_ex(q, k_ring, v_ring, out, nullptr, pos, B, H, Hkv, D, W, 0.f, stream);
+}
+
+SWA_API int swa_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return SWA_ERR_CUDA;
+  int* err = device_error_word();
+  if (!err) return SWA_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpy(&h, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return SWA_ERR_CUDA;
+  if (h != 0) {
+    int zero = 0;
+    if (cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return SWA_ERR_CUDA;
+    // An aborted kernel may have left split counters mid-count.
+    release_workspaces();
+    return SWA_ERR_TIMEOUT;
+  }
+  return SWA_OK;
+}
+
+SWA_API int swa_selftest_timeout(int limit_us, void* stream) {
+  if (limit_us <= 0) return SWA_ERR_ARG;
+  return launch_timeout_selftest(limit_us, static_cast<cudaStream_t>(stream));
+}
+
+SWA_API int swa_schedule(int N, int win_left, int win_right, int dilation, int dilation_block,
+                         int32_t* tile_out, int cap) {
+  if (N < 0 || dilation < 1 || dilation_block < 0 || cap < 0) return SWA_ERR_ARG;
+  if (dilation_block > 1 && dilation_block != kBlockRows) return SWA_ERR_UNSUPPORTED;
+  Geometry g = make_geometry(N, win_left, win_right, dilation, dilation_block);
+  int n = 0;
+  for (int c = 0; c < g.nclass; ++c) {
+    const int Mv = class_valid_rows(g, c);
+    const int nqt = (Mv + kTileM - 1) / kTileM;
+    for (int qt = 0; qt < nqt; ++qt) {
+      if (tile_out && n < cap) {
+        TileRange r = tile_range(g, Mv, qt);
+        int edges = 0;
+        for (int t = r.kv_begin; t < r.kv_end; ++t) edges += tile_interior(g, Mv, qt, t) ? 0 : 1;
+        int32_t* o = tile_out + 6 * n;
+        o[0] = c;
+        o[1] = qt;
+        o[2] = qt * kTileM;
+        o[3] = r.kv_begin;
+        o[4] = r.kv_end;
+        o[5] = edges;
+      }
+      ++n;
+    }
+  }
+  return n;
+}
+
+SWA_API int swa_release(void) {
+  release_workspaces();
+  return SWA_OK;
+}
+
+SWA_API const char* swa_status_string(int status) {
+  switch (status) {
+    case SWA_OK: return "ok";
+    case SWA_ERR_ARG: return "invalid argument";
+    case SWA_ERR_ALIGN: return "tensor pointer not 16-byte aligned";
+    case SWA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SWA_ERR_CUDA: return "CUDA error";
+    case SWA_ERR_TIMEOUT: return "device-side wait timed out";
+    case SWA_ERR_NOMEM: return "workspace allocation failed";
+    default: return "unknown status";
+  }
+}
+
+SWA_API int swa_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,43 @@
+// swa_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "swa.h"
+
+namespace swa {
+
+// Device error word of the current device (bounded waits write into it).
+int* device_error_word();
+
+// Encodes a tiled tensor map through the driver entry point (no -lcuda).
+CUresult encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* base,
+                      const uint64_t* dims, const uint64_t* strides_bytes,
+                      const uint32_t* box, CUtensorMapSwizzle swizzle);
+
+int launch_fwd_f32(const float* q, const float* k, const float* v, float* out, float* lse,
+                   int B, int H, int Hkv, int N, int D, int L, int R, int d, int bs,
+                   const int32_t* G, int ng, float scale, cudaStream_t stream);
+
+int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, float* lse,
+                     int B, int H, int Hkv, int N, int D, int L, int R, int d, int bs,
+                     const int32_t* G, int ng, float scale, cudaStream_t stream);
+
+// Dense rows for global queries: every global row i attends keys
+// [0, N) (causal: [0, i]); overwrites those rows of out / lse.
+int launch_global_rows(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int H, int Hkv, int N, int D, bool causal, const int32_t* G,
+                       int ng, float scale, cudaStream_t stream);
+
+int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* out,
+                  float* lse, const int64_t* pos, int B, int H, int Hkv, int D, int W,
+                  float scale, cudaStream_t stream);
+
+int launch_timeout_selftest(int limit_us, cudaStream_t stream);
+
+void release_workspaces();
+
+}  // namespace swa

@@ -1,0 +1,582 @@
+// swa_rowattn.cu -- split-KV attention of a few query vectors against a long
+// contiguous run of key rows, on CUDA cores.  Two users:
+//
+//  * ring-buffer decode: one new token per sequence attends the valid slots
+//    of its W-slot cache (page "大模型窗口扩展技术" §3.1: token t lives in
+//    slot t % W; aiqz.cc page, "推理优化策略": the cache rolls like a
+//    conveyor belt, old entries are overwritten);
+//  * global query rows: a global token attends every key (aiqz.cc page,
+//    "全局注意力token"); causal problems clip it to keys <= its position.
+//
+// The work is HBM-bound (each key/value byte is used for a handful of
+// flops), so the kernel is built for bandwidth: one CTA streams a chunk of
+// key rows of one (batch, kv head) through a 3-stage TMA ring (64 rows per
+// stage, 128-byte swizzle so the reads below are bank-conflict free) and
+// serves all NQ query vectors that read those rows (the GQA group of the kv
+// head, and for global rows several global tokens) from that single read.
+// Math is fp32 on the FMA pipe.  Chunks of one query set are merged with
+// the log-sum-exp identity by whichever CTA of the set finishes last.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "swa_internal.h"
+#include "swa_ptx.cuh"
+
+namespace swa {
+namespace {
+
+constexpr int kRows = 64;           // key rows per stage
+constexpr int kStagesR = 3;
+constexpr int kComputeWarps = 4;
+constexpr int kThreadsR = (kComputeWarps + 1) * 32;
+
+struct RowParams {
+  CUtensorMap tmK;
+  CUtensorMap tmV;
+  const uint16_t* q;
+  uint16_t* out;
+  float* lse;
+  const int64_t* pos;
+  const int32_t* G;
+  float* ws_o;
+  float* ws_ml;
+  int* cnt;
+  int* err;
+  int mode;  // 0: decode, 1: global rows
+  int B, H, Hkv, N, W, grp, ng, causal;
+  int rows_per_cta, nrowchunks;
+  int chunk, nsplit;
+  float scale_log2;
+};
+
+template <int D, int NQ>
+struct RSmem {
+  static constexpr int kTile = kRows * D * 2;
+  static constexpr int kStage = 2 * kTile;
+  static constexpr int kSc = kStagesR * kStage;
+  static constexpr int kPc = kSc + kRows * NQ * 4;
+  static constexpr int kCorr = kPc + kRows * NQ * 4;
+  static constexpr int kBar = kCorr + 64;
+  static constexpr int kMisc = kBar + 2 * kStagesR * 8;
+  static constexpr int kTotal = kMisc + 16;
+  static constexpr int kAlloc = kTotal + 1024;
+  static_assert((128 / (D / 8)) * NQ * D * 4 <= kSc, "reduction buffer must fit in the ring");
+};
+
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+template <int D, int NQ>
+__global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_constant__ RowParams p) {
+  using S = RSmem<D, NQ>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  float* sc = reinterpret_cast<float*>(smem + S::kSc);
+  float* pc = reinterpret_cast<float*>(smem + S::kPc);
+  float* corr_s = reinterpret_cast<float*>(smem + S::kCorr);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint64_t* empty = full + kStagesR;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kMisc);
+  int* last_flag = reinterpret_cast<int*>(smem + S::kMisc + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int split = blockIdx.x;
+  const int gi = blockIdx.y;  // query set
+
+  // ---- the query set: kv head, batch, query vectors and their key limits
+  int b, g, rowchunk = 0;
+  if (p.mode == 0) {
+    g = gi % p.Hkv;
+    b = gi / p.Hkv;
+  } else {
+    rowchunk = gi % p.nrowchunks;
+    g = (gi / p.nrowchunks) % p.Hkv;
+    b = gi / (p.nrowchunks * p.Hkv);
+  }
+  // per slot: query row pointer offset and key limit (keys [0, limit))
+  long qoff[NQ];
+  int limit[NQ];
+  int max_limit = 0;
+#pragma unroll
+  for (int s = 0; s < NQ; ++s) {
+    const int hsub = s % p.grp, rsub = s / p.grp;
+    const int h = g * p.grp + hsub;
+    qoff[s] = -1;
+    limit[s] = 0;
+    if (rsub < p.rows_per_cta) {
+      if (p.mode == 0) {
+        long long ps = p.pos[b];
+        limit[s] = ps + 1 < (long long)p.W ? (int)(ps + 1) : p.W;
+        qoff[s] = ((long)b * p.H + h) * D;
+      } else {
+        const int j = rowchunk * p.rows_per_cta + rsub;
+        if (j < p.ng) {
+          int i = p.G[j];
+          i = i < 0 ? 0 : (i >= p.N ? p.N - 1 : i);
+          limit[s] = p.causal ? i + 1 : p.N;
+          qoff[s] = (((long)b * p.N + i) * p.H + h) * D;
+        }
+      }
+    }
+    max_limit = limit[s] > max_limit ? limit[s] : max_limit;
+  }
+  const int key0 = split * p.chunk;
+  int nk = max_limit - key0;
+  nk = nk < 0 ? 0 : (nk > p.chunk ? p.chunk : nk);
+  const int n_stages = (nk + kRows - 1) / kRows;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kStagesR; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kComputeWarps * 32);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // running softmax state of the slots this warp owns in the stats phase
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+  constexpr int kCPL = D / 64;        // 16-byte chunks per lane per row (QK)
+  constexpr int kLanesPV = D / 8;     // lanes per value row (PV)
+  constexpr int kRG = 128 / kLanesPV; // row groups in PV
+  float acc[NQ][8];
+#pragma unroll
+  for (int s = 0; s < NQ; ++s)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[s][e] = 0.f;
+
+  if (warp == kComputeWarps) {
+    // ============================ producer ============================
+    if (lane == 0) {
+      prefetch_tensormap(&p.tmK);
+      prefetch_tensormap(&p.tmV);
+      for (int k = 0; k < n_stages; ++k) {
+        const int st = k % kStagesR;
+        if (k >= kStagesR &&
+            !mbar_wait(&empty[st], ((uint32_t)(k / kStagesR) & 1u) ^ 1u, p.err, abort_flag))
+          break;
+        uint8_t* kb = smem + st * S::kStage;
+        uint8_t* vb = kb + S::kTile;
+        mbar_arrive_expect_tx(&full[st], S::kStage);
+        for (int cc = 0; cc < D / 64; ++cc) {
+          tma_load_4d(kb + cc * (kRows * 128), &p.tmK, &full[st], cc * 64, g, key0 + k * kRows, b);
+          tma_load_4d(vb + cc * (kRows * 128), &p.tmV, &full[st], cc * 64, g, key0 + k * kRows, b);
+        }
+      }
+    }
+  } else {
+    // ============================ compute ============================
+    // QK mapping: 8 lanes per key row, lane t reads 16-byte chunk t of each
+    // 128-byte half of the row; a warp covers 4 rows per step.
+    const int t8 = lane & 7, rsub = lane >> 3;
+    float qv[NQ][kCPL * 8];
+#pragma unroll
+    for (int s = 0; s < NQ; ++s) {
+#pragma unroll
+      for (int hh = 0; hh < kCPL; ++hh) {
+        uint4 w = make_uint4(0u, 0u, 0u, 0u);
+        if (qoff[s] >= 0) w = __ldg(reinterpret_cast<const uint4*>(p.q + qoff[s] + hh * 64 + t8 * 8));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          qv[s][hh * 8 + 2 * e] = bf_lo(ws[e]) * p.scale_log2;
+          qv[s][hh * 8 + 2 * e + 1] = bf_hi(ws[e]) * p.scale_log2;
+        }
+      }
+    }
+    const int pv_chunk = threadIdx.x % kLanesPV;  // 16-byte chunk of a value row
+    const int pv_rg = threadIdx.x / kLanesPV;
+
+    for (int k = 0; k < n_stages; ++k) {
+      const int st = k % kStagesR;
+      // A wait that gives up (error recorded, abort set) does not leave the
+      // loop: every compute warp keeps taking the same named barriers, so the
+      // CTA always finishes; its output is then garbage and the host sees
+      // SWA_ERR_TIMEOUT.
+      mbar_wait(&full[st], (uint32_t)(k / kStagesR) & 1u, p.err, abort_flag);
+      const uint8_t* kb = smem + st * S::kStage;
+      const uint8_t* vb = kb + S::kTile;
+      // ---- scores: warp w handles rows [16w, 16w+16)
+#pragma unroll
+      for (int step = 0; step < 4; ++step) {
+        const int r = warp * 16 + step * 4 + rsub;
+        float dot[NQ];
+#pragma unroll
+        for (int s = 0; s < NQ; ++s) dot[s] = 0.f;
+#pragma unroll
+        for (int hh = 0; hh < kCPL; ++hh) {
+          const uint4 w = *reinterpret_cast<const uint4*>(kb + hh * (kRows * 128) + r * 128 +
+                                                          ((t8 ^ (r & 7)) * 16));
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float k0 = bf_lo(ws[e]), k1 = bf_hi(ws[e]);
+#pragma unroll
+            for (int s = 0; s < NQ; ++s) {
+              dot[s] = fmaf(qv[s][hh * 8 + 2 * e], k0, dot[s]);
+              dot[s] = fmaf(qv[s][hh * 8 + 2 * e + 1], k1, dot[s]);
+            }
+          }
+        }
+#pragma unroll
+        for (int s = 0; s < NQ; ++s) {
+          dot[s] += __shfl_xor_sync(0xffffffffu, dot[s], 4);
+          dot[s] += __shfl_xor_sync(0xffffffffu, dot[s], 2);
+          dot[s] += __shfl_xor_sync(0xffffffffu, dot[s], 1);
+        }
+        if (t8 == 0) {
+          const int key = key0 + k * kRows + r;
+#pragma unroll
+          for (int s = 0; s < NQ; ++s) sc[r * NQ + s] = key < limit[s] ? dot[s] : -INFINITY;
+        }
+      }
+      named_sync(1, kComputeWarps * 32);
+      // ---- online softmax statistics: warp w owns slots w and w + 4
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int s = warp + 4 * u;
+        if (s < NQ) {
+          const float a0 = sc[lane * NQ + s], a1 = sc[(lane + 32) * NQ + s];
+          float mx = fmaxf(a0, a1);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          const float m_new = fmaxf(m_run[u], mx);
+          const float m_safe = m_new == -INFINITY ? 0.f : m_new;
+          const float cf = ex2_approx(m_run[u] - m_safe);
+          const float p0 = ex2_approx(a0 - m_safe), p1 = ex2_approx(a1 - m_safe);
+          pc[lane * NQ + s] = p0;
+          pc[(lane + 32) * NQ + s] = p1;
+          float sum = p0 + p1;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+          l_run[u] = l_run[u] * cf + sum;
+          m_run[u] = m_new;
+          if (lane == 0) corr_s[s] = cf;
+        }
+      }
+      named_sync(1, kComputeWarps * 32);
+      // ---- O += P V: thread owns 8 columns of the value row for all slots
+#pragma unroll
+      for (int s = 0; s < NQ; ++s) {
+        const float cf = corr_s[s];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[s][e] *= cf;
+      }
+      const int hh = pv_chunk / 8, c8 = pv_chunk % 8;
+#pragma unroll 4
+      for (int r = pv_rg; r < kRows; r += kRG) {
+        const uint4 w = *reinterpret_cast<const uint4*>(vb + hh * (kRows * 128) + r * 128 +
+                                                        ((c8 ^ (r & 7)) * 16));
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+        float vv[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          vv[2 * e] = bf_lo(ws[e]);
+          vv[2 * e + 1] = bf_hi(ws[e]);
+        }
+#pragma unroll
+        for (int s = 0; s < NQ; ++s) {
+          const float pr = pc[r * NQ + s];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[s][e] = fmaf(pr, vv[e], acc[s][e]);
+        }
+      }
+      mbar_arrive(&empty[st]);
+    }
+  }
+  __syncthreads();  // every stage consumed: the ring can be reused below
+
+  // ---- reduce the row groups' partial sums: red[rg][slot][D]
+  float* red = reinterpret_cast<float*>(smem);
+  if (warp < kComputeWarps) {
+    const int pv_chunk = threadIdx.x % kLanesPV;
+    const int pv_rg = threadIdx.x / kLanesPV;
+#pragma unroll
+    for (int s = 0; s < NQ; ++s)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red[(pv_rg * NQ + s) * D + pv_chunk * 8 + e] = acc[s][e];
+    if (lane == 0) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int s = warp + 4 * u;
+        if (s < NQ) {
+          sc[s] = m_run[u];
+          sc[NQ + s] = l_run[u];
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  const size_t part = (size_t)gi * p.nsplit + split;
+  if (p.nsplit == 1) {
+    // single chunk: finish in place
+    for (int idx = threadIdx.x; idx < NQ * D; idx += blockDim.x) {
+      const int s = idx / D, dd = idx % D;
+      if (qoff[s] < 0) continue;
+      float o = 0.f;
+      for (int rg = 0; rg < kRG; ++rg) o += red[(rg * NQ + s) * D + dd];
+      const float l = sc[NQ + s];
+      p.out[qoff[s] + dd] = __bfloat16_as_ushort(__float2bfloat16_rn(o / l));
+    }
+    if (p.lse && threadIdx.x < NQ && qoff[threadIdx.x] >= 0) {
+      const int s = threadIdx.x;
+      const float lv = (sc[s] + __log2f(sc[NQ + s])) * 0.69314718055994531f;
+      const long row = qoff[s] / D;  // decode: b*H + h; global: (b*N + i)*H + h
+      long li;
+      if (p.mode == 0) li = row;
+      else {
+        const int h = (int)(row % p.H);
+        const long bi = row / p.H;
+        li = ((bi / p.N) * p.H + h) * p.N + (bi % p.N);
+      }
+      p.lse[li] = lv;
+    }
+    return;
+  }
+  for (int idx = threadIdx.x; idx < NQ * D; idx += blockDim.x) {
+    const int s = idx / D, dd = idx % D;
+    float o = 0.f;
+    for (int rg = 0; rg < kRG; ++rg) o += red[(rg * NQ + s) * D + dd];
+    p.ws_o[part * NQ * D + idx] = o;
+  }
+  if (threadIdx.x < NQ) {
+    p.ws_ml[(part * NQ + threadIdx.x) * 2] = sc[threadIdx.x];
+    p.ws_ml[(part * NQ + threadIdx.x) * 2 + 1] = sc[NQ + threadIdx.x];
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int ticket = atomicAdd(&p.cnt[gi], 1);
+    *last_flag = ticket == p.nsplit - 1;
+  }
+  __syncthreads();
+  if (!*last_flag) return;
+  __threadfence();
+  // ---- last chunk of this query set: merge all chunks
+  const size_t base = (size_t)gi * p.nsplit;
+  float* Ms = sc;          // [NQ] global max
+  float* Ls = sc + NQ;     // [NQ] merged denominator
+  if (threadIdx.x < NQ) {
+    const int s = threadIdx.x;
+    float M = -INFINITY;
+    for (int sp = 0; sp < p.nsplit; ++sp) M = fmaxf(M, __ldcg(&p.ws_ml[((base + sp) * NQ + s) * 2]));
+    const float Msafe = M == -INFINITY ? 0.f : M;
+    float L = 0.f;
+    for (int sp = 0; sp < p.nsplit; ++sp) {
+      const float m = __ldcg(&p.ws_ml[((base + sp) * NQ + s) * 2]);
+      L += __ldcg(&p.ws_ml[((base + sp) * NQ + s) * 2 + 1]) * ex2_approx(m - Msafe);
+    }
+    Ms[s] = Msafe;
+    Ls[s] = L;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < NQ * D; idx += blockDim.x) {
+    const int s = idx / D, dd = idx % D;
+    if (qoff[s] < 0) continue;
+    float o = 0.f;
+    for (int sp = 0; sp < p.nsplit; ++sp) {
+      const float m = __ldcg(&p.ws_ml[((base + sp) * NQ + s) * 2]);
+      o += __ldcg(&p.ws_o[(base + sp) * NQ * D + idx]) * ex2_approx(m - Ms[s]);
+    }
+    p.out[qoff[s] + dd] = __bfloat16_as_ushort(__float2bfloat16_rn(o / Ls[s]));
+  }
+  if (p.lse && threadIdx.x < NQ && qoff[threadIdx.x] >= 0) {
+    const int s = threadIdx.x;
+    const float lv = (Ms[s] + __log2f(Ls[s])) * 0.69314718055994531f;
+    const long row = qoff[s] / D;
+    long li;
+    if (p.mode == 0) li = row;
+    else {
+      const int h = (int)(row % p.H);
+      const long bi = row / p.H;
+      li = ((bi / p.N) * p.H + h) * p.N + (bi % p.N);
+    }
+    p.lse[li] = lv;
+  }
+  if (threadIdx.x == 0) p.cnt[gi] = 0;  // ready for the next call
+}
+
+// ------------------------------------------------------------ workspaces
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+constexpr int kMaxDev = 64;
+Workspace g_ws[kMaxDev][2];  // [device][0: decode, 1: global rows]
+std::mutex g_ws_mu;
+
+// Returns a workspace of at least `bytes`; the first `zero_bytes` are zero
+// (split counters, which every merge resets to zero after use).
+void* get_workspace(int which, size_t bytes, size_t zero_bytes, cudaStream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  Workspace& w = g_ws[dev][which];
+  if (w.bytes < bytes) {
+    if (w.ptr) {
+      cudaStreamSynchronize(stream);
+      cudaFree(w.ptr);
+      w.ptr = nullptr;
+      w.bytes = 0;
+    }
+    void* p = nullptr;
+    if (cudaMalloc(&p, bytes) != cudaSuccess) return nullptr;
+    if (cudaMemsetAsync(p, 0, zero_bytes, stream) != cudaSuccess) {
+      cudaFree(p);
+      return nullptr;
+    }
+    w.ptr = p;
+    w.bytes = bytes;
+  }
+  return w.ptr;
+}
+
+template <int D, int NQ>
+int launch_rows(RowParams& p, int nsets, cudaStream_t stream) {
+  using S = RSmem<D, NQ>;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(swa_rowattn_kernel<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             S::kAlloc) != cudaSuccess)
+      return SWA_ERR_CUDA;
+    attr = true;
+  }
+  dim3 grid(p.nsplit, nsets);
+  swa_rowattn_kernel<D, NQ><<<grid, kThreadsR, S::kAlloc, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
+template <int D>
+int dispatch_nq(RowParams& p, int nq, int nsets, cudaStream_t stream) {
+  switch (nq) {
+    case 1: return launch_rows<D, 1>(p, nsets, stream);
+    case 2: return launch_rows<D, 2>(p, nsets, stream);
+    case 4: return launch_rows<D, 4>(p, nsets, stream);
+    case 8: return launch_rows<D, 8>(p, nsets, stream);
+    default: return SWA_ERR_UNSUPPORTED;
+  }
+}
+
+int pow2_at_least(int x) {
+  int r = 1;
+  while (r < x) r <<= 1;
+  return r;
+}
+
+int encode_kv(CUtensorMap* m, const void* base, int D, int Hkv, int rows, int B) {
+  const uint64_t dims[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)rows, (uint64_t)B};
+  const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2, (uint64_t)rows * Hkv * D * 2};
+  const uint32_t box[4] = {64, 1, (uint32_t)kRows, 1};
+  return encode_tiled(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                      strides, box, CU_TENSOR_MAP_SWIZZLE_128B) == CUDA_SUCCESS
+             ? SWA_OK
+             : SWA_ERR_CUDA;
+}
+
+int run(RowParams& p, int D, int nq, int nsets, int which, cudaStream_t stream) {
+  const size_t cnt_bytes = ((size_t)nsets * 4 + 255) & ~size_t(255);
+  if (p.nsplit > 1) {
+    const size_t o_bytes = (size_t)nsets * p.nsplit * nq * D * 4;
+    const size_t ml_bytes = (size_t)nsets * p.nsplit * nq * 2 * 4;
+    uint8_t* ws = static_cast<uint8_t*>(
+        get_workspace(which, cnt_bytes + o_bytes + ml_bytes, cnt_bytes, stream));
+    if (!ws) return SWA_ERR_NOMEM;
+    p.cnt = reinterpret_cast<int*>(ws);
+    p.ws_o = reinterpret_cast<float*>(ws + cnt_bytes);
+    p.ws_ml = reinterpret_cast<float*>(ws + cnt_bytes + o_bytes);
+  }
+  if (D == 128) return dispatch_nq<128>(p, nq, nsets, stream);
+  if (D == 64) return dispatch_nq<64>(p, nq, nsets, stream);
+  return SWA_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
+int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* out, float* lse,
+                  const int64_t* pos, int B, int H, int Hkv, int D, int W, float scale,
+                  cudaStream_t stream) {
+  RowParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (encode_kv(&p.tmK, k_ring, D, Hkv, W, B) != SWA_OK ||
+      encode_kv(&p.tmV, v_ring, D, Hkv, W, B) != SWA_OK)
+    return SWA_ERR_CUDA;
+  p.q = static_cast<const uint16_t*>(q);
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.pos = pos;
+  p.err = device_error_word();
+  if (!p.err) return SWA_ERR_CUDA;
+  p.mode = 0;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.W = W;
+  p.grp = H / Hkv;
+  p.rows_per_cta = 1;
+  p.nrowchunks = 1;
+  p.chunk = 512;
+  p.nsplit = (W + p.chunk - 1) / p.chunk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int nq = pow2_at_least(p.grp);
+  return run(p, D, nq, B * Hkv, 0, stream);
+}
+
+int launch_global_rows(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int H, int Hkv, int N, int D, bool causal, const int32_t* G,
+                       int ng, float scale, cudaStream_t stream) {
+  RowParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (encode_kv(&p.tmK, k, D, Hkv, N, B) != SWA_OK || encode_kv(&p.tmV, v, D, Hkv, N, B) != SWA_OK)
+    return SWA_ERR_CUDA;
+  p.q = static_cast<const uint16_t*>(q);
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.G = G;
+  p.err = device_error_word();
+  if (!p.err) return SWA_ERR_CUDA;
+  p.mode = 1;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.grp = H / Hkv;
+  p.ng = ng;
+  p.causal = causal ? 1 : 0;
+  const int nq = 8;
+  p.rows_per_cta = nq / p.grp;
+  p.nrowchunks = (ng + p.rows_per_cta - 1) / p.rows_per_cta;
+  p.chunk = 512;
+  p.nsplit = (N + p.chunk - 1) / p.chunk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  return run(p, D, nq, B * Hkv * p.nrowchunks, 1, stream);
+}
+
+void release_workspaces() {
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  for (int d = 0; d < kMaxDev; ++d)
+    for (int w = 0; w < 2; ++w)
+      if (g_ws[d][w].ptr) {
+        int cur = 0;
+        cudaGetDevice(&cur);
+        cudaSetDevice(d);
+        cudaDeviceSynchronize();
+        cudaFree(g_ws[d][w].ptr);
+        cudaSetDevice(cur);
+        g_ws[d][w].ptr = nullptr;
+        g_ws[d][w].bytes = 0;
+      }
+}
+
+}  // namespace swa

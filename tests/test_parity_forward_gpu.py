@@ -1,0 +1,157 @@
+"""Forward parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small and shrunken cases are compared on every element; the full-size
+workloads on a seeded sample of rows (edges included) that the oracle
+computes one by one.  Tolerances: fp32 max abs 1e-4; bf16 max abs 2e-2 and
+mean abs 2e-3; lse abs 1e-3.  Every output lives inside NaN guard bands that
+must survive the launch.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import (BF16_MAX_ABS, BF16_MEAN_ABS, F32_MAX_ABS, LSE_ABS, check_guards, compare,
+                      guarded, sample_rows)
+from sliding_window_attention_fwd_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def swa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import sliding_window_attention_fwd_b200 as m
+    return m
+
+
+def run_forward(swa, q, k, v, L, R, d=1, bs=0, G=None, scale=0.0, f32=False):
+    B, N, H, D = q.shape
+    dt = torch.float32 if f32 else torch.bfloat16
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    obuf, out = guarded((B, N, H, D), dt)
+    lbuf, lse = guarded((B, H, N), torch.float32)
+    Gd = None if G is None or len(G) == 0 else torch.as_tensor(G, dtype=torch.int32).cuda()
+    if f32:
+        swa.swa_forward_f32(qd, kd, vd, out, lse, L, R, d, bs, Gd, scale)
+    elif bs:
+        swa.swa_forward_ex(qd, kd, vd, out, lse, L, R, d, bs, Gd, scale)
+    else:
+        swa.swa_forward(qd, kd, vd, out, lse, L, R, d, Gd, scale)
+    torch.cuda.synchronize()
+    assert swa.swa_device_error() == 0
+    check_guards(obuf)
+    check_guards(lbuf)
+    return out.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def full_check(swa, cfg_or_args, f32=False):
+    q, k, v, L, R, d, bs, G, scale = cfg_or_args
+    out, lse = run_forward(swa, q, k, v, L, R, d, bs, G, scale, f32)
+    ref_o, ref_l = oracle.forward(q, k, v, L, R, d, bs, [] if G is None else G, scale)
+    if f32:
+        compare(out, ref_o, F32_MAX_ABS, what="out")
+        compare(lse, ref_l, F32_MAX_ABS, what="lse")
+    else:
+        compare(out, ref_o, BF16_MAX_ABS, BF16_MEAN_ABS, what="out")
+        compare(lse, ref_l, LSE_ABS, what="lse")
+
+
+def rand_case(B, N, H, Hkv, D, seed, dtype=torch.bfloat16):
+    q = inputs.normal((B, N, H, D), seed, 0, dtype)
+    k = inputs.normal((B, N, Hkv, D), seed, 1, dtype)
+    v = inputs.normal((B, N, Hkv, D), seed, 2, dtype)
+    return q, k, v
+
+
+# ------------------------------------------------------------------ fp32 path
+def test_config_tiny_bidirectional_fp32(swa):
+    cfg = inputs.CONFIGS["tiny_bidir_fp32"]
+    q, k, v, G = inputs.forward_inputs(cfg)
+    full_check(swa, (q, k, v, cfg.win_left, cfg.win_right, 1, 0, None, cfg.scale), f32=True)
+
+
+@pytest.mark.parametrize("case", [
+    # (B, N, H, Hkv, D, L, R, d, bs, G)
+    (1, 100, 4, 2, 64, 10, 0, 1, 0, None),
+    (2, 77, 2, 1, 32, 5, 5, 3, 0, None),
+    (1, 130, 2, 2, 96, 64, 64, 2, 16, None),
+    (1, 90, 2, 2, 128, 4, 4, 1, 0, [0, 30, 89]),
+    (1, 90, 2, 2, 64, 6, 0, 1, 0, [0, 45]),
+    (1, 1, 1, 1, 64, 3, 3, 1, 0, None),
+    (1, 50, 2, 1, 64, -1, -1, 1, 0, None),
+])
+def test_fp32_variants(swa, case):
+    B, N, H, Hkv, D, L, R, d, bs, G = case
+    q, k, v = rand_case(B, N, H, Hkv, D, 31, torch.float32)
+    full_check(swa, (q, k, v, L, R, d, bs, G, 0.0), f32=True)
+
+
+# ------------------------------------------------------------ bf16 tcgen05 path
+SMALL_BF16 = [
+    # (B, N, H, Hkv, D, L, R, d, bs, G)
+    (1, 128, 1, 1, 128, 127, 0, 1, 0, None),       # one full causal tile
+    (1, 256, 2, 1, 128, 300, 0, 1, 0, None),       # window longer than N
+    (1, 1000, 8, 2, 128, 300, 0, 1, 0, None),      # ragged tail, GQA 4
+    (1, 129, 2, 2, 64, 64, 64, 1, 0, None),        # tile + 1
+    (1, 127, 2, 2, 64, 16, 16, 1, 0, None),        # tile - 1
+    (1, 1, 1, 1, 128, 5, 0, 1, 0, None),           # N = 1
+    (2, 300, 2, 2, 64, 0, 0, 1, 0, None),          # one-key window
+    (1, 400, 2, 1, 128, -1, -1, 1, 0, None),       # unbounded = full attention
+    (1, 500, 2, 2, 64, -1, 0, 1, 0, None),         # unbounded causal
+    (2, 700, 3, 3, 64, 40, 40, 1, 0, [0, 128, 256, 384, 512, 640]),
+    (1, 600, 4, 2, 128, 100, 0, 1, 0, [0, 7, 300]),  # causal + globals
+    (1, 1003, 2, 2, 64, 50, 50, 3, 0, None),       # dilated, N mod d != 0
+    (1, 2000, 2, 2, 128, 20, 30, 16, 0, None),     # d > 8 classes per launch
+    (1, 1344, 2, 1, 64, 128, 128, 4, 64, None),    # block-level dilation
+    (1, 1000, 2, 2, 64, 128, 0, 2, 64, [3, 500]),  # block, causal, ragged, globals
+]
+
+
+@pytest.mark.parametrize("case", SMALL_BF16)
+def test_bf16_small(swa, case):
+    B, N, H, Hkv, D, L, R, d, bs, G = case
+    q, k, v = rand_case(B, N, H, Hkv, D, 7)
+    full_check(swa, (q, k, v, L, R, d, bs, G, 0.0))
+
+
+@pytest.mark.parametrize("name", ["small_causal", "small_global", "small_dilated", "small_block"])
+def test_bf16_shrunken_configs(swa, name):
+    cfg = inputs.CONFIGS[name]
+    q, k, v, G = inputs.forward_inputs(cfg)
+    full_check(swa, (q, k, v, cfg.win_left, cfg.win_right, cfg.dilation, cfg.dilation_block,
+                     G.numpy() if len(G) else None, cfg.scale))
+
+
+def test_bf16_large_scores_rescale(swa):
+    """Scores that grow along the row force the lazy max rescaling path."""
+    B, N, H, D = 1, 1024, 2, 128
+    q, k, v = rand_case(B, N, H, H, D, 11)
+    ramp = torch.linspace(0.1, 4.0, N).view(1, N, 1, 1)
+    k = (k.float() * ramp).to(torch.bfloat16)
+    q = (q.float() * 2.0).to(torch.bfloat16)
+    full_check(swa, (q, k, v, 900, 0, 1, 0, None, 0.0))
+
+
+# ------------------------------------------------------- full-size workloads
+@pytest.mark.parametrize("name", ["mistral_causal_prefill", "longformer_global", "dilated_token",
+                                  "dilated_block"])
+def test_full_size_sampled(swa, name):
+    cfg = inputs.CONFIGS[name]
+    q, k, v, G = inputs.forward_inputs(cfg)
+    Gn = G.numpy() if len(G) else None
+    out, lse = run_forward(swa, q, k, v, cfg.win_left, cfg.win_right, cfg.dilation,
+                           cfg.dilation_block, Gn, cfg.scale)
+    N = cfg.N
+    edges = [0, 1, 127, 128, 129, 511, 512, 513, 4095, 4096, N // 2, N - 129, N - 128, N - 2,
+             N - 1]
+    rows = sample_rows(cfg.B, cfg.H, N, 1500, seed=5, extra_i=edges)
+    ref_o, ref_l = oracle.forward(q, k, v, cfg.win_left, cfg.win_right, cfg.dilation,
+                                  cfg.dilation_block, [] if Gn is None else Gn, cfg.scale,
+                                  rows=rows)
+    got_o = out[rows[:, 0], rows[:, 2], rows[:, 1]]
+    got_l = lse[rows[:, 0], rows[:, 1], rows[:, 2]]
+    compare(got_o, ref_o, BF16_MAX_ABS, BF16_MEAN_ABS, what=f"{name} out")
+    compare(got_l, ref_l, LSE_ABS, what=f"{name} lse")
+    assert np.isfinite(out).all()
