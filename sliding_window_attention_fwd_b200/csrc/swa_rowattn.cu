@@ -409,38 +409,58 @@ __global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_
 }
 
 // ------------------------------------------------------------ workspaces
+// Per device and per user (0: decode, 1: global rows): split counters and
+// split partials in separate buffers.  Every merge resets its counter to
+// zero, so between complete calls all counters are zero; the counter buffer
+// is zeroed whenever it is (re)allocated and is never overlapped by the
+// partials, whatever the number of query sets of later calls.
 struct Workspace {
-  void* ptr = nullptr;
-  size_t bytes = 0;
+  void* cnt = nullptr;
+  size_t cnt_bytes = 0;
+  void* part = nullptr;
+  size_t part_bytes = 0;
 };
 constexpr int kMaxDev = 64;
-Workspace g_ws[kMaxDev][2];  // [device][0: decode, 1: global rows]
+Workspace g_ws[kMaxDev][2];
 std::mutex g_ws_mu;
 
-// Returns a workspace of at least `bytes`; the first `zero_bytes` are zero
-// (split counters, which every merge resets to zero after use).
-void* get_workspace(int which, size_t bytes, size_t zero_bytes, cudaStream_t stream) {
+bool get_workspace(int which, size_t cnt_bytes, size_t part_bytes, cudaStream_t stream,
+                   int** cnt, void** part) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
   std::lock_guard<std::mutex> lk(g_ws_mu);
   Workspace& w = g_ws[dev][which];
-  if (w.bytes < bytes) {
-    if (w.ptr) {
+  if (w.cnt_bytes < cnt_bytes) {
+    if (w.cnt) {
       cudaStreamSynchronize(stream);
-      cudaFree(w.ptr);
-      w.ptr = nullptr;
-      w.bytes = 0;
+      cudaFree(w.cnt);
+      w.cnt = nullptr;
+      w.cnt_bytes = 0;
     }
     void* p = nullptr;
-    if (cudaMalloc(&p, bytes) != cudaSuccess) return nullptr;
-    if (cudaMemsetAsync(p, 0, zero_bytes, stream) != cudaSuccess) {
+    if (cudaMalloc(&p, cnt_bytes) != cudaSuccess) return false;
+    if (cudaMemsetAsync(p, 0, cnt_bytes, stream) != cudaSuccess) {
       cudaFree(p);
-      return nullptr;
+      return false;
     }
-    w.ptr = p;
-    w.bytes = bytes;
+    w.cnt = p;
+    w.cnt_bytes = cnt_bytes;
   }
-  return w.ptr;
+  if (w.part_bytes < part_bytes) {
+    if (w.part) {
+      cudaStreamSynchronize(stream);
+      cudaFree(w.part);
+      w.part = nullptr;
+      w.part_bytes = 0;
+    }
+    void* p = nullptr;
+    if (cudaMalloc(&p, part_bytes) != cudaSuccess) return false;
+    w.part = p;
+    w.part_bytes = part_bytes;
+  }
+  *cnt = static_cast<int*>(w.cnt);
+  *part = w.part;
+  return true;
 }
 
 template <int D, int NQ>
@@ -486,16 +506,17 @@ int encode_kv(CUtensorMap* m, const void* base, int D, int Hkv, int rows, int B)
 }
 
 int run(RowParams& p, int D, int nq, int nsets, int which, cudaStream_t stream) {
-  const size_t cnt_bytes = ((size_t)nsets * 4 + 255) & ~size_t(255);
   if (p.nsplit > 1) {
+    const size_t cnt_bytes = ((size_t)nsets * 4 + 255) & ~size_t(255);
     const size_t o_bytes = (size_t)nsets * p.nsplit * nq * D * 4;
     const size_t ml_bytes = (size_t)nsets * p.nsplit * nq * 2 * 4;
-    uint8_t* ws = static_cast<uint8_t*>(
-        get_workspace(which, cnt_bytes + o_bytes + ml_bytes, cnt_bytes, stream));
-    if (!ws) return SWA_ERR_NOMEM;
-    p.cnt = reinterpret_cast<int*>(ws);
-    p.ws_o = reinterpret_cast<float*>(ws + cnt_bytes);
-    p.ws_ml = reinterpret_cast<float*>(ws + cnt_bytes + o_bytes);
+    int* cnt = nullptr;
+    void* part = nullptr;
+    if (!get_workspace(which, cnt_bytes, o_bytes + ml_bytes, stream, &cnt, &part))
+      return SWA_ERR_NOMEM;
+    p.cnt = cnt;
+    p.ws_o = static_cast<float*>(part);
+    p.ws_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(part) + o_bytes);
   }
   if (D == 128) return dispatch_nq<128>(p, nq, nsets, stream);
   if (D == 64) return dispatch_nq<64>(p, nq, nsets, stream);
@@ -566,17 +587,19 @@ int launch_global_rows(const void* q, const void* k, const void* v, void* out, f
 void release_workspaces() {
   std::lock_guard<std::mutex> lk(g_ws_mu);
   for (int d = 0; d < kMaxDev; ++d)
-    for (int w = 0; w < 2; ++w)
-      if (g_ws[d][w].ptr) {
-        int cur = 0;
-        cudaGetDevice(&cur);
-        cudaSetDevice(d);
-        cudaDeviceSynchronize();
-        cudaFree(g_ws[d][w].ptr);
-        cudaSetDevice(cur);
-        g_ws[d][w].ptr = nullptr;
-        g_ws[d][w].bytes = 0;
-      }
+    for (int w = 0; w < 2; ++w) {
+      Workspace& ws = g_ws[d][w];
+      if (!ws.cnt && !ws.part) continue;
+      int cur = 0;
+      cudaGetDevice(&cur);
+      cudaSetDevice(d);
+      cudaDeviceSynchronize();
+      if (ws.cnt) cudaFree(ws.cnt);
+      if (ws.part) cudaFree(ws.part);
+      cudaSetDevice(cur);
+      ws = Workspace();
+    }
 }
+
 
 }  // namespace swa

@@ -78,3 +78,17 @@ def test_ring_decode_wrapped_equals_forward(swa):
     out_f = swa.swa_forward(qs.cuda(), seq.cuda(), vseq.cuda(), win_left=W - 1, win_right=0)
     torch.cuda.synchronize()
     np.testing.assert_allclose(out_d[0], out_f[0, p].float().cpu().numpy(), atol=2e-2)
+
+
+def test_workspace_reuse_across_sizes(swa):
+    """Calls with fewer and then more query sets reuse one workspace: the
+    split counters of the big call must still start at zero afterwards."""
+    big = inputs.decode_inputs(inputs.DECODE_CONFIGS["ring_decode"])
+    small = inputs.decode_inputs(inputs.DECODE_CONFIGS["small_ring_partial"])
+    check(swa, *big)
+    check(swa, *small)
+    q = inputs.normal((2, 8, 128), 17, 0)
+    kr = inputs.normal((2, 2048, 4, 128), 17, 1)
+    vr = inputs.normal((2, 2048, 4, 128), 17, 2)
+    check(swa, q, kr, vr, torch.tensor([5000, 100], dtype=torch.int64))
+    check(swa, *big)
