@@ -54,6 +54,7 @@
 #ifndef SWA_H_
 #define SWA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -140,6 +141,43 @@ SWA_API int swa_decode(const void* q, const void* k_ring, const void* v_ring,
 SWA_API int swa_decode_ex(const void* q, const void* k_ring, const void* v_ring,
                           void* out, float* lse, const int64_t* pos, int B, int H,
                           int Hkv, int D, int W, float scale, void* stream);
+
+/*
+ * swa_decode_noalloc -- swa_decode for callers that must not have the
+ * library allocate device memory.  (No counterpart on the method's pages:
+ * this is a deployment variant of swa_decode, same arguments, same result.)
+ *
+ * Who needs it: callers that route every byte of device memory through
+ * their own pre-sized pool or arena (a serving engine with a fixed memory
+ * budget, where a library cudaMalloc would break the budget or fragment the
+ * pool), and callers on latency-critical paths that cannot accept the
+ * device-wide synchronisation a cudaMalloc may imply.  swa_decode keeps its
+ * split partials in a workspace it cudaMalloc's on first use; this call
+ * instead uses a fixed array compiled into the library
+ * (swa_decode_noalloc_scratch_bytes() bytes, 16 MiB), which every GPU that
+ * loads the library holds until the process exits.  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.  The caller still passes inputs and
+ * outputs.
+ *
+ * Limits and behaviour:
+ *  - a problem whose split partials need more than the array holds (about
+ *    B * Hkv * ceil(W / 512) * pow2(H/Hkv) * (D + 2) * 4 bytes) returns
+ *    SWA_ERR_UNSUPPORTED and launches nothing;
+ *  - the first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before
+ *    any stream capture;
+ *  - every call on a device shares the one array, which keeps the last
+ *    call's contents (the call clears the part that must start at zero on
+ *    `stream`): calls that overlap on the GPU, e.g. on two streams, race and
+ *    must be serialised by the caller.
+ */
+SWA_API int swa_decode_noalloc(const void* q, const void* k_ring, const void* v_ring,
+                               void* out, const int64_t* pos, int B, int H, int Hkv,
+                               int D, int W, void* stream);
+
+/* swa_decode_noalloc_scratch_bytes -- size of swa_decode_noalloc's fixed
+   device array, per GPU. */
+SWA_API size_t swa_decode_noalloc_scratch_bytes(void);
 
 /*
  * swa_device_error -- synchronises `stream`, then reports (and clears) a

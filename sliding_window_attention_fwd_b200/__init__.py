@@ -13,6 +13,8 @@ from .binding import (  # noqa: F401
     library_path,
     swa_decode,
     swa_decode_ex,
+    swa_decode_noalloc,
+    swa_decode_noalloc_scratch_bytes,
     swa_device_error,
     swa_forward,
     swa_forward_ex,

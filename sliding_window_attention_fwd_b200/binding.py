@@ -26,6 +26,10 @@ _lib.swa_forward_ex.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, 
 _lib.swa_forward_f32.argtypes = _lib.swa_forward_ex.argtypes
 _lib.swa_decode.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
 _lib.swa_decode_ex.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
+_lib.swa_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
+_lib.swa_decode_noalloc.restype = _I
+_lib.swa_decode_noalloc_scratch_bytes.argtypes = []
+_lib.swa_decode_noalloc_scratch_bytes.restype = ctypes.c_size_t
 _lib.swa_device_error.argtypes = [_P]
 _lib.swa_selftest_timeout.argtypes = [_I, _P]
 _lib.swa_schedule.argtypes = [_I, _I, _I, _I, _I, _P, _I]
@@ -166,6 +170,24 @@ def swa_decode_ex(q, k_ring, v_ring, pos, out=None, lse=None, scale=0.0, stream=
                               _ptr(pos), B, H, Hkv, D, W, float(scale), _stream(stream)),
            "swa_decode_ex")
     return out
+
+
+def swa_decode_noalloc(q, k_ring, v_ring, pos, out, stream=None):
+    """swa_decode without any device allocation by the library (C:
+    swa_decode_noalloc): for callers whose device memory is a fixed pool, or
+    whose hot loop cannot take a cudaMalloc.  Its split partials live in a
+    fixed array inside the library, shared by all calls on a device, so calls
+    must not overlap on the GPU.  `out` must be given (nothing is allocated
+    here either)."""
+    B, H, Hkv, D, W, out = _dec_common(q, k_ring, v_ring, out, pos)
+    _check(_lib.swa_decode_noalloc(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(out), _ptr(pos),
+                                   B, H, Hkv, D, W, _stream(stream)), "swa_decode_noalloc")
+    return out
+
+
+def swa_decode_noalloc_scratch_bytes() -> int:
+    """Bytes of the fixed device array swa_decode_noalloc uses (per GPU)."""
+    return int(_lib.swa_decode_noalloc_scratch_bytes())
 
 
 def swa_device_error(stream=None) -> int:

@@ -189,6 +189,24 @@ SWA_API int swa_decode(const void* q, const void* k_ring, const void* v_ring, vo
   return swa_decode_ex(q, k_ring, v_ring, out, nullptr, pos, B, H, Hkv, D, W, 0.f, stream);
 }
 
+SWA_API int swa_decode_noalloc(const void* q, const void* k_ring, const void* v_ring, void* out,
+                               const int64_t* pos, int B, int H, int Hkv, int D, int W,
+                               void* stream) {
+  if (B < 0 || H <= 0 || Hkv <= 0 || D <= 0 || W <= 0) return SWA_ERR_ARG;
+  if (H % Hkv != 0) return SWA_ERR_ARG;
+  if (!q || !k_ring || !v_ring || !out || !pos) return SWA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_ring) || !aligned16(v_ring) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(pos) & 7u))
+    return SWA_ERR_ALIGN;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (H / Hkv > 8) return SWA_ERR_UNSUPPORTED;
+  if (B == 0) return SWA_OK;
+  return launch_decode_noalloc(q, k_ring, v_ring, out, pos, B, H, Hkv, D, W,
+                               resolve_scale(0.f, D), static_cast<cudaStream_t>(stream));
+}
+
+SWA_API size_t swa_decode_noalloc_scratch_bytes(void) { return noalloc_scratch_bytes(); }
+
 SWA_API int swa_device_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return SWA_ERR_CUDA;

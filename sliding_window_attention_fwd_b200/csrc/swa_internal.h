@@ -36,6 +36,13 @@ int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* o
                   float* lse, const int64_t* pos, int B, int H, int Hkv, int D, int W,
                   float scale, cudaStream_t stream);
 
+// Decode with its split partials in a fixed file-scope device array (no
+// allocation by the library).
+int launch_decode_noalloc(const void* q, const void* k_ring, const void* v_ring, void* out,
+                          const int64_t* pos, int B, int H, int Hkv, int D, int W,
+                          float scale, cudaStream_t stream);
+size_t noalloc_scratch_bytes();
+
 int launch_timeout_selftest(int limit_us, cudaStream_t stream);
 
 void release_workspaces();

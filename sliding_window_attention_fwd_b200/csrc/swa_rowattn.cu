@@ -602,4 +602,95 @@ void release_workspaces() {
 }
 
 
+// ------------------------------------------------------------------------
+// Decode without any device allocation by the library.
+//
+// The ordinary swa_decode path keeps its split partials in a workspace that
+// the library cudaMalloc's on first use.  Some callers cannot allow that:
+// serving engines that hand every byte of device memory to their own
+// pre-sized pool or arena (a stray cudaMalloc breaks their budget and
+// fragments the pool), and latency-critical loops that cannot afford the
+// implicit device-wide synchronisation cudaMalloc may cause.  For them the
+// partials live in this fixed file-scope array instead.  Every GPU that
+// loads the library holds it (kNoAllocScratchBytes) until the process
+// exits, and all calls share it.
+constexpr size_t kNoAllocScratchBytes = 16u << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+void* g_noalloc_ptr[kMaxDev] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the symbol is only a stand-in, so the address is looked up once per
+// device with that device current (first call on the device).
+void* noalloc_scratch(int* status) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+    *status = SWA_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+      *status = SWA_ERR_CUDA;
+      return nullptr;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+int launch_decode_noalloc(const void* q, const void* k_ring, const void* v_ring, void* out,
+                          const int64_t* pos, int B, int H, int Hkv, int D, int W,
+                          float scale, cudaStream_t stream) {
+  RowParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const uint16_t*>(q);
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = nullptr;
+  p.pos = pos;
+  p.mode = 0;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.W = W;
+  p.grp = H / Hkv;
+  p.rows_per_cta = 1;
+  p.nrowchunks = 1;
+  p.chunk = 512;
+  p.nsplit = (W + p.chunk - 1) / p.chunk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int nq = pow2_at_least(p.grp);
+  const int nsets = B * Hkv;
+  const size_t cnt_bytes = ((size_t)nsets * 4 + 255) & ~size_t(255);
+  const size_t o_bytes = (size_t)nsets * p.nsplit * nq * D * 4;
+  const size_t ml_bytes = (size_t)nsets * p.nsplit * nq * 2 * 4;
+  if (p.nsplit > 1 && cnt_bytes + o_bytes + ml_bytes > kNoAllocScratchBytes)
+    return SWA_ERR_UNSUPPORTED;  // problem needs more scratch than the array holds
+  int status = SWA_OK;
+  uint8_t* ws = static_cast<uint8_t*>(noalloc_scratch(&status));
+  if (!ws) return status;
+  p.err = device_error_word();
+  if (!p.err) return SWA_ERR_CUDA;
+  if (encode_kv(&p.tmK, k_ring, D, Hkv, W, B) != SWA_OK ||
+      encode_kv(&p.tmV, v_ring, D, Hkv, W, B) != SWA_OK)
+    return SWA_ERR_CUDA;
+  if (p.nsplit > 1) {
+    // The array keeps whatever the last call left; the split counters must
+    // start at zero, so clear them on the caller's stream.
+    if (cudaMemsetAsync(ws, 0, cnt_bytes, stream) != cudaSuccess) return SWA_ERR_CUDA;
+    p.cnt = reinterpret_cast<int*>(ws);
+    p.ws_o = reinterpret_cast<float*>(ws + cnt_bytes);
+    p.ws_ml = reinterpret_cast<float*>(ws + cnt_bytes + o_bytes);
+  }
+  if (D == 128) return dispatch_nq<128>(p, nq, nsets, stream);
+  if (D == 64) return dispatch_nq<64>(p, nq, nsets, stream);
+  return SWA_ERR_UNSUPPORTED;
+}
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
 }  // namespace swa
