@@ -1,29 +1,36 @@
 // swa_fwd_sm100.cu -- fused bf16 sliding-window attention forward for B200.
 //
-// One CTA computes one 128-row query tile of one (batch, head, residue
-// class).  Only the key tiles the band-aware scheduler lists are visited
-// (page "别再只加Mask了", §1: out-of-window pairs are skipped, not masked;
-// "空洞滑窗机制" §四: dilation is handled on dense tiles of whole blocks),
-// plus, when global tokens exist, tiles of gathered global keys
-// (aiqz.cc page, "全局注意力token").
+// A CTA computes the same 128-row query tile of one (batch, residue class)
+// for NSLOT (1 or 2) query heads.  Only the key tiles the band-aware
+// scheduler lists are visited (page "别再只加Mask了", §1: out-of-window
+// pairs are skipped, not masked; "空洞滑窗机制" §四: dilation handled on
+// dense tiles of whole blocks), followed, when global tokens exist, by
+// tiles of gathered global keys (aiqz.cc page, "全局注意力token").
 //
-// Warp roles (256 threads):
-//   warp 0     producer: TMA loads of Q once and K/V tiles into a
-//              3-stage shared-memory ring (128-byte swizzle), or a gather of
-//              global-key rows with plain loads for global tiles;
-//   warp 1     TMEM owner and MMA issuer (one thread):
-//                S_j  = Q K_j^T      tcgen05.mma, both operands in smem,
-//                                    fp32 accumulator in TMEM (two buffers);
-//                O   += P_j V_j      tcgen05.mma, P read from TMEM (bf16,
-//                                    aliasing S_j), V from smem;
-//   warps 4-7  softmax: thread t owns query row t of the tile, so the row
-//              max / row sum are thread-local (no shuffles).  Scores are
-//              masked only on tiles the scheduler marks as edge tiles.
-//              The running max is rescaled lazily: O is corrected only when
-//              the max grows by more than 2^8, otherwise the stale max is
-//              kept (the final O / l is exact either way).
-//   warps 2-3  idle after set-up.
-// Per row: out = O / l (bf16), lse = ln l + m (fp32).
+// Two query heads per CTA let the tensor core alternate between them:
+// while one softmax warpgroup turns S into P for head 0, the MMAs of head 1
+// run, and the other way round.  The two heads either share a kv head (GQA:
+// one K/V stream) or read two kv heads (two K/V streams, D = 64 only, to fit
+// shared memory).
+//
+// Warp roles (warpgroup 0 = warps 0-3; warpgroup 1 + s = softmax of slot s):
+//   warp 0     producer: TMA loads of the Q tiles once and of the K/V tiles
+//              into a shared-memory ring (128-byte swizzle); global keys are
+//              gathered with plain 16-byte loads into the same layout;
+//   warp 1     TMEM owner (512 columns) and the single MMA-issuing thread:
+//                S_s  = Q_s K^T     tcgen05.mma, operands in smem, fp32 in TMEM
+//                O_s += P_s V       tcgen05.mma, P (bf16) read from TMEM where
+//                                   it overwrote S_s, V from smem
+//              issued in the order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1);
+//   softmax    thread t of warpgroup 1+s owns query row t of slot s: row max
+//              and row sum are thread-local tree reductions, no shuffles.
+//              Element masks only on tiles the scheduler marks as edges.
+//              Scores are read from TMEM 64 columns at a time and turned into
+//              P against the current running max in the same pass (the max
+//              changes rarely); a max that grows by more than 2^8 is adopted
+//              before the next tile by rescaling O and l, and the final
+//              O / l is exact either way.
+// Per row: out = O / l (bf16), lse = m + ln l (fp32).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -39,7 +46,6 @@ namespace swa {
 namespace {
 
 constexpr int kMaxClasses = 8;   // residue classes per launch (tensor maps in params)
-constexpr int kThreads = 256;
 constexpr int kChunkBytes = kTileM * 128;  // one 64-column slice of a 128-row tile
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kTmemCols = 512;
@@ -63,68 +69,57 @@ struct FwdParams {
   float scale_log2;
 };
 
-template <int D>
-struct Smem {
-  // K/V ring depth; also sized so that exactly one CTA fits on an SM (each
-  // CTA owns all 512 TMEM columns).
-  static constexpr int kStages = D == 64 ? 4 : 3;
-  static constexpr int kTileBytes = D / 64 * kChunkBytes;  // 128 x D bf16
+template <int D, int NSLOT, int NSTREAM>
+struct Cfg {
+  static constexpr int kTile = D / 64 * kChunkBytes;        // 128 rows x D bf16
+  static constexpr int kStageBytes = 2 * NSTREAM * kTile;   // K and V of every stream
+  static constexpr int kQBytes = NSLOT * kTile;
+  static constexpr int kBudget = 224 * 1024;
+  static constexpr int kFit = (kBudget - kQBytes) / kStageBytes;
+  static constexpr int kStages = kFit > 4 ? 4 : kFit;
+  static_assert(kStages >= 2, "K/V ring needs two stages");
+  static constexpr int kThreads = 128 * (1 + NSLOT);
   static constexpr int kQ = 0;
-  static constexpr int kK = kQ + kTileBytes;
-  static constexpr int kV = kK + kStages * kTileBytes;
-  static constexpr int kBar = kV + kStages * kTileBytes;
-  // barriers: full_q, full_k[S], empty_k[S], full_v[S], empty_v[S],
-  //           s_full[2], p_full[2], o_done, o_final
-  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2;
+  static constexpr int kRing = kQ + kQBytes;
+  static constexpr int kBar = kRing + kStages * kStageBytes;
+  // full_q, full_k[S], empty_k[S], full_v[S], empty_v[S],
+  // s_full[2], p_full[2], o_done[2], o_final[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 8;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
+  static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
-__device__ __forceinline__ bool in_band_phys(int L, int R, int d, int bs, int i, int j) {
-  long diff, lo, hi;
-  if (bs > 1) {
-    diff = (long)(j / bs) - (long)(i / bs);
-    lo = -(long)(L / bs) * d;
-    hi = (long)(R / bs) * d;
-  } else {
-    diff = (long)j - (long)i;
-    lo = -(long)L * d;
-    hi = (long)R * d;
-  }
-  if (diff % d != 0) return false;
-  if (L >= 0 && diff < lo) return false;
-  if (R >= 0 && diff > hi) return false;
-  return true;
-}
-
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1) swa_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
-  using S = Smem<D>;
-  constexpr int kStages = S::kStages;
+template <int D, int NSLOT, int NSTREAM>
+__global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
+    swa_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
+  using C = Cfg<D, NSLOT, NSTREAM>;
+  constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBar);
   uint64_t* full_q = bars;
   uint64_t* full_k = bars + 1;
   uint64_t* empty_k = full_k + kStages;
   uint64_t* full_v = empty_k + kStages;
   uint64_t* empty_v = full_v + kStages;
-  uint64_t* s_full = empty_v + kStages;
+  uint64_t* s_full = empty_v + kStages;  // [slot]
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
-  uint64_t* o_final = o_done + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + S::kMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kMisc + 4);
+  uint64_t* o_final = o_done + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
 
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // ---- work item: (class, q tile, batch, head); heavy (late) tiles first.
+  // ---- work item: (class, q tile, batch, head pair); heavy (late) tiles first
+  const int npair = (p.H + NSLOT - 1) / NSLOT;
   int x = blockIdx.x;
-  const int h = x % p.H;
-  x /= p.H;
+  const int hp = x % npair;
+  x /= npair;
   const int b = x % p.B;
   x /= p.B;
   const int jt = p.qtile_prefix[p.nclass] - 1 - x;
@@ -132,7 +127,16 @@ __global__ void __launch_bounds__(kThreads, 1) swa_fwd_sm100_kernel(const __grid
   while (cl + 1 < p.nclass && p.qtile_prefix[cl + 1] <= jt) ++cl;
   const int qt = jt - p.qtile_prefix[cl];
   const int c = p.class0 + cl;
-  const int hkv = h / (p.H / p.Hkv);
+  const int grp = p.H / p.Hkv;
+  int head[NSLOT], kvh[NSLOT];
+  bool slot_ok[NSLOT];
+#pragma unroll
+  for (int s = 0; s < NSLOT; ++s) {
+    head[s] = hp * NSLOT + s;
+    slot_ok[s] = head[s] < p.H;
+    if (!slot_ok[s]) head[s] = p.H - 1;
+    kvh[s] = head[s] / grp;
+  }
   const Geometry g = make_geometry(p.N, p.L, p.R, p.d, p.bs);
   const int Mv = p.Mv[cl];
   const TileRange tr = tile_range(g, Mv, qt);
@@ -154,9 +158,9 @@ __global__ void __launch_bounds__(kThreads, 1) swa_fwd_sm100_kernel(const __grid
     for (int s = 0; s < 2; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], 128);
+      mbar_init(&o_done[s], 1);
+      mbar_init(&o_final[s], 1);
     }
-    mbar_init(o_done, 1);
-    mbar_init(o_final, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -167,221 +171,368 @@ __global__ void __launch_bounds__(kThreads, 1) swa_fwd_sm100_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  // TMEM columns: S/P buffers at [0,128) and [128,256), O at [256, 256+D)
-  auto tS = [&](int it) -> uint32_t { return tmem + (uint32_t)(it & 1) * 128u; };
-  const uint32_t tO = tmem + 256;
-
-  const uint32_t q_addr = smem_u32(smem + S::kQ);
-  const uint32_t k_addr = smem_u32(smem + S::kK);
-  const uint32_t v_addr = smem_u32(smem + S::kV);
+  // TMEM columns: slot s has S/P at [128 s, 128 s + 128) and O at 256 + 128 s.
+  const uint32_t q_addr = smem_u32(smem + C::kQ);
+  const uint32_t ring_addr = smem_u32(smem + C::kRing);
 
   // virtual row -> TMA row coordinate of a 64-row box
   auto box_row = [&](int vrow) -> int {
     return block_mode ? (c + p.d * (vrow / kBlockRows)) * kBlockRows : vrow;
   };
 
-  if (warp == 0) {
-    // =========================== producer ===========================
-    if (lane == 0) {
-      prefetch_tensormap(&p.tmQ[map_idx]);
-      prefetch_tensormap(&p.tmK[map_idx]);
-      prefetch_tensormap(&p.tmV[map_idx]);
-      mbar_arrive_expect_tx(full_q, S::kTileBytes);
-      for (int cc = 0; cc < D / 64; ++cc)
-        for (int hh = 0; hh < 2; ++hh)
-          tma_load_4d(smem + S::kQ + cc * kChunkBytes + hh * (kChunkBytes / 2), &p.tmQ[map_idx],
-                      full_q, cc * 64, h, box_row(qt * kTileM + hh * 64), b);
-    }
-    for (int it = 0; it < n_tiles; ++it) {
-      const int st = it % kStages;
-      const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-      for (int kv = 0; kv < 2; ++kv) {  // 0: K, 1: V
-        uint64_t* emp = kv ? &empty_v[st] : &empty_k[st];
-        uint64_t* ful = kv ? &full_v[st] : &full_k[st];
-        uint8_t* dst = smem + (kv ? S::kV : S::kK) + st * S::kTileBytes;
-        if (it >= kStages && !mbar_wait(emp, ph ^ 1u, p.err, abort_flag)) goto producer_done;
-        if (it < n_band) {
-          if (lane == 0) {
-            const CUtensorMap* m = kv ? &p.tmV[map_idx] : &p.tmK[map_idx];
-            const int t = tr.kv_begin + it;
-            mbar_arrive_expect_tx(ful, S::kTileBytes);
-            for (int cc = 0; cc < D / 64; ++cc)
-              for (int hh = 0; hh < 2; ++hh)
-                tma_load_4d(dst + cc * kChunkBytes + hh * (kChunkBytes / 2), m, ful, cc * 64,
-                            hkv, box_row(t * kTileN + hh * 64), b);
-          }
-        } else {
-          // gather global-key rows with plain 16-byte loads into the
-          // swizzled layout the MMA expects
-          const int g0 = (it - n_band) * kTileN;
-          const int cnt = min(kTileN, p.n_global - g0);
-          const uint16_t* src_base = kv ? p.v_raw : p.k_raw;
-          constexpr int kC16 = D / 8;  // 16-byte chunks per row
-          for (int idx = lane; idx < kTileN * kC16; idx += 32) {
-            const int row = idx / kC16, c16 = idx % kC16;
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (row < cnt) {
-              int gv = __ldg(p.G + g0 + row);
-              gv = gv < 0 ? 0 : (gv >= p.N ? p.N - 1 : gv);
-              const uint16_t* src =
-                  src_base + (((size_t)b * p.N + gv) * p.Hkv + hkv) * D + c16 * 8;
-              val = __ldg(reinterpret_cast<const uint4*>(src));
+  if (warp < 4) {
+    if (warp == 0) {
+      // =========================== producer ===========================
+      if (lane == 0) {
+        prefetch_tensormap(&p.tmQ[map_idx]);
+        prefetch_tensormap(&p.tmK[map_idx]);
+        prefetch_tensormap(&p.tmV[map_idx]);
+        mbar_arrive_expect_tx(full_q, C::kQBytes);
+        for (int s = 0; s < NSLOT; ++s)
+          for (int cc = 0; cc < D / 64; ++cc)
+            for (int hh = 0; hh < 2; ++hh)
+              tma_load_4d(smem + C::kQ + s * C::kTile + cc * kChunkBytes + hh * (kChunkBytes / 2),
+                          &p.tmQ[map_idx], full_q, cc * 64, head[s],
+                          box_row(qt * kTileM + hh * 64), b);
+      }
+      for (int it = 0; it < n_tiles; ++it) {
+        const int st = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
+        for (int kv = 0; kv < 2; ++kv) {  // 0: K, 1: V
+          uint64_t* emp = kv ? &empty_v[st] : &empty_k[st];
+          uint64_t* ful = kv ? &full_v[st] : &full_k[st];
+          uint8_t* dst = smem + C::kRing + st * C::kStageBytes + kv * NSTREAM * C::kTile;
+          if (it >= kStages && !mbar_wait(emp, ph ^ 1u, p.err, abort_flag)) goto producer_done;
+          if (it < n_band) {
+            if (lane == 0) {
+              const CUtensorMap* m = kv ? &p.tmV[map_idx] : &p.tmK[map_idx];
+              const int t = tr.kv_begin + it;
+              mbar_arrive_expect_tx(ful, NSTREAM * C::kTile);
+              for (int s = 0; s < NSTREAM; ++s)
+                for (int cc = 0; cc < D / 64; ++cc)
+                  for (int hh = 0; hh < 2; ++hh)
+                    tma_load_4d(dst + s * C::kTile + cc * kChunkBytes + hh * (kChunkBytes / 2), m,
+                                ful, cc * 64, kvh[s], box_row(t * kTileN + hh * 64), b);
             }
-            uint8_t* d8 = dst + (c16 / 8) * kChunkBytes + row * 128 + (((c16 % 8) ^ (row % 8)) * 16);
-            *reinterpret_cast<uint4*>(d8) = val;
+          } else {
+            // gather global-key rows with plain 16-byte loads into the
+            // swizzled layout the MMA expects
+            const int g0 = (it - n_band) * kTileN;
+            const int cnt = min(kTileN, p.n_global - g0);
+            const uint16_t* src_base = kv ? p.v_raw : p.k_raw;
+            constexpr int kC16 = D / 8;  // 16-byte chunks per row
+            for (int s = 0; s < NSTREAM; ++s) {
+              for (int idx = lane; idx < kTileN * kC16; idx += 32) {
+                const int row = idx / kC16, c16 = idx % kC16;
+                uint4 val = make_uint4(0u, 0u, 0u, 0u);
+                if (row < cnt) {
+                  int gv = __ldg(p.G + g0 + row);
+                  gv = gv < 0 ? 0 : (gv >= p.N ? p.N - 1 : gv);
+                  const uint16_t* src =
+                      src_base + (((size_t)b * p.N + gv) * p.Hkv + kvh[s]) * D + c16 * 8;
+                  val = __ldg(reinterpret_cast<const uint4*>(src));
+                }
+                uint8_t* d8 = dst + s * C::kTile + (c16 / 8) * kChunkBytes + row * 128 +
+                              (((c16 % 8) ^ (row % 8)) * 16);
+                *reinterpret_cast<uint4*>(d8) = val;
+              }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ful);
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(ful);
         }
       }
-    }
-  producer_done:;
-  } else if (warp == 1) {
-    // ============================ MMA issuer ============================
-    if (lane == 0 && n_tiles > 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(kTileM, kTileN, 0, 0);
-      const uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, 0, 1);
-      bool ok = mbar_wait(full_q, 0, p.err, abort_flag);
-      tc_fence_after();
-      auto issue_qk = [&](int it) -> bool {
-        const int st = it % kStages;
-        if (!mbar_wait(&full_k[st], (uint32_t)(it / kStages) & 1u, p.err, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t kb = k_addr + st * S::kTileBytes;
+    producer_done:;
+    } else if (warp == 1) {
+      // ============================ MMA issuer ============================
+      if (lane == 0 && n_tiles > 0) {
+        const uint32_t idesc_qk = idesc_bf16_f32(kTileM, kTileN, 0, 0);
+        const uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, 0, 1);
+        // Descriptors are built once; every MMA then only adds a compile-time
+        // offset (start address field, 16-byte units) to a base descriptor,
+        // so the single issuing thread keeps up with the tensor core.
+        const uint64_t dq0 = sdesc_sw128(q_addr, 16, 1024);
+        const uint64_t dk0 = sdesc_sw128(ring_addr, 16, 1024);
+        const uint64_t dv0 = sdesc_sw128(ring_addr + NSTREAM * C::kTile, kChunkBytes, 1024);
+        constexpr uint64_t kStageStep = C::kStageBytes >> 4;
+        constexpr uint64_t kTileStep = C::kTile >> 4;
+        auto qk = [&](int it, int s) {
+          const uint64_t dq = dq0 + (uint64_t)s * kTileStep;
+          const uint64_t dk = dk0 + (uint64_t)(it % kStages) * kStageStep +
+                              (NSTREAM == 2 ? (uint64_t)s * kTileStep : 0ull);
+          const uint32_t ts = tmem + 128u * s;
 #pragma unroll
-        for (int s = 0; s < D / 16; ++s) {
-          const uint32_t off = (s / 4) * kChunkBytes + (s % 4) * 32;
-          mma_ss(tS(it), sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
-                 idesc_qk, s > 0 ? 1u : 0u);
-        }
-        tc_commit(&empty_k[st]);
-        tc_commit(&s_full[it & 1]);
-        return true;
-      };
-      if (ok) ok = issue_qk(0);
-      for (int it = 0; ok && it < n_tiles; ++it) {
-        if (it + 1 < n_tiles && !issue_qk(it + 1)) break;
-        if (!mbar_wait(&p_full[it & 1], (uint32_t)(it >> 1) & 1u, p.err, abort_flag)) break;
-        tc_fence_after();
-        const int st = it % kStages;
-        if (!mbar_wait(&full_v[st], (uint32_t)(it / kStages) & 1u, p.err, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t vb = v_addr + st * S::kTileBytes;
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t off = (uint64_t)(((k / 4) * kChunkBytes + (k % 4) * 32) >> 4);
+            mma_ss(ts, dq + off, dk + off, idesc_qk, k > 0 ? 1u : 0u);
+          }
+          tc_commit(&s_full[s]);
+        };
+        auto pv = [&](int it, int s) {
+          const uint64_t dv = dv0 + (uint64_t)(it % kStages) * kStageStep +
+                              (NSTREAM == 2 ? (uint64_t)s * kTileStep : 0ull);
+          const uint32_t to = tmem + 256u + 128u * s, ts = tmem + 128u * s;
 #pragma unroll
-        for (int s = 0; s < kTileN / 16; ++s) {
-          mma_ts(tO, tS(it) + s * 8, sdesc_sw128(vb + s * 2048, kChunkBytes, 1024), idesc_pv,
-                 (it > 0 || s > 0) ? 1u : 0u);
+          for (int k = 0; k < kTileN / 16; ++k)
+            mma_ts(to, ts + k * 8, dv + (uint64_t)((k * 2048) >> 4), idesc_pv,
+                   (it > 0 || k > 0) ? 1u : 0u);
+          tc_commit(&o_done[s]);
+        };
+        bool ok = mbar_wait(full_q, 0, p.err, abort_flag);
+        tc_fence_after();
+        if (ok) ok = mbar_wait(&full_k[0], 0, p.err, abort_flag);
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int s = 0; s < NSLOT; ++s)
+            if (slot_ok[s]) qk(0, s);
+          tc_commit(&empty_k[0]);
         }
-        tc_commit(&empty_v[st]);
-        tc_commit(o_done);
+        for (int it = 0; ok && it < n_tiles; ++it) {
+          const int st = it % kStages;
+          const bool more = it + 1 < n_tiles;
+          if (!mbar_wait(&full_v[st], (uint32_t)(it / kStages) & 1u, p.err, abort_flag)) break;
+          tc_fence_after();
+          bool k_next_ready = false;
+#pragma unroll
+          for (int s = 0; s < NSLOT; ++s) {
+            if (!slot_ok[s]) continue;
+            if (!mbar_wait(&p_full[s], (uint32_t)it & 1u, p.err, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            pv(it, s);
+            if (more) {
+              if (!k_next_ready) {
+                if (!mbar_wait(&full_k[(it + 1) % kStages], (uint32_t)((it + 1) / kStages) & 1u,
+                               p.err, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                k_next_ready = true;
+              }
+              qk(it + 1, s);
+            }
+          }
+          if (!ok) break;
+          tc_commit(&empty_v[st]);
+          if (more) tc_commit(&empty_k[(it + 1) % kStages]);
+        }
+        // o_final completes once every MMA issued above has finished (also on
+        // the abort path, so TMEM is quiescent before it is freed).
+        tc_commit(&o_final[0]);
+        tc_commit(&o_final[1]);
       }
-      // o_final completes once every MMA issued above has finished (also on
-      // the abort path, so TMEM is quiescent before it is freed).
-      tc_commit(o_final);
     }
-  } else if (warp >= 4) {
+  } else {
     // ============================ softmax ============================
+    const int slot = warp / 4 - 1;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + 128u * slot + lane_off;
+    const uint32_t tO = tmem + 256u + 128u * slot + lane_off;
+    const int h = head[slot];
     const int m_row = qt * kTileM + r;
-    const bool row_valid = m_row < Mv;
+    const bool row_valid = m_row < Mv && slot_ok[slot];
     const int klo = key_lo(g, m_row);
     const int khi = key_hi(g, m_row, Mv);
-    const int64_t i_phys = phys_row(g, c, m_row);
+    const int i_phys = (int)phys_row(g, c, m_row);
     const bool causal = p.R == 0;
+    // band of the row in physical positions, for the global-key test
+    const int glo = p.L < 0 ? -0x40000000
+                            : (block_mode ? (i_phys / p.bs - (p.L / p.bs) * p.d) * p.bs
+                                          : i_phys - p.L * p.d);
+    const int ghi = p.R < 0 ? 0x40000000
+                            : (block_mode ? (i_phys / p.bs + (p.R / p.bs) * p.d + 1) * p.bs - 1
+                                          : i_phys + p.R * p.d);
     const float sl2 = p.scale_log2;
     float m_used = -INFINITY;  // running max, scaled log2 units
     float l = 0.f;
-    bool ok = true;
+    bool ok = slot_ok[slot];
 
-    for (int it = 0; it < n_tiles; ++it) {
-      const bool w_ok = mbar_wait(&s_full[it & 1], (uint32_t)(it >> 1) & 1u, p.err, abort_flag);
-      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-      tc_fence_after();
-      float s[kTileN];
+    float m_pend = -INFINITY;  // max seen but not yet adopted (adopted next tile)
+
+    // 64 score columns [64 hf, 64 hf + 64) of tile `it`, masked on edge and
+    // global tiles (-inf outside the row's key set).
+    auto load_half = [&](int it, int hf, bool edge, float (&sv)[64]) {
 #pragma unroll
-      for (int j = 0; j < kTileN / 32; ++j) {
+      for (int jj = 0; jj < 2; ++jj) {
         uint32_t v[32];
-        tmem_ld32(tS(it) + lane_off + j * 32, v);
+        tmem_ld32(tS + hf * 64 + jj * 32, v);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s[j * 32 + e] = __uint_as_float(v[e]);
+        for (int e = 0; e < 32; ++e) sv[jj * 32 + e] = __uint_as_float(v[e]);
       }
       tmem_wait_ld();
-
       if (it < n_band) {
-        const int t = tr.kv_begin + it;
-        if (!tile_interior(g, Mv, qt, t)) {
-          const int n0 = t * kTileN;
+        if (edge) {
+          const int n0 = (tr.kv_begin + it) * kTileN + hf * 64;
 #pragma unroll
-          for (int j = 0; j < kTileN; ++j) {
+          for (int j = 0; j < 64; ++j) {
             const int n = n0 + j;
-            if (n < klo || n > khi || n >= Mv) s[j] = -INFINITY;
+            if (n < klo || n > khi || n >= Mv) sv[j] = -INFINITY;
           }
         }
       } else {
-        const int g0 = (it - n_band) * kTileN;
+        // a global key joins the row unless it is already in the row's band
+        // (same residue class and inside [glo, ghi]) or, causal, after it
+        const int g0 = (it - n_band) * kTileN + hf * 64;
 #pragma unroll
-        for (int j = 0; j < kTileN; ++j) {
+        for (int j = 0; j < 64; ++j) {
           bool keep = false;
           if (g0 + j < p.n_global) {
             int gv = __ldg(p.G + g0 + j);
             gv = gv < 0 ? 0 : (gv >= p.N ? p.N - 1 : gv);
-            keep = !in_band_phys(p.L, p.R, p.d, p.bs, (int)i_phys, gv) &&
-                   (!causal || gv <= i_phys);
+            bool same = true;
+            if (p.d > 1) same = ((block_mode ? gv / p.bs : gv) % p.d) == c;
+            const bool inband = same && gv >= glo && gv <= ghi;
+            keep = !inband && (!causal || gv <= i_phys);
           }
-          if (!keep) s[j] = -INFINITY;
+          if (!keep) sv[j] = -INFINITY;
         }
       }
-
-      float mx = -INFINITY;
+    };
+    auto half_max = [&](const float (&sv)[64]) -> float {
+      float t[8];
 #pragma unroll
-      for (int j = 0; j < kTileN; ++j) mx = fmaxf(mx, s[j]);
-      const float m_new = fmaxf(m_used, mx * sl2);
-      const bool rescale = m_new > m_used + kRescaleThreshold;
-      if (it > 0 && __any_sync(0xffffffffu, rescale)) {
-        // O holds P_0..P_{it-1} V; wait until the last of those MMAs is done.
-        const bool o_ok = mbar_wait(o_done, (uint32_t)(it - 1) & 1u, p.err, abort_flag);
-        if (!__all_sync(0xffffffffu, o_ok)) { ok = false; break; }
-        tc_fence_after();
-        const float f = rescale ? ex2_approx(m_used - m_new) : 1.f;
-        l *= f;
+      for (int e = 0; e < 8; ++e) t[e] = max3f(sv[e], sv[8 + e], sv[16 + e]);
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
-          uint32_t v[32];
-          tmem_ld32(tO + lane_off + j * 32, v);
-          tmem_wait_ld();
+      for (int j = 24; j < 64; j += 16)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-          tmem_st32(tO + lane_off + j * 32, v);
-        }
-        tmem_wait_st();
-      }
-      if (rescale) m_used = m_new;
-      const float m_safe = m_used == -INFINITY ? 0.f : m_used;
-
-      float lsum = 0.f;
+        for (int e = 0; e < 8; ++e) t[e] = max3f(t[e], sv[j + e], sv[j + 8 + e]);
+      return max3f(max3f(t[0], t[1], t[2]), max3f(t[3], t[4], t[5]), fmaxf(t[6], t[7]));
+    };
+    // P = 2^(s * scale * log2 e - m_ref) for one half, stored as bf16 pairs
+    // over the half's S columns.  Three of every four column pairs go to the
+    // MUFU ex2 unit and one to the FMA pipe (polynomial), so the two softmax
+    // warpgroups of the SM do not saturate MUFU.
+    auto exp_half = [&](int hf, const float (&sv)[64], float m_ref, float2 (&ls)[4]) {
+      const float2 sl2_2 = make_float2(sl2, sl2), negm2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
-      for (int j = 0; j < kTileN / 32; ++j) {
+      for (int jj = 0; jj < 2; ++jj) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2_approx(fmaf(s[j * 32 + 2 * e], sl2, -m_safe));
-          const float p1 = ex2_approx(fmaf(s[j * 32 + 2 * e + 1], sl2, -m_safe));
-          lsum += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          const float2 xa =
+              fma2(make_float2(sv[jj * 32 + 2 * e], sv[jj * 32 + 2 * e + 1]), sl2_2, negm2);
+          float2 pr;
+          if ((e & 3) == 3) {
+            pr = exp2_poly2(xa);
+          } else {
+            pr.x = ex2_approx(xa.x);
+            pr.y = ex2_approx(xa.y);
+          }
+          ls[e & 3] = add2(ls[e & 3], pr);
+          pk[e] = pack_bf16x2(pr.x, pr.y);
         }
-        tmem_st16(tS(it) + lane_off + j * 16, pk);
+        tmem_st16(tS + hf * 32 + jj * 16, pk);
       }
-      l += lsum;
+    };
+    // Multiplies O (and l) by 2^(m_from - m_to) and adopts m_to; O holds
+    // P_0..P_{it-1} V, whose MMA finished before S of tile it was produced.
+    auto rescale_o = [&](int it, bool mine, float m_to) -> bool {
+      const bool o_ok = mbar_wait(&o_done[slot], (uint32_t)(it - 1) & 1u, p.err, abort_flag);
+      if (!__all_sync(0xffffffffu, o_ok)) return false;
+      tc_fence_after();
+      const float f = mine ? ex2_approx(m_used - m_to) : 1.f;
+      l *= f;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        uint32_t v[32];
+        tmem_ld32(tO + j * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+        tmem_st32(tO + j * 32, v);
+      }
+      tmem_wait_st();
+      if (mine) m_used = m_to;
+      return true;
+    };
+
+    for (int it = 0; ok && it < n_tiles; ++it) {
+      const bool w_ok = mbar_wait(&s_full[slot], (uint32_t)it & 1u, p.err, abort_flag);
+      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+      tc_fence_after();
+      const bool edge = it < n_band && !tile_interior(g, Mv, qt, tr.kv_begin + it);
+
+      // adopt a larger max seen on the previous tile (rare after the start)
+      const bool pend = m_pend > m_used;
+      if (__any_sync(0xffffffffu, pend)) {
+        if (!rescale_o(it, pend, m_pend)) { ok = false; break; }
+      }
+
+      float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
+      // TMEM columns of this slot: S half 0 at [0, 64), S half 1 at [64, 128);
+      // P (bf16 pairs) of half 0 goes to [0, 32) and of half 1 to [32, 64),
+      // so S is never read after its columns have been overwritten.
+      float tmax;
+      float sv[64];
+      if (!__any_sync(0xffffffffu, m_used == -INFINITY)) {
+        // Fast path: exponentiate against the current max in one pass and
+        // track the tile max on the way.  Scores above the current max only
+        // enlarge P (by at most 2^64 here, safe in fp32 and bf16).
+        load_half(it, 0, edge, sv);
+        tmax = half_max(sv);
+        if (__any_sync(0xffffffffu, tmax * sl2 > m_used + 64.f)) {
+          // a large jump in half 0: adopt the new max before any P exists
+          const bool up = tmax * sl2 > m_used;
+          if (!rescale_o(it, up, fmaxf(m_used, tmax * sl2))) { ok = false; break; }
+        }
+        exp_half(0, sv, m_used, ls);
+        load_half(it, 1, edge, sv);
+        const float tmax1 = half_max(sv);
+        tmax = fmaxf(tmax, tmax1);
+        const bool jump = tmax1 * sl2 > m_used + 64.f;
+        if (__any_sync(0xffffffffu, jump)) {
+          // a large jump in half 1: rescale O, l, the partial sums and the
+          // bf16 P of half 0 already in TMEM to the new max
+          const float m_old = m_used;
+          if (!rescale_o(it, jump, fmaxf(m_used, tmax1 * sl2))) { ok = false; break; }
+          const float f = jump ? ex2_approx(m_old - m_used) : 1.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) ls[e] = make_float2(ls[e].x * f, ls[e].y * f);
+          uint32_t v[32];
+          tmem_wait_st();
+          tmem_ld32(tS, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            v[e] = pack_bf16x2(__uint_as_float(v[e] << 16) * f,
+                               __uint_as_float(v[e] & 0xFFFF0000u) * f);
+          tmem_st32(tS, v);
+        }
+        exp_half(1, sv, m_used, ls);
+      } else {
+        // Some row has no key yet: find the tile max first (one pass over
+        // the scores), then exponentiate (a second pass).
+        load_half(it, 1, edge, sv);
+        tmax = half_max(sv);
+        load_half(it, 0, edge, sv);
+        tmax = fmaxf(tmax, half_max(sv));
+        const float m_new = fmaxf(m_used, tmax * sl2);
+        const bool up = m_new > m_used;
+        if (it > 0 && __any_sync(0xffffffffu, up)) {
+          if (!rescale_o(it, up, m_new)) { ok = false; break; }
+        } else if (up) {
+          m_used = m_new;
+        }
+        const float m_safe = m_used == -INFINITY ? 0.f : m_used;
+        exp_half(0, sv, m_safe, ls);
+        load_half(it, 1, edge, sv);
+        exp_half(1, sv, m_safe, ls);
+      }
+      {
+        const float2 a = add2(add2(ls[0], ls[1]), add2(ls[2], ls[3]));
+        l += a.x + a.y;
+      }
+      // a max that grew by more than 2^8 is adopted before the next tile
+      if (tmax * sl2 > m_used + kRescaleThreshold) m_pend = tmax * sl2;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[it & 1]);
+      mbar_arrive(&p_full[slot]);
     }
 
     bool fin = ok && n_tiles > 0;
-    if (fin) fin = mbar_wait(o_final, 0, p.err, abort_flag);
+    if (fin) fin = mbar_wait(&o_final[slot], 0, p.err, abort_flag);
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
       const float inv = 1.f / l;
@@ -390,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1) swa_fwd_sm100_kernel(const __grid
       for (int j = 0; j < D / 32; ++j) {
         uint32_t v[32];
         __syncwarp();
-        tmem_ld32(tO + lane_off + j * 32, v);
+        tmem_ld32(tO + j * 32, v);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
@@ -413,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1) swa_fwd_sm100_kernel(const __grid
     // abort path: o_final was committed after the last issued MMA; give it
     // a bounded chance to land before TMEM is released.
     volatile int no_abort = 0;
-    mbar_wait(o_final, 0, nullptr, &no_abort, 100000000ull);
+    mbar_wait(&o_final[0], 0, nullptr, &no_abort, 100000000ull);
   }
   tc_fence_before();
   __syncthreads();
@@ -424,15 +575,15 @@ __global__ void __launch_bounds__(kThreads, 1) swa_fwd_sm100_kernel(const __grid
   }
 }
 
-template <int D>
+template <int D, int NSLOT, int NSTREAM>
 int launch_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
                 int Hkv, int N, int L, int R, int d, int bs, const int32_t* G, int ng,
                 float scale, cudaStream_t stream) {
-  using S = Smem<D>;
+  using C = Cfg<D, NSLOT, NSTREAM>;
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(swa_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             S::kAlloc) != cudaSuccess)
+    if (cudaFuncSetAttribute(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess)
       return SWA_ERR_CUDA;
     attr_set = true;
   }
@@ -489,10 +640,10 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
                        CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return SWA_ERR_CUDA;
     }
-    const long grid = (long)p.qtile_prefix[p.nclass] * B * H;
+    const long grid = (long)p.qtile_prefix[p.nclass] * B * ((H + NSLOT - 1) / NSLOT);
     if (grid <= 0) continue;
     if (grid > 0x7fffffffL) return SWA_ERR_UNSUPPORTED;
-    swa_fwd_sm100_kernel<D><<<(unsigned)grid, kThreads, S::kAlloc, stream>>>(p);
+    swa_fwd_sm100_kernel<D, NSLOT, NSTREAM><<<(unsigned)grid, C::kThreads, C::kAlloc, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
   }
   return SWA_OK;
@@ -500,13 +651,27 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
 
 }  // namespace
 
+// Two query heads per CTA when they share a kv head (GQA group of even
+// size), or, at D = 64, when two K/V streams fit in shared memory; one head
+// per CTA otherwise.
 int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                      int H, int Hkv, int N, int D, int L, int R, int d, int bs, const int32_t* G,
                      int ng, float scale, cudaStream_t stream) {
-  if (D == 128)
-    return launch_impl<128>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale, stream);
-  if (D == 64)
-    return launch_impl<64>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale, stream);
+  const bool gqa_pair = (H / Hkv) % 2 == 0;
+  if (D == 128) {
+    if (gqa_pair)
+      return launch_impl<128, 2, 1>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
+                                    stream);
+    return launch_impl<128, 1, 1>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
+                                  stream);
+  }
+  if (D == 64) {
+    if (gqa_pair)
+      return launch_impl<64, 2, 1>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
+                                   stream);
+    return launch_impl<64, 2, 2>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
+                                 stream);
+  }
   return SWA_ERR_UNSUPPORTED;
 }
 

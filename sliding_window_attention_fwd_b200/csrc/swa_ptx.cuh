@@ -233,6 +233,57 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Three-input max.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed fp32 pair arithmetic (one instruction for two lanes of work).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x on the FMA pipe, for x <= 2^20 (and x = -inf), two lanes at a time.
+// Cody-Waite style split x = n + f with n = rint(x) (adding 1.5 * 2^23
+// leaves rint(x) in the low mantissa bits) and f in [-1/2, 1/2]; 2^f from a
+// degree-3 polynomial fitted by iterated weighted least squares to minimise
+// the relative error on [-1/2, 1/2] (max relative error 7.6e-5); 2^n is
+// applied by adding n to the exponent field.  Inputs below -125 are clamped
+// to -125, so the result is >= 2^-125 (never denormal, never 0): callers use
+// it only where such a value is negligible against a sum >= 1.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kC0 = 0.99992823600769043f, kC1 = 0.69326096773147583f,
+                  kC2 = 0.24260851740837097f, kC3 = 0.05517049878835678f;
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = add2(x, make_float2(kMagic, kMagic));
+  const float2 n = add2(t, make_float2(-kMagic, -kMagic));
+  const float2 f = fma2(n, make_float2(-1.f, -1.f), x);
+  float2 q = fma2(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
+  q = fma2(q, f, make_float2(kC1, kC1));
+  q = fma2(q, f, make_float2(kC0, kC0));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
 // Packs two floats to bf16x2 (round to nearest even): lo -> bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

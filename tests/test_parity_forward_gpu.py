@@ -155,3 +155,18 @@ def test_full_size_sampled(swa, name):
     compare(got_o, ref_o, BF16_MAX_ABS, BF16_MEAN_ABS, what=f"{name} out")
     compare(got_l, ref_l, LSE_ABS, what=f"{name} lse")
     assert np.isfinite(out).all()
+
+
+@pytest.mark.parametrize("D,H,Hkv", [(128, 4, 2), (64, 2, 2), (128, 3, 3)])
+def test_bf16_score_jumps(swa, D, H, Hkv):
+    """A few keys with huge scores appear late in a row's window: the running
+    max jumps by far more than 2^64 in both halves of a key tile, which forces
+    the kernel to rescale O, l and the already written P."""
+    B, N = 1, 1024
+    q, k, v = rand_case(B, N, H, Hkv, D, 23)
+    k = k.float()
+    for pos in (300, 330, 700, 770, 1000):  # first and second halves of key tiles
+        k[:, pos] *= 40.0
+    k = k.to(torch.bfloat16)
+    full_check(swa, (q, k, v, 600, 0, 1, 0, None, 0.0))
+    full_check(swa, (q, k, v, 200, 200, 1, 0, None, 0.0))
