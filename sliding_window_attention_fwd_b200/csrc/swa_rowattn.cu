@@ -31,7 +31,7 @@ namespace swa {
 namespace {
 
 constexpr int kRows = 64;           // key rows per stage
-constexpr int kStagesR = 3;
+constexpr int kStagesR = 2;
 constexpr int kComputeWarps = 4;
 constexpr int kThreadsR = (kComputeWarps + 1) * 32;
 
@@ -58,14 +58,16 @@ template <int D, int NQ>
 struct RSmem {
   static constexpr int kTile = kRows * D * 2;
   static constexpr int kStage = 2 * kTile;
-  static constexpr int kSc = kStagesR * kStage;
-  static constexpr int kPc = kSc + kRows * NQ * 4;
-  static constexpr int kCorr = kPc + kRows * NQ * 4;
+  static constexpr int kSc = kStagesR * kStage;       // scores [row][slot]
+  static constexpr int kPc = kSc + kRows * NQ * 4;    // probabilities [row][slot]
+  static constexpr int kCorr = kPc + kRows * NQ * 4;  // per-slot rescale factor
   static constexpr int kBar = kCorr + 64;
   static constexpr int kMisc = kBar + 2 * kStagesR * 8;
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;
-  static_assert((128 / (D / 8)) * NQ * D * 4 <= kSc, "reduction buffer must fit in the ring");
+  // epilogue reduction buffer [warp][slot][D] floats, reusing the ring
+  static_assert(kComputeWarps * NQ * D * 4 <= kSc, "reduction buffer must fit in the ring");
+  static_assert((kRows / 4) % kComputeWarps == 0, "row groups split evenly over the warps");
 };
 
 __device__ __forceinline__ void named_sync(int id, int n) {
@@ -74,9 +76,45 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ float2 bf2(uint32_t w) { return make_float2(bf_lo(w), bf_hi(w)); }
+
+// Sum of v[0..NQ) over the 8 lanes of a row group, transposed: at each of
+// the three exchange levels a lane sends the half of its values it does not
+// keep, so NQ values need NQ-1 shuffles (butterfly: 3 NQ).  Lane t ends up
+// with the full sum of slot (t >> (3 - log2 NQ)) & (NQ - 1) (for NQ < 8 two
+// or more neighbouring lanes hold the same slot).
+template <int NQ>
+__device__ __forceinline__ float reduce8_transposed(float (&v)[NQ], int t, int* slot_out) {
+  float w[NQ];
+#pragma unroll
+  for (int i = 0; i < NQ; ++i) w[i] = v[i];
+  int n = NQ, base = 0;
+#pragma unroll
+  for (int lvl = 4; lvl >= 1; lvl >>= 1) {
+    if (n > 1) {
+      const bool upper = (t & lvl) != 0;  // keep the upper half of the values
+      const int h = n / 2;
+#pragma unroll
+      for (int i = 0; i < NQ / 2; ++i) {
+        if (i < h) {
+          const float send = upper ? w[i] : w[i + h];
+          const float keep = upper ? w[i + h] : w[i];
+          w[i] = keep + __shfl_xor_sync(0xffffffffu, send, lvl);
+        }
+      }
+      base += upper ? h : 0;
+      n = h;
+    } else {
+      w[0] += __shfl_xor_sync(0xffffffffu, w[0], lvl);
+    }
+  }
+  *slot_out = base;
+  return w[0];
+}
 
 template <int D, int NQ>
-__global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_constant__ RowParams p) {
+__global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
+    swa_rowattn_kernel(const __grid_constant__ RowParams p) {
   using S = RSmem<D, NQ>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -103,7 +141,7 @@ __global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_
     g = (gi / p.nrowchunks) % p.Hkv;
     b = gi / (p.nrowchunks * p.Hkv);
   }
-  // per slot: query row pointer offset and key limit (keys [0, limit))
+  // per slot: query row offset and key limit (keys [0, limit))
   long qoff[NQ];
   int limit[NQ];
   int max_limit = 0;
@@ -145,16 +183,15 @@ __global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_
   }
   __syncthreads();
 
-  // running softmax state of the slots this warp owns in the stats phase
+  // PV mapping: every warp handles whole value rows; lane owns EPL columns.
+  constexpr int EPL = D / 32;
+  // running stats of the slots this warp owns: warp + 4 u
   float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-  constexpr int kCPL = D / 64;        // 16-byte chunks per lane per row (QK)
-  constexpr int kLanesPV = D / 8;     // lanes per value row (PV)
-  constexpr int kRG = 128 / kLanesPV; // row groups in PV
-  float acc[NQ][8];
+  float2 acc[NQ][EPL / 2];
 #pragma unroll
   for (int s = 0; s < NQ; ++s)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[s][e] = 0.f;
+    for (int e = 0; e < EPL / 2; ++e) acc[s][e] = make_float2(0.f, 0.f);
 
   if (warp == kComputeWarps) {
     // ============================ producer ============================
@@ -178,9 +215,11 @@ __global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_
   } else {
     // ============================ compute ============================
     // QK mapping: 8 lanes per key row, lane t reads 16-byte chunk t of each
-    // 128-byte half of the row; a warp covers 4 rows per step.
+    // 128-byte half of the row (conflict free under the swizzle); a warp
+    // covers 4 rows per step, the 8 warps a 64-row stage in two steps.
+    constexpr int kCPL = D / 64;
     const int t8 = lane & 7, rsub = lane >> 3;
-    float qv[NQ][kCPL * 8];
+    float2 qv[NQ][kCPL * 4];
 #pragma unroll
     for (int s = 0; s < NQ; ++s) {
 #pragma unroll
@@ -190,13 +229,11 @@ __global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_
         const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          qv[s][hh * 8 + 2 * e] = bf_lo(ws[e]) * p.scale_log2;
-          qv[s][hh * 8 + 2 * e + 1] = bf_hi(ws[e]) * p.scale_log2;
+          const float2 f = bf2(ws[e]);
+          qv[s][hh * 4 + e] = make_float2(f.x * p.scale_log2, f.y * p.scale_log2);
         }
       }
     }
-    const int pv_chunk = threadIdx.x % kLanesPV;  // 16-byte chunk of a value row
-    const int pv_rg = threadIdx.x / kLanesPV;
 
     for (int k = 0; k < n_stages; ++k) {
       const int st = k % kStagesR;
@@ -207,13 +244,13 @@ __global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_
       mbar_wait(&full[st], (uint32_t)(k / kStagesR) & 1u, p.err, abort_flag);
       const uint8_t* kb = smem + st * S::kStage;
       const uint8_t* vb = kb + S::kTile;
-      // ---- scores: warp w handles rows [16w, 16w+16)
+      // ---- scores of the stage's 64 key rows, for every slot
 #pragma unroll
-      for (int step = 0; step < 4; ++step) {
-        const int r = warp * 16 + step * 4 + rsub;
-        float dot[NQ];
+      for (int j = 0; j < kRows / 4 / kComputeWarps; ++j) {
+        const int r = (warp + j * kComputeWarps) * 4 + rsub;
+        float2 d2[NQ];
 #pragma unroll
-        for (int s = 0; s < NQ; ++s) dot[s] = 0.f;
+        for (int s = 0; s < NQ; ++s) d2[s] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int hh = 0; hh < kCPL; ++hh) {
           const uint4 w = *reinterpret_cast<const uint4*>(kb + hh * (kRows * 128) + r * 128 +
@@ -221,75 +258,90 @@ __global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_
           const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float k0 = bf_lo(ws[e]), k1 = bf_hi(ws[e]);
+            const float2 kk = bf2(ws[e]);
 #pragma unroll
-            for (int s = 0; s < NQ; ++s) {
-              dot[s] = fmaf(qv[s][hh * 8 + 2 * e], k0, dot[s]);
-              dot[s] = fmaf(qv[s][hh * 8 + 2 * e + 1], k1, dot[s]);
-            }
+            for (int s = 0; s < NQ; ++s) d2[s] = fma2(qv[s][hh * 4 + e], kk, d2[s]);
           }
         }
+        float dot[NQ];
 #pragma unroll
-        for (int s = 0; s < NQ; ++s) {
-          dot[s] += __shfl_xor_sync(0xffffffffu, dot[s], 4);
-          dot[s] += __shfl_xor_sync(0xffffffffu, dot[s], 2);
-          dot[s] += __shfl_xor_sync(0xffffffffu, dot[s], 1);
-        }
-        if (t8 == 0) {
+        for (int s = 0; s < NQ; ++s) dot[s] = d2[s].x + d2[s].y;
+        int myslot;
+        const float tot = reduce8_transposed<NQ>(dot, t8, &myslot);
+        // after the reduction lanes t with t % (8 / NQ) == 0 hold distinct
+        // slots; each writes its (row, slot) score
+        if ((t8 & (8 / NQ - 1)) == 0) {
           const int key = key0 + k * kRows + r;
+          int lim = 0;
 #pragma unroll
-          for (int s = 0; s < NQ; ++s) sc[r * NQ + s] = key < limit[s] ? dot[s] : -INFINITY;
+          for (int s = 0; s < NQ; ++s)
+            if (s == myslot) lim = limit[s];
+          sc[r * NQ + myslot] = key < lim ? tot : -INFINITY;
         }
       }
       named_sync(1, kComputeWarps * 32);
-      // ---- online softmax statistics: warp w owns slots w and w + 4
+      // ---- online softmax statistics: warp w owns slots w, w + 4
+      for (int s = warp; s < NQ; s += kComputeWarps) {
+        const int u = s / kComputeWarps;
+        const float a0 = sc[lane * NQ + s], a1 = sc[(lane + 32) * NQ + s];
+        float mx = fmaxf(a0, a1);
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int s = warp + 4 * u;
-        if (s < NQ) {
-          const float a0 = sc[lane * NQ + s], a1 = sc[(lane + 32) * NQ + s];
-          float mx = fmaxf(a0, a1);
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float m_new = fmaxf(m_run[u], mx);
+        const float m_safe = m_new == -INFINITY ? 0.f : m_new;
+        const float cf = ex2_approx(m_run[u] - m_safe);
+        const float p0 = ex2_approx(a0 - m_safe), p1 = ex2_approx(a1 - m_safe);
+        pc[lane * NQ + s] = p0;
+        pc[(lane + 32) * NQ + s] = p1;
+        float sum = p0 + p1;
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          const float m_new = fmaxf(m_run[u], mx);
-          const float m_safe = m_new == -INFINITY ? 0.f : m_new;
-          const float cf = ex2_approx(m_run[u] - m_safe);
-          const float p0 = ex2_approx(a0 - m_safe), p1 = ex2_approx(a1 - m_safe);
-          pc[lane * NQ + s] = p0;
-          pc[(lane + 32) * NQ + s] = p1;
-          float sum = p0 + p1;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-          l_run[u] = l_run[u] * cf + sum;
-          m_run[u] = m_new;
-          if (lane == 0) corr_s[s] = cf;
-        }
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        l_run[u] = l_run[u] * cf + sum;
+        m_run[u] = m_new;
+        if (lane == 0) corr_s[s] = cf;
       }
       named_sync(1, kComputeWarps * 32);
-      // ---- O += P V: thread owns 8 columns of the value row for all slots
+      // ---- O += P V: warp w takes rows w, w + 4, ...; lane owns EPL columns
 #pragma unroll
       for (int s = 0; s < NQ; ++s) {
         const float cf = corr_s[s];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[s][e] *= cf;
+        for (int e = 0; e < EPL / 2; ++e) acc[s][e] = make_float2(acc[s][e].x * cf, acc[s][e].y * cf);
       }
-      const int hh = pv_chunk / 8, c8 = pv_chunk % 8;
+      // lane's EPL columns: byte offset lane * 2 * EPL of the row, in the
+      // 128-byte half (lane * 2 * EPL) / 128
+      const int byte0 = lane * 2 * EPL;
+      const int hh = byte0 / 128, c16 = (byte0 % 128) / 16, in16 = byte0 % 16;
 #pragma unroll 4
-      for (int r = pv_rg; r < kRows; r += kRG) {
-        const uint4 w = *reinterpret_cast<const uint4*>(vb + hh * (kRows * 128) + r * 128 +
-                                                        ((c8 ^ (r & 7)) * 16));
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-        float vv[8];
+      for (int r = warp; r < kRows; r += kComputeWarps) {
+        const uint8_t* src = vb + hh * (kRows * 128) + r * 128 + ((c16 ^ (r & 7)) * 16) + in16;
+        uint32_t vw[EPL / 2];
+        if (EPL == 4) {
+          const uint2 w = *reinterpret_cast<const uint2*>(src);
+          vw[0] = w.x;
+          vw[EPL / 2 - 1] = w.y;
+        } else {
+          vw[0] = *reinterpret_cast<const uint32_t*>(src);
+        }
+        float pr[NQ];
+        if (NQ >= 4) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          vv[2 * e] = bf_lo(ws[e]);
-          vv[2 * e + 1] = bf_hi(ws[e]);
+          for (int s4 = 0; s4 < NQ; s4 += 4) {
+            const float4 p4 = *reinterpret_cast<const float4*>(pc + r * NQ + s4);
+            pr[s4] = p4.x;
+            pr[s4 + 1] = p4.y;
+            pr[s4 + 2] = p4.z;
+            pr[s4 + 3] = p4.w;
+          }
+        } else {
+#pragma unroll
+          for (int s = 0; s < NQ; ++s) pr[s] = pc[r * NQ + s];
         }
 #pragma unroll
-        for (int s = 0; s < NQ; ++s) {
-          const float pr = pc[r * NQ + s];
+        for (int e = 0; e < EPL / 2; ++e) {
+          const float2 vv = bf2(vw[e]);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[s][e] = fmaf(pr, vv[e], acc[s][e]);
+          for (int s = 0; s < NQ; ++s) acc[s][e] = fma2(make_float2(pr[s], pr[s]), vv, acc[s][e]);
         }
       }
       mbar_arrive(&empty[st]);
@@ -297,23 +349,23 @@ __global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_
   }
   __syncthreads();  // every stage consumed: the ring can be reused below
 
-  // ---- reduce the row groups' partial sums: red[rg][slot][D]
+  // ---- reduce the warps' partial sums: red[warp][slot][D]
   float* red = reinterpret_cast<float*>(smem);
   if (warp < kComputeWarps) {
-    const int pv_chunk = threadIdx.x % kLanesPV;
-    const int pv_rg = threadIdx.x / kLanesPV;
 #pragma unroll
-    for (int s = 0; s < NQ; ++s)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) red[(pv_rg * NQ + s) * D + pv_chunk * 8 + e] = acc[s][e];
+    for (int s = 0; s < NQ; ++s) {
+      float* dst = red + (warp * NQ + s) * D + lane * EPL;
+      if (EPL == 4) {
+        *reinterpret_cast<float4*>(dst) = make_float4(acc[s][0].x, acc[s][0].y, acc[s][EPL / 2 - 1].x,
+                                                      acc[s][EPL / 2 - 1].y);
+      } else {
+        *reinterpret_cast<float2*>(dst) = acc[s][0];
+      }
+    }
     if (lane == 0) {
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int s = warp + 4 * u;
-        if (s < NQ) {
-          sc[s] = m_run[u];
-          sc[NQ + s] = l_run[u];
-        }
+      for (int s = warp; s < NQ; s += kComputeWarps) {
+        sc[s] = m_run[s / kComputeWarps];
+        sc[NQ + s] = l_run[s / kComputeWarps];
       }
     }
   }
@@ -326,7 +378,7 @@ __global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_
       const int s = idx / D, dd = idx % D;
       if (qoff[s] < 0) continue;
       float o = 0.f;
-      for (int rg = 0; rg < kRG; ++rg) o += red[(rg * NQ + s) * D + dd];
+      for (int w = 0; w < kComputeWarps; ++w) o += red[(w * NQ + s) * D + dd];
       const float l = sc[NQ + s];
       p.out[qoff[s] + dd] = __bfloat16_as_ushort(__float2bfloat16_rn(o / l));
     }
@@ -348,7 +400,7 @@ __global__ void __launch_bounds__(kThreadsR, 2) swa_rowattn_kernel(const __grid_
   for (int idx = threadIdx.x; idx < NQ * D; idx += blockDim.x) {
     const int s = idx / D, dd = idx % D;
     float o = 0.f;
-    for (int rg = 0; rg < kRG; ++rg) o += red[(rg * NQ + s) * D + dd];
+    for (int w = 0; w < kComputeWarps; ++w) o += red[(w * NQ + s) * D + dd];
     p.ws_o[part * NQ * D + idx] = o;
   }
   if (threadIdx.x < NQ) {
