@@ -599,7 +599,7 @@ int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* o
   p.grp = H / Hkv;
   p.rows_per_cta = 1;
   p.nrowchunks = 1;
-  p.chunk = 512;
+  p.chunk = 1024;  // keys per CTA: amortises the per-CTA set-up and merge
   p.nsplit = (W + p.chunk - 1) / p.chunk;
   p.scale_log2 = scale * 1.4426950408889634f;
   const int nq = pow2_at_least(p.grp);
