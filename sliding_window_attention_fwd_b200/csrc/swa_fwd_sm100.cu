@@ -49,6 +49,22 @@ constexpr int kMaxClasses = 8;   // residue classes per launch (tensor maps in p
 constexpr int kChunkBytes = kTileM * 128;  // one 64-column slice of a 128-row tile
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kTmemCols = 512;
+constexpr int kBarIssue = 1;  // named barrier: waiter warp -> MMA-issuing warp
+
+// bar.red.and over `nthreads` threads (whole warps) on named barrier `id`:
+// returns true when every participating thread passed true.
+__device__ __forceinline__ bool named_barrier_and(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
 
 struct FwdParams {
   CUtensorMap tmQ[kMaxClasses];
@@ -246,17 +262,22 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     producer_done:;
     } else if (warp == 1) {
       // ============================ MMA issuer ============================
-      if (lane == 0 && n_tiles > 0) {
+      // The whole warp walks the schedule and lane 0 issues.  The issuer
+      // never polls an mbarrier itself: such a poll queues behind the MMAs
+      // in flight and leaves the tensor core idle until it returns.  Warp 2
+      // does every wait and releases this warp through named barrier
+      // kBarIssue, whose AND-reduction carries "all waits succeeded".
+      if (n_tiles > 0) {
         const uint32_t idesc_qk = idesc_bf16_f32(kTileM, kTileN, 0, 0);
         const uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, 0, 1);
         // Descriptors are built once; every MMA then only adds a compile-time
-        // offset (start address field, 16-byte units) to a base descriptor,
-        // so the single issuing thread keeps up with the tensor core.
+        // offset (start address field, 16-byte units) to a base descriptor.
         const uint64_t dq0 = sdesc_sw128(q_addr, 16, 1024);
         const uint64_t dk0 = sdesc_sw128(ring_addr, 16, 1024);
         const uint64_t dv0 = sdesc_sw128(ring_addr + NSTREAM * C::kTile, kChunkBytes, 1024);
         constexpr uint64_t kStageStep = C::kStageBytes >> 4;
         constexpr uint64_t kTileStep = C::kTile >> 4;
+        const bool issuer = lane == 0;
         auto qk = [&](int it, int s) {
           const uint64_t dq = dq0 + (uint64_t)s * kTileStep;
           const uint64_t dk = dk0 + (uint64_t)(it % kStages) * kStageStep +
@@ -279,46 +300,72 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
                    (it > 0 || k > 0) ? 1u : 0u);
           tc_commit(&o_done[s]);
         };
-        bool ok = mbar_wait(full_q, 0, p.err, abort_flag);
+        // release 0: Q and K of tile 0 are in shared memory
+        bool ok = named_barrier_and(kBarIssue, 64, true);
         tc_fence_after();
-        if (ok) ok = mbar_wait(&full_k[0], 0, p.err, abort_flag);
-        if (ok) {
-          tc_fence_after();
+        if (ok && issuer) {
 #pragma unroll
           for (int s = 0; s < NSLOT; ++s)
             if (slot_ok[s]) qk(0, s);
           tc_commit(&empty_k[0]);
         }
-        for (int it = 0; ok && it < n_tiles; ++it) {
+        __syncwarp();
+        for (int it = 0; it < n_tiles; ++it) {
           const int st = it % kStages;
           const bool more = it + 1 < n_tiles;
-          if (!mbar_wait(&full_v[st], (uint32_t)(it / kStages) & 1u, p.err, abort_flag)) break;
-          tc_fence_after();
-          bool k_next_ready = false;
 #pragma unroll
           for (int s = 0; s < NSLOT; ++s) {
             if (!slot_ok[s]) continue;
-            if (!mbar_wait(&p_full[s], (uint32_t)it & 1u, p.err, abort_flag)) { ok = false; break; }
+            // release: P of slot s (and, for the first slot, V of this tile
+            // and K of the next) are ready
+            ok = named_barrier_and(kBarIssue, 64, true) && ok;
             tc_fence_after();
-            pv(it, s);
-            if (more) {
-              if (!k_next_ready) {
-                if (!mbar_wait(&full_k[(it + 1) % kStages], (uint32_t)((it + 1) / kStages) & 1u,
-                               p.err, abort_flag)) { ok = false; break; }
-                tc_fence_after();
-                k_next_ready = true;
-              }
-              qk(it + 1, s);
+            if (ok && issuer) {
+              pv(it, s);
+              if (more) qk(it + 1, s);
             }
+            __syncwarp();
           }
-          if (!ok) break;
-          tc_commit(&empty_v[st]);
-          if (more) tc_commit(&empty_k[(it + 1) % kStages]);
+          if (ok && issuer) {
+            tc_commit(&empty_v[st]);
+            if (more) tc_commit(&empty_k[(it + 1) % kStages]);
+          }
+          __syncwarp();
         }
         // o_final completes once every MMA issued above has finished (also on
         // the abort path, so TMEM is quiescent before it is freed).
-        tc_commit(&o_final[0]);
-        tc_commit(&o_final[1]);
+        if (issuer) {
+          tc_commit(&o_final[0]);
+          tc_commit(&o_final[1]);
+        }
+        __syncwarp();
+      }
+    } else if (warp == 2) {
+      // ============================ waiter ============================
+      // Mirrors the issuer's releases one for one.  After a failed wait
+      // (error recorded, abort set) it stops waiting but keeps releasing,
+      // so both warps always pass the same number of named barriers.
+      if (n_tiles > 0) {
+        bool ok = mbar_wait(full_q, 0, p.err, abort_flag) &&
+                  mbar_wait(&full_k[0], 0, p.err, abort_flag);
+        ok = named_barrier_and(kBarIssue, 64, ok);
+        for (int it = 0; it < n_tiles; ++it) {
+          const int st = it % kStages;
+          const bool more = it + 1 < n_tiles;
+          bool first = true;
+#pragma unroll
+          for (int s = 0; s < NSLOT; ++s) {
+            if (!slot_ok[s]) continue;
+            if (ok && first)
+              ok = mbar_wait(&full_v[st], (uint32_t)(it / kStages) & 1u, p.err, abort_flag);
+            if (ok) ok = mbar_wait(&p_full[s], (uint32_t)it & 1u, p.err, abort_flag);
+            if (ok && first && more)
+              ok = mbar_wait(&full_k[(it + 1) % kStages], (uint32_t)((it + 1) / kStages) & 1u,
+                             p.err, abort_flag);
+            first = false;
+            ok = named_barrier_and(kBarIssue, 64, ok);
+          }
+        }
       }
     }
   } else {
@@ -361,32 +408,35 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
         for (int e = 0; e < 32; ++e) sv[jj * 32 + e] = __uint_as_float(v[e]);
       }
       tmem_wait_ld();
+      // keep-mask of the half's 64 keys (bit j: key j is in the row's key
+      // set), applied by one shared select loop
+      uint64_t keep = ~0ull;
       if (it < n_band) {
         if (edge) {
           const int n0 = (tr.kv_begin + it) * kTileN + hf * 64;
-#pragma unroll
-          for (int j = 0; j < 64; ++j) {
-            const int n = n0 + j;
-            if (n < klo || n > khi || n >= Mv) sv[j] = -INFINITY;
-          }
+          const int lo = max(klo - n0, 0);
+          const int hi = min(min(khi, Mv - 1) - n0, 63);  // inclusive
+          keep = hi < lo ? 0ull : ((~0ull >> (63 - hi)) & (~0ull << lo));
         }
       } else {
         // a global key joins the row unless it is already in the row's band
         // (same residue class and inside [glo, ghi]) or, causal, after it
         const int g0 = (it - n_band) * kTileN + hf * 64;
-#pragma unroll
-        for (int j = 0; j < 64; ++j) {
-          bool keep = false;
-          if (g0 + j < p.n_global) {
-            int gv = __ldg(p.G + g0 + j);
-            gv = gv < 0 ? 0 : (gv >= p.N ? p.N - 1 : gv);
-            bool same = true;
-            if (p.d > 1) same = ((block_mode ? gv / p.bs : gv) % p.d) == c;
-            const bool inband = same && gv >= glo && gv <= ghi;
-            keep = !inband && (!causal || gv <= i_phys);
-          }
-          if (!keep) sv[j] = -INFINITY;
+        keep = 0ull;
+#pragma unroll 1
+        for (int j = 0; j < 64 && g0 + j < p.n_global; ++j) {
+          int gv = __ldg(p.G + g0 + j);
+          gv = gv < 0 ? 0 : (gv >= p.N ? p.N - 1 : gv);
+          bool same = true;
+          if (p.d > 1) same = ((block_mode ? gv / p.bs : gv) % p.d) == c;
+          const bool inband = same && gv >= glo && gv <= ghi;
+          if (!inband && (!causal || gv <= i_phys)) keep |= 1ull << j;
         }
+      }
+      if (__any_sync(0xffffffffu, keep != ~0ull)) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j)
+          if (!((keep >> j) & 1ull)) sv[j] = -INFINITY;
       }
     };
     auto half_max = [&](const float (&sv)[64]) -> float {
