@@ -243,8 +243,11 @@ SWA_API int swa_schedule(int N, int win_left, int win_right, int dilation, int d
     for (int qt = 0; qt < nqt; ++qt) {
       if (tile_out && n < cap) {
         TileRange r = tile_range(g, Mv, qt);
-        int edges = 0;
-        for (int t = r.kv_begin; t < r.kv_end; ++t) edges += tile_interior(g, Mv, qt, t) ? 0 : 1;
+        int ilo, ihi;
+        interior_tiles(g, Mv, qt, &ilo, &ihi);
+        if (ilo < r.kv_begin) ilo = r.kv_begin;
+        if (ihi > r.kv_end - 1) ihi = r.kv_end - 1;
+        const int edges = (r.kv_end - r.kv_begin) - (ihi >= ilo ? ihi - ilo + 1 : 0);
         int32_t* o = tile_out + 6 * n;
         o[0] = c;
         o[1] = qt;

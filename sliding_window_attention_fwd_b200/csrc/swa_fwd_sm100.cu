@@ -49,23 +49,6 @@ constexpr int kMaxClasses = 8;   // residue classes per launch (tensor maps in p
 constexpr int kChunkBytes = kTileM * 128;  // one 64-column slice of a 128-row tile
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kTmemCols = 512;
-constexpr int kBarIssue = 1;  // named barrier: waiter warp -> MMA-issuing warp
-
-// bar.red.and over `nthreads` threads (whole warps) on named barrier `id`:
-// returns true when every participating thread passed true.
-__device__ __forceinline__ bool named_barrier_and(int id, int nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-
 struct FwdParams {
   CUtensorMap tmQ[kMaxClasses];
   CUtensorMap tmK[kMaxClasses];
@@ -99,8 +82,8 @@ struct Cfg {
   static constexpr int kRing = kQ + kQBytes;
   static constexpr int kBar = kRing + kStages * kStageBytes;
   // full_q, full_k[S], empty_k[S], full_v[S], empty_v[S],
-  // s_full[2], p_full[2], o_done[2], o_final[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 8;
+  // se_full[2], sl_full[2], l_free[2], p_full[2], o_done[2], o_final[2]
+  static constexpr int kNumBars = 1 + 4 * kStages + 12;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
@@ -121,8 +104,10 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
   uint64_t* empty_k = full_k + kStages;
   uint64_t* full_v = empty_k + kStages;
   uint64_t* empty_v = full_v + kStages;
-  uint64_t* s_full = empty_v + kStages;  // [slot]
-  uint64_t* p_full = s_full + 2;
+  uint64_t* se_full = empty_v + kStages;  // [slot]: early half of S ready
+  uint64_t* sl_full = se_full + 2;        // [slot]: late half of S ready
+  uint64_t* l_free = sl_full + 2;         // [slot]: late half of S read out
+  uint64_t* p_full = l_free + 2;
   uint64_t* o_done = p_full + 2;
   uint64_t* o_final = o_done + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
@@ -165,14 +150,19 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(full_q, 1);
+    // every issuing slot releases each K/V stage once
+    int n_issuers = 0;
+    for (int s = 0; s < NSLOT; ++s) n_issuers += slot_ok[s] ? 1 : 0;
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full_k[s], 1);
-      mbar_init(&empty_k[s], 1);
+      mbar_init(&empty_k[s], n_issuers);
       mbar_init(&full_v[s], 1);
-      mbar_init(&empty_v[s], 1);
+      mbar_init(&empty_v[s], n_issuers);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
+      mbar_init(&se_full[s], 1);
+      mbar_init(&sl_full[s], 1);
+      mbar_init(&l_free[s], 128);
       mbar_init(&p_full[s], 128);
       mbar_init(&o_done[s], 1);
       mbar_init(&o_final[s], 1);
@@ -260,113 +250,98 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
         }
       }
     producer_done:;
-    } else if (warp == 1) {
-      // ============================ MMA issuer ============================
-      // The whole warp walks the schedule and lane 0 issues.  The issuer
-      // never polls an mbarrier itself: such a poll queues behind the MMAs
-      // in flight and leaves the tensor core idle until it returns.  Warp 2
-      // does every wait and releases this warp through named barrier
-      // kBarIssue, whose AND-reduction carries "all waits succeeded".
-      if (n_tiles > 0) {
-        const uint32_t idesc_qk = idesc_bf16_f32(kTileM, kTileN, 0, 0);
+    } else if (warp <= NSLOT) {
+      // =========================== MMA issuers ===========================
+      // Warp 1 + s issues the MMAs of slot s (lane 0; the rest of the warp
+      // idles at __syncwarp).  Each issuer sits on its own SM sub-partition:
+      // a single issuer sharing its sub-partition with two busy softmax
+      // warps gets too few issue slots to keep the tensor core fed, two of
+      // them together do.  A wait of one issuer leaves the tensor core to
+      // the other's MMAs.
+      //
+      // S of a slot is computed in two 64-key halves.  Tile j's P lives in
+      // the TMEM columns of its early half E(j) = j & 1, so the other half's
+      // columns are free as soon as the softmax has read them: the early
+      // half of tile j+1 (same columns) is issued then, while the softmax
+      // is still busy with tile j, and only the late half waits for PV(j).
+      const int s = warp - 1;
+      if (n_tiles > 0 && slot_ok[s] && lane == 0) {
+        const uint32_t idesc_qk = idesc_bf16_f32(kTileM, kTileN / 2, 0, 0);
         const uint32_t idesc_pv = idesc_bf16_f32(kTileM, D, 0, 1);
         // Descriptors are built once; every MMA then only adds a compile-time
         // offset (start address field, 16-byte units) to a base descriptor.
-        const uint64_t dq0 = sdesc_sw128(q_addr, 16, 1024);
-        const uint64_t dk0 = sdesc_sw128(ring_addr, 16, 1024);
-        const uint64_t dv0 = sdesc_sw128(ring_addr + NSTREAM * C::kTile, kChunkBytes, 1024);
+        const uint64_t dq = sdesc_sw128(q_addr, 16, 1024) + (uint64_t)s * (C::kTile >> 4);
+        const uint64_t dk0 = sdesc_sw128(ring_addr, 16, 1024) +
+                             (NSTREAM == 2 ? (uint64_t)s * (C::kTile >> 4) : 0ull);
+        const uint64_t dv0 = sdesc_sw128(ring_addr + NSTREAM * C::kTile, kChunkBytes, 1024) +
+                             (NSTREAM == 2 ? (uint64_t)s * (C::kTile >> 4) : 0ull);
         constexpr uint64_t kStageStep = C::kStageBytes >> 4;
-        constexpr uint64_t kTileStep = C::kTile >> 4;
-        const bool issuer = lane == 0;
-        auto qk = [&](int it, int s) {
-          const uint64_t dq = dq0 + (uint64_t)s * kTileStep;
-          const uint64_t dk = dk0 + (uint64_t)(it % kStages) * kStageStep +
-                              (NSTREAM == 2 ? (uint64_t)s * kTileStep : 0ull);
-          const uint32_t ts = tmem + 128u * s;
+        constexpr uint64_t kHalfRows = (64 * 128) >> 4;  // 64 K rows inside a 64-column chunk
+        const uint32_t tslot = tmem + 128u * s;
+        // S[:, 64 hf : 64 hf + 64] = Q_s K[64 hf : 64 hf + 64]^T of tile it
+        auto qk_half = [&](int it, int hf, uint64_t* done) {
+          const uint64_t dk = dk0 + (uint64_t)(it % kStages) * kStageStep + (uint64_t)hf * kHalfRows;
+          const uint32_t ts = tslot + 64u * hf;
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint64_t off = (uint64_t)(((k / 4) * kChunkBytes + (k % 4) * 32) >> 4);
             mma_ss(ts, dq + off, dk + off, idesc_qk, k > 0 ? 1u : 0u);
           }
-          tc_commit(&s_full[s]);
+          tc_commit(done);
         };
-        auto pv = [&](int it, int s) {
-          const uint64_t dv = dv0 + (uint64_t)(it % kStages) * kStageStep +
-                              (NSTREAM == 2 ? (uint64_t)s * kTileStep : 0ull);
-          const uint32_t to = tmem + 256u + 128u * s, ts = tmem + 128u * s;
+        // O_s += P_s V of tile it; P (bf16 pairs) sits in the columns of the
+        // early half e: keys of half e at [64 e, 64 e + 32), keys of the
+        // other half at [64 e + 32, 64 e + 64)
+        auto pv = [&](int it) {
+          const uint64_t dv = dv0 + (uint64_t)(it % kStages) * kStageStep;
+          const uint32_t to = tmem + 256u + 128u * s;
+          const uint32_t tp = tslot + 64u * (uint32_t)(it & 1);
+          const int odd = it & 1;
 #pragma unroll
-          for (int k = 0; k < kTileN / 16; ++k)
-            mma_ts(to, ts + k * 8, dv + (uint64_t)((k * 2048) >> 4), idesc_pv,
+          for (int k = 0; k < kTileN / 16; ++k) {
+            const uint32_t col = ((k / 4) != odd ? 32u : 0u) + 8u * (k % 4);
+            mma_ts(to, tp + col, dv + (uint64_t)((k * 2048) >> 4), idesc_pv,
                    (it > 0 || k > 0) ? 1u : 0u);
+          }
           tc_commit(&o_done[s]);
         };
-        // release 0: Q and K of tile 0 are in shared memory
-        bool ok = named_barrier_and(kBarIssue, 64, true);
+        bool ok = mbar_wait(full_q, 0, p.err, abort_flag) &&
+                  mbar_wait(&full_k[0], 0, p.err, abort_flag);
         tc_fence_after();
-        if (ok && issuer) {
-#pragma unroll
-          for (int s = 0; s < NSLOT; ++s)
-            if (slot_ok[s]) qk(0, s);
+        if (ok) {
+          qk_half(0, 0, &se_full[s]);
+          qk_half(0, 1, &sl_full[s]);
           tc_commit(&empty_k[0]);
         }
-        __syncwarp();
-        for (int it = 0; it < n_tiles; ++it) {
+        for (int it = 0; ok && it < n_tiles; ++it) {
           const int st = it % kStages;
           const bool more = it + 1 < n_tiles;
-#pragma unroll
-          for (int s = 0; s < NSLOT; ++s) {
-            if (!slot_ok[s]) continue;
-            // release: P of slot s (and, for the first slot, V of this tile
-            // and K of the next) are ready
-            ok = named_barrier_and(kBarIssue, 64, true) && ok;
+          const int e_next = (it + 1) & 1;  // early half of tile it + 1
+          if (more) {
+            // the softmax has read the late half of tile it; K of tile it + 1
+            if (!mbar_wait(&l_free[s], (uint32_t)it & 1u, p.err, abort_flag)) break;
+            if (!mbar_wait(&full_k[(it + 1) % kStages], (uint32_t)((it + 1) / kStages) & 1u,
+                           p.err, abort_flag))
+              break;
             tc_fence_after();
-            if (ok && issuer) {
-              pv(it, s);
-              if (more) qk(it + 1, s);
-            }
-            __syncwarp();
+            qk_half(it + 1, e_next, &se_full[s]);
           }
-          if (ok && issuer) {
-            tc_commit(&empty_v[st]);
-            if (more) tc_commit(&empty_k[(it + 1) % kStages]);
+          // P of tile it is in TMEM; V of tile it
+          if (!mbar_wait(&p_full[s], (uint32_t)it & 1u, p.err, abort_flag)) break;
+          if (!mbar_wait(&full_v[st], (uint32_t)(it / kStages) & 1u, p.err, abort_flag)) break;
+          tc_fence_after();
+          pv(it);
+          tc_commit(&empty_v[st]);
+          if (more) {
+            qk_half(it + 1, e_next ^ 1, &sl_full[s]);
+            tc_commit(&empty_k[(it + 1) % kStages]);
           }
-          __syncwarp();
         }
         // o_final completes once every MMA issued above has finished (also on
         // the abort path, so TMEM is quiescent before it is freed).
-        if (issuer) {
-          tc_commit(&o_final[0]);
-          tc_commit(&o_final[1]);
-        }
-        __syncwarp();
+        tc_commit(&o_final[s]);
       }
-    } else if (warp == 2) {
-      // ============================ waiter ============================
-      // Mirrors the issuer's releases one for one.  After a failed wait
-      // (error recorded, abort set) it stops waiting but keeps releasing,
-      // so both warps always pass the same number of named barriers.
-      if (n_tiles > 0) {
-        bool ok = mbar_wait(full_q, 0, p.err, abort_flag) &&
-                  mbar_wait(&full_k[0], 0, p.err, abort_flag);
-        ok = named_barrier_and(kBarIssue, 64, ok);
-        for (int it = 0; it < n_tiles; ++it) {
-          const int st = it % kStages;
-          const bool more = it + 1 < n_tiles;
-          bool first = true;
-#pragma unroll
-          for (int s = 0; s < NSLOT; ++s) {
-            if (!slot_ok[s]) continue;
-            if (ok && first)
-              ok = mbar_wait(&full_v[st], (uint32_t)(it / kStages) & 1u, p.err, abort_flag);
-            if (ok) ok = mbar_wait(&p_full[s], (uint32_t)it & 1u, p.err, abort_flag);
-            if (ok && first && more)
-              ok = mbar_wait(&full_k[(it + 1) % kStages], (uint32_t)((it + 1) / kStages) & 1u,
-                             p.err, abort_flag);
-            first = false;
-            ok = named_barrier_and(kBarIssue, 64, ok);
-          }
-        }
-      }
+      __syncwarp();
     }
   } else {
     // ============================ softmax ============================
@@ -396,10 +371,11 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     bool ok = slot_ok[slot];
 
     float m_pend = -INFINITY;  // max seen but not yet adopted (adopted next tile)
+    int int_lo, int_hi;        // key tiles that need no element mask
+    interior_tiles(g, Mv, qt, &int_lo, &int_hi);
 
-    // 64 score columns [64 hf, 64 hf + 64) of tile `it`, masked on edge and
-    // global tiles (-inf outside the row's key set).
-    auto load_half = [&](int it, int hf, bool edge, float (&sv)[64]) {
+    // the 64 score columns of key half hf (TMEM -> registers)
+    auto read_half = [&](int hf, float (&sv)[64]) {
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
         uint32_t v[32];
@@ -408,8 +384,11 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
         for (int e = 0; e < 32; ++e) sv[jj * 32 + e] = __uint_as_float(v[e]);
       }
       tmem_wait_ld();
-      // keep-mask of the half's 64 keys (bit j: key j is in the row's key
-      // set), applied by one shared select loop
+    };
+    // -inf outside the row's key set, on edge and global tiles: a keep-mask
+    // of the half's 64 keys (bit j: key j is in the set) applied by one
+    // shared select loop
+    auto mask_half = [&](int it, int hf, bool edge, float (&sv)[64]) {
       uint64_t keep = ~0ull;
       if (it < n_band) {
         if (edge) {
@@ -449,11 +428,11 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
         for (int e = 0; e < 8; ++e) t[e] = max3f(t[e], sv[j + e], sv[j + 8 + e]);
       return max3f(max3f(t[0], t[1], t[2]), max3f(t[3], t[4], t[5]), fmaxf(t[6], t[7]));
     };
-    // P = 2^(s * scale * log2 e - m_ref) for one half, stored as bf16 pairs
-    // over the half's S columns.  Three of every four column pairs go to the
-    // MUFU ex2 unit and one to the FMA pipe (polynomial), so the two softmax
-    // warpgroups of the SM do not saturate MUFU.
-    auto exp_half = [&](int hf, const float (&sv)[64], float m_ref, float2 (&ls)[4]) {
+    // P = 2^(s * scale * log2 e - m_ref) for one key half, stored as 32
+    // columns of bf16 pairs from TMEM column pcol.  Three of every four
+    // column pairs go to the MUFU ex2 unit and one to the FMA pipe
+    // (polynomial), so the two softmax warpgroups do not saturate MUFU.
+    auto exp_half = [&](int pcol, const float (&sv)[64], float m_ref, float2 (&ls)[4]) {
       const float2 sl2_2 = make_float2(sl2, sl2), negm2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
       for (int jj = 0; jj < 2; ++jj) {
@@ -472,11 +451,11 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
           ls[e & 3] = add2(ls[e & 3], pr);
           pk[e] = pack_bf16x2(pr.x, pr.y);
         }
-        tmem_st16(tS + hf * 32 + jj * 16, pk);
+        tmem_st16(tS + pcol + jj * 16, pk);
       }
     };
     // Multiplies O (and l) by 2^(m_from - m_to) and adopts m_to; O holds
-    // P_0..P_{it-1} V, whose MMA finished before S of tile it was produced.
+    // P_0..P_{it-1} V, whose MMAs are complete once o_done says so.
     auto rescale_o = [&](int it, bool mine, float m_to) -> bool {
       const bool o_ok = mbar_wait(&o_done[slot], (uint32_t)(it - 1) & 1u, p.err, abort_flag);
       if (!__all_sync(0xffffffffu, o_ok)) return false;
@@ -497,11 +476,17 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
       return true;
     };
 
+    // Scores are exponentiated against the running max as it stands (a row
+    // without keys so far adopts the max of the half at hand; its O and l
+    // are still zero), and the tile max is tracked on the way.  Scores
+    // above the running max only enlarge P, by at most 2^64 (safe in fp32
+    // and bf16); a larger jump is adopted at once by rescaling O, l, the
+    // partial sums and the P already written.
     for (int it = 0; ok && it < n_tiles; ++it) {
-      const bool w_ok = mbar_wait(&s_full[slot], (uint32_t)it & 1u, p.err, abort_flag);
-      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-      tc_fence_after();
-      const bool edge = it < n_band && !tile_interior(g, Mv, qt, tr.kv_begin + it);
+      const int e = it & 1;  // early key half; P of the tile lives in its columns
+      const uint32_t ph = (uint32_t)it & 1u;
+      const int t_kv = tr.kv_begin + it;
+      const bool edge = it < n_band && !(t_kv >= int_lo && t_kv <= int_hi);
 
       // adopt a larger max seen on the previous tile (rare after the start)
       const bool pend = m_pend > m_used;
@@ -511,68 +496,61 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
 
       float2 ls[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                       make_float2(0.f, 0.f)};
-      // TMEM columns of this slot: S half 0 at [0, 64), S half 1 at [64, 128);
-      // P (bf16 pairs) of half 0 goes to [0, 32) and of half 1 to [32, 64),
-      // so S is never read after its columns have been overwritten.
-      float tmax;
       float sv[64];
-      if (!__any_sync(0xffffffffu, m_used == -INFINITY)) {
-        // Fast path: exponentiate against the current max in one pass and
-        // track the tile max on the way.  Scores above the current max only
-        // enlarge P (by at most 2^64 here, safe in fp32 and bf16).
-        load_half(it, 0, edge, sv);
-        tmax = half_max(sv);
-        if (__any_sync(0xffffffffu, tmax * sl2 > m_used + 64.f)) {
-          // a large jump in half 0: adopt the new max before any P exists
-          const bool up = tmax * sl2 > m_used;
-          if (!rescale_o(it, up, fmaxf(m_used, tmax * sl2))) { ok = false; break; }
-        }
-        exp_half(0, sv, m_used, ls);
-        load_half(it, 1, edge, sv);
-        const float tmax1 = half_max(sv);
-        tmax = fmaxf(tmax, tmax1);
-        const bool jump = tmax1 * sl2 > m_used + 64.f;
+
+      // ---- early half
+      bool w_ok = mbar_wait(&se_full[slot], ph, p.err, abort_flag);
+      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+      tc_fence_after();
+      read_half(e, sv);
+      mask_half(it, e, edge, sv);
+      float tmax = half_max(sv);
+      {
+        const bool adopt = m_used == -INFINITY;
+        const bool jump = !adopt && tmax * sl2 > m_used + 64.f;
+        if (adopt) m_used = tmax * sl2;
         if (__any_sync(0xffffffffu, jump)) {
-          // a large jump in half 1: rescale O, l, the partial sums and the
-          // bf16 P of half 0 already in TMEM to the new max
+          if (!rescale_o(it, jump, fmaxf(m_used, tmax * sl2))) { ok = false; break; }
+        }
+      }
+      exp_half(64 * e, sv, m_used == -INFINITY ? 0.f : m_used, ls);
+
+      // ---- late half
+      w_ok = mbar_wait(&sl_full[slot], ph, p.err, abort_flag);
+      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+      tc_fence_after();
+      read_half(e ^ 1, sv);
+      // these columns now belong to the early half of the next tile
+      tc_fence_before();
+      mbar_arrive(&l_free[slot]);
+      mask_half(it, e ^ 1, edge, sv);
+      const float tmax1 = half_max(sv);
+      tmax = fmaxf(tmax, tmax1);
+      {
+        const bool adopt = m_used == -INFINITY;
+        const bool jump = !adopt && tmax1 * sl2 > m_used + 64.f;
+        if (adopt) m_used = tmax1 * sl2;
+        if (__any_sync(0xffffffffu, jump)) {
           const float m_old = m_used;
           if (!rescale_o(it, jump, fmaxf(m_used, tmax1 * sl2))) { ok = false; break; }
           const float f = jump ? ex2_approx(m_old - m_used) : 1.f;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) ls[e] = make_float2(ls[e].x * f, ls[e].y * f);
+          for (int j = 0; j < 4; ++j) ls[j] = make_float2(ls[j].x * f, ls[j].y * f);
           uint32_t v[32];
           tmem_wait_st();
-          tmem_ld32(tS, v);
+          tmem_ld32(tS + 64 * e, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            v[e] = pack_bf16x2(__uint_as_float(v[e] << 16) * f,
-                               __uint_as_float(v[e] & 0xFFFF0000u) * f);
-          tmem_st32(tS, v);
+          for (int j = 0; j < 32; ++j)
+            v[j] = pack_bf16x2(__uint_as_float(v[j] << 16) * f,
+                               __uint_as_float(v[j] & 0xFFFF0000u) * f);
+          tmem_st32(tS + 64 * e, v);
         }
-        exp_half(1, sv, m_used, ls);
-      } else {
-        // Some row has no key yet: find the tile max first (one pass over
-        // the scores), then exponentiate (a second pass).
-        load_half(it, 1, edge, sv);
-        tmax = half_max(sv);
-        load_half(it, 0, edge, sv);
-        tmax = fmaxf(tmax, half_max(sv));
-        const float m_new = fmaxf(m_used, tmax * sl2);
-        const bool up = m_new > m_used;
-        if (it > 0 && __any_sync(0xffffffffu, up)) {
-          if (!rescale_o(it, up, m_new)) { ok = false; break; }
-        } else if (up) {
-          m_used = m_new;
-        }
-        const float m_safe = m_used == -INFINITY ? 0.f : m_used;
-        exp_half(0, sv, m_safe, ls);
-        load_half(it, 1, edge, sv);
-        exp_half(1, sv, m_safe, ls);
       }
+      exp_half(64 * e + 32, sv, m_used == -INFINITY ? 0.f : m_used, ls);
       {
-        const float2 a = add2(add2(ls[0], ls[1]), add2(ls[2], ls[3]));
-        l += a.x + a.y;
+        const float2 a2 = add2(add2(ls[0], ls[1]), add2(ls[2], ls[3]));
+        l += a2.x + a2.y;
       }
       // a max that grew by more than 2^8 is adopted before the next tile
       if (tmax * sl2 > m_used + kRescaleThreshold) m_pend = tmax * sl2;
@@ -610,11 +588,12 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
   }
 
   // ---- teardown: make sure no MMA is in flight, then free TMEM.
-  if (warp == 1 && lane == 0 && n_tiles > 0 && *abort_flag) {
-    // abort path: o_final was committed after the last issued MMA; give it
-    // a bounded chance to land before TMEM is released.
+  if (warp >= 1 && warp <= NSLOT && lane == 0 && n_tiles > 0 && slot_ok[warp - 1] &&
+      *abort_flag) {
+    // abort path: o_final was committed after the last MMA this issuer
+    // issued; give it a bounded chance to land before TMEM is released.
     volatile int no_abort = 0;
-    mbar_wait(&o_final[0], 0, nullptr, &no_abort, 100000000ull);
+    mbar_wait(&o_final[warp - 1], 0, nullptr, &no_abort, 100000000ull);
   }
   tc_fence_before();
   __syncthreads();

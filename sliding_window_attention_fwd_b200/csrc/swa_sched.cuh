@@ -123,17 +123,23 @@ SWA_HD TileRange tile_range(const Geometry& g, int Mv, int qt) {
   return r;
 }
 
-// True when every (row, key) pair of (query tile qt, kv tile t) is inside
-// the window and in range, so the tile needs no element mask.
-SWA_HD bool tile_interior(const Geometry& g, int Mv, int qt, int t) {
-  int m0 = qt * kTileM;
-  int m1 = m0 + kTileM - 1;
-  int n0 = t * kTileN;
-  int n1 = n0 + kTileN - 1;
-  if (m1 > Mv - 1 || n1 > Mv - 1) return false;
-  if (key_lo(g, m1) > n0) return false;
-  if (key_hi(g, m0, Mv) < n1) return false;
-  return true;
+// KV tiles [*lo, *hi] of query tile qt whose every (row, key) pair is inside
+// the window and in range, so they need no element mask (empty when
+// *lo > *hi).  Key bounds are monotone in the row, so the keys every row of
+// the tile sees are [key_lo(last row), key_hi(first row)], and those tiles
+// form one contiguous run.
+SWA_HD void interior_tiles(const Geometry& g, int Mv, int qt, int* lo, int* hi) {
+  const int m0 = qt * kTileM;
+  const int m1 = m0 + kTileM - 1;
+  *lo = 1;
+  *hi = 0;
+  if (m1 > Mv - 1) return;
+  int a = key_lo(g, m1);
+  if (a < 0) a = 0;
+  int b = key_hi(g, m0, Mv);
+  if (b > Mv - 1) b = Mv - 1;
+  *lo = (a + kTileN - 1) / kTileN;
+  *hi = (b + 1) / kTileN - 1;
 }
 
 }  // namespace swa
