@@ -17,11 +17,18 @@
 //   warp 0     producer: TMA loads of the Q tiles once and of the K/V tiles
 //              into a shared-memory ring (128-byte swizzle); global keys are
 //              gathered with plain 16-byte loads into the same layout;
-//   warp 1     TMEM owner (512 columns) and the single MMA-issuing thread:
-//                S_s  = Q_s K^T     tcgen05.mma, operands in smem, fp32 in TMEM
+//   warp 1 + s MMA issuer of slot s (warp 1 also owns the 512 TMEM columns):
+//                S_s  = Q_s K^T     tcgen05.mma, operands in smem, fp32 in
+//                                   TMEM, in two 64-key halves
 //                O_s += P_s V       tcgen05.mma, P (bf16) read from TMEM where
 //                                   it overwrote S_s, V from smem
-//              issued in the order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1);
+//              Tile j's P is kept in the columns of its early half (j & 1);
+//              the early half of tile j+1 goes to the other columns as soon
+//              as the softmax has read them, so it is ready when the softmax
+//              finishes tile j, and only the late half waits for PV(j).  One
+//              issuer per slot, each on its own SM sub-partition: a single
+//              issuer sharing a sub-partition with two busy softmax warps
+//              gets too few issue slots to keep the tensor core fed;
 //   softmax    thread t of warpgroup 1+s owns query row t of slot s: row max
 //              and row sum are thread-local tree reductions, no shuffles.
 //              Element masks only on tiles the scheduler marks as edges.
