@@ -398,7 +398,7 @@ def run_ours(args, rank, world, local_rank):
             "gpu_launches": args.steps,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                          "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-                         "traffic": captured_traffic("swa_fwd_sm100_kernel<128>"),
+                         "traffic": captured_traffic("swa_fwd_sm100_kernel<128,2,1>"),
                          "peak_source": peak_src,
                          "algorithmic_bytes": alg_bytes},
             "clocks": clk.summary(t_timed0, t_timed1),
