@@ -49,6 +49,12 @@ def _load():
         lib.oracle_forward.restype = None
         lib.oracle_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, ctypes.c_double, I]
         lib.oracle_decode.restype = None
+        lib.oracle_decode_paged.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I,
+                                            ctypes.c_double, I]
+        lib.oracle_decode_paged.restype = None
+        lib.oracle_append.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I,
+                                      ctypes.c_double, I]
+        lib.oracle_append.restype = None
         _lib = lib
     return _lib
 
@@ -127,4 +133,51 @@ def decode(q, k_ring, v_ring, pos, scale=None, threads=None):
     lse = np.zeros((B, H), dtype=np.float64)
     lib.oracle_decode(_ptr(q), _ptr(kr), _ptr(vr), _ptr(pos), _ptr(out), _ptr(lse),
                       B, H, Hkv, D, W, float(scale), int(threads or default_threads()))
+    return out, lse
+
+
+def _i64(a) -> np.ndarray:
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int64))
+
+
+def decode_paged(q, k_pages, v_pages, block_table, pos, page_size, W, scale=None, threads=None):
+    """fp64 paged decode.  q [B,H,D]; k_pages/v_pages [rows,Hkv,D] with rows a
+    multiple of page_size; block_table [B,max_pages] int32 (logical page ->
+    physical page); pos [B].  Returns (out [B,H,D], lse [B,H])."""
+    lib = _load()
+    q, kp, vp = _f32(q), _f32(k_pages), _f32(v_pages)
+    if hasattr(block_table, "detach"):
+        block_table = block_table.detach().cpu().numpy()
+    table = np.ascontiguousarray(np.asarray(block_table, dtype=np.int32))
+    pos = _i64(pos)
+    B, H, D = q.shape
+    Hkv = kp.shape[1]
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    out = np.zeros((B, H, D), dtype=np.float64)
+    lse = np.zeros((B, H), dtype=np.float64)
+    lib.oracle_decode_paged(_ptr(q), _ptr(kp), _ptr(vp), _ptr(table), _ptr(pos), _ptr(out),
+                            _ptr(lse), B, H, Hkv, D, int(page_size), table.shape[1], int(W),
+                            float(scale), int(threads or default_threads()))
+    return out, lse
+
+
+def append(q, k_ring, v_ring, k_new, v_new, pos0, scale=None, threads=None):
+    """fp64 chunked append.  q [B,C,H,D]; k_ring/v_ring [B,W,Hkv,D] (the cache
+    before the chunk); k_new/v_new [B,C,Hkv,D]; pos0 [B] = position of the
+    chunk's first token.  Returns (out [B,C,H,D], lse [B,H,C])."""
+    lib = _load()
+    q, kr, vr, kn, vn = _f32(q), _f32(k_ring), _f32(v_ring), _f32(k_new), _f32(v_new)
+    pos0 = _i64(pos0)
+    B, C, H, D = q.shape
+    W, Hkv = kr.shape[1], kr.shape[2]
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    out = np.zeros((B, C, H, D), dtype=np.float64)
+    lse = np.zeros((B, H, C), dtype=np.float64)
+    lib.oracle_append(_ptr(q), _ptr(kr), _ptr(vr), _ptr(kn), _ptr(vn), _ptr(pos0), _ptr(out),
+                      _ptr(lse), B, C, H, Hkv, D, W, float(scale),
+                      int(threads or default_threads()))
     return out, lse

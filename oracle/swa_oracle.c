@@ -262,6 +262,147 @@ void oracle_decode(const float* q, const float* k_ring, const float* v_ring,
   free(jobs);
 }
 
+/*
+ * Paged decode oracle ("空洞滑窗机制" page, §四, KV cache management with
+ * PagedAttention: the cache lives in fixed-size pages found through a block
+ * table, and pages that fall out of the window can be released).  Token t
+ * of sequence b sits in row block_table[b * max_pages + t / page_size] *
+ * page_size + t % page_size of k_pages / v_pages ([rows, Hkv, D]).  The new
+ * token at pos attends positions [max(0, pos - W + 1), pos] (the same key
+ * set as the ring decode).  q [B,H,D]; out [B,H,D], lse [B,H].
+ */
+typedef struct {
+  const float *q, *kp, *vp;
+  const int32_t* table;
+  const int64_t* pos;
+  double *out, *lse;
+  int B, H, Hkv, D, ps, max_pages, W;
+  double scale;
+  int tid, nthreads;
+} paged_job;
+
+static void* paged_worker(void* arg) {
+  paged_job* J = (paged_job*)arg;
+  int* keys = (int*)malloc(sizeof(int) * (size_t)J->W);
+  double* s = (double*)malloc(sizeof(double) * (size_t)J->W);
+  int grp = J->H / J->Hkv;
+  for (int64_t r = J->tid; r < (int64_t)J->B * J->H; r += J->nthreads) {
+    int b = (int)(r / J->H), h = (int)(r % J->H), g = h / grp;
+    int64_t p = J->pos[b];
+    int64_t first = p - J->W + 1 < 0 ? 0 : p - J->W + 1;
+    int nk = 0;
+    for (int64_t t = first; t <= p; ++t) {
+      int64_t page = J->table[(int64_t)b * J->max_pages + t / J->ps];
+      keys[nk++] = (int)(page * J->ps + t % J->ps);
+    }
+    const float* qrow = J->q + ((long)b * J->H + h) * J->D;
+    attend(qrow, J->kp + (long)g * J->D, J->vp + (long)g * J->D, (long)J->Hkv * J->D, keys, nk,
+           J->D, J->scale, s, J->out + r * J->D, J->lse + r);
+  }
+  free(keys);
+  free(s);
+  return NULL;
+}
+
+void oracle_decode_paged(const float* q, const float* k_pages, const float* v_pages,
+                         const int32_t* block_table, const int64_t* pos, double* out,
+                         double* lse, int B, int H, int Hkv, int D, int page_size,
+                         int max_pages, int W, double scale, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  paged_job* jobs = (paged_job*)malloc(sizeof(paged_job) * (size_t)nthreads);
+  for (int t = 0; t < nthreads; ++t) {
+    paged_job J = {q, k_pages, v_pages, block_table, pos, out, lse, B, H, Hkv, D,
+                   page_size, max_pages, W, scale, t, nthreads};
+    jobs[t] = J;
+    pthread_create(&th[t], NULL, paged_worker, &jobs[t]);
+  }
+  for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+  free(th);
+  free(jobs);
+}
+
+/*
+ * Chunked append oracle (aiqz.cc page, "推理优化策略": streaming inference
+ * reads new tokens while computing and drops what leaves the window;
+ * "大模型窗口扩展技术" page §3.1: position t lives in ring slot t % W).
+ * C new tokens of sequence b take positions pos0[b] .. pos0[b] + C - 1.
+ * Query c (position p = pos0 + c) attends positions [max(0, p - W + 1), p];
+ * position t's key and value are the new token t - pos0 when t >= pos0,
+ * else ring slot t % W of the cache as it was before the chunk.
+ * q [B,C,H,D], k_ring / v_ring [B,W,Hkv,D], k_new / v_new [B,C,Hkv,D];
+ * out [B,C,H,D], lse [B,H,C].
+ */
+typedef struct {
+  const float *q, *kr, *vr, *kn, *vn;
+  const int64_t* pos0;
+  double *out, *lse;
+  int B, C, H, Hkv, D, W;
+  double scale;
+  int tid, nthreads;
+} app_job;
+
+static void* app_worker(void* arg) {
+  app_job* J = (app_job*)arg;
+  const int D = J->D;
+  float* kb = (float*)malloc(sizeof(float) * (size_t)J->W * D);
+  float* vb = (float*)malloc(sizeof(float) * (size_t)J->W * D);
+  int* keys = (int*)malloc(sizeof(int) * (size_t)J->W);
+  double* s = (double*)malloc(sizeof(double) * (size_t)J->W);
+  int grp = J->H / J->Hkv;
+  for (int64_t r = J->tid; r < (int64_t)J->B * J->C * J->H; r += J->nthreads) {
+    int h = (int)(r % J->H);
+    int c = (int)((r / J->H) % J->C);
+    int b = (int)(r / ((int64_t)J->H * J->C));
+    int g = h / grp;
+    int64_t p = J->pos0[b] + c;
+    int64_t first = p - J->W + 1 < 0 ? 0 : p - J->W + 1;
+    int nk = 0;
+    for (int64_t t = first; t <= p; ++t) {
+      const float *ks, *vs;
+      if (t >= J->pos0[b]) {
+        long row = ((long)b * J->C + (t - J->pos0[b])) * J->Hkv + g;
+        ks = J->kn + row * D;
+        vs = J->vn + row * D;
+      } else {
+        long row = ((long)b * J->W + t % J->W) * J->Hkv + g;
+        ks = J->kr + row * D;
+        vs = J->vr + row * D;
+      }
+      memcpy(kb + (size_t)nk * D, ks, sizeof(float) * (size_t)D);
+      memcpy(vb + (size_t)nk * D, vs, sizeof(float) * (size_t)D);
+      keys[nk] = nk;
+      ++nk;
+    }
+    const float* qrow = J->q + r * D;
+    int64_t li = ((int64_t)b * J->H + h) * J->C + c;
+    attend(qrow, kb, vb, D, keys, nk, D, J->scale, s, J->out + r * D, J->lse + li);
+  }
+  free(kb);
+  free(vb);
+  free(keys);
+  free(s);
+  return NULL;
+}
+
+void oracle_append(const float* q, const float* k_ring, const float* v_ring,
+                   const float* k_new, const float* v_new, const int64_t* pos0, double* out,
+                   double* lse, int B, int C, int H, int Hkv, int D, int W, double scale,
+                   int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  app_job* jobs = (app_job*)malloc(sizeof(app_job) * (size_t)nthreads);
+  for (int t = 0; t < nthreads; ++t) {
+    app_job J = {q, k_ring, v_ring, k_new, v_new, pos0, out, lse, B, C, H, Hkv, D, W, scale,
+                 t, nthreads};
+    jobs[t] = J;
+    pthread_create(&th[t], NULL, app_worker, &jobs[t]);
+  }
+  for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+  free(th);
+  free(jobs);
+}
+
 #ifdef __cplusplus
 }
 #endif
