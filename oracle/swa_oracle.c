@@ -354,18 +354,18 @@ static void* app_worker(void* arg) {
     int h = (int)(r % J->H);
     int c = (int)((r / J->H) % J->C);
     int b = (int)(r / ((int64_t)J->H * J->C));
-    int g = h / grp;
+    int kvh = h / grp;
     int64_t p = J->pos0[b] + c;
     int64_t first = p - J->W + 1 < 0 ? 0 : p - J->W + 1;
     int nk = 0;
     for (int64_t t = first; t <= p; ++t) {
       const float *ks, *vs;
       if (t >= J->pos0[b]) {
-        long row = ((long)b * J->C + (t - J->pos0[b])) * J->Hkv + g;
+        long row = ((long)b * J->C + (t - J->pos0[b])) * J->Hkv + kvh;
         ks = J->kn + row * D;
         vs = J->vn + row * D;
       } else {
-        long row = ((long)b * J->W + t % J->W) * J->Hkv + g;
+        long row = ((long)b * J->W + t % J->W) * J->Hkv + kvh;
         ks = J->kr + row * D;
         vs = J->vr + row * D;
       }

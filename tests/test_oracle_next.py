@@ -147,8 +147,8 @@ MUTANTS = {
     "paged_window_one_short": ("for (int64_t t = first; t <= p; ++t) {\n      int64_t page",
                                "for (int64_t t = first + 1; t <= p; ++t) {\n      int64_t page"),
     "append_first_new_from_ring": ("if (t >= J->pos0[b]) {", "if (t > J->pos0[b]) {"),
-    "append_slot_from_position": ("long row = ((long)b * J->W + t % J->W) * J->Hkv + g;",
-                                  "long row = ((long)b * J->W + (t + 1) % J->W) * J->Hkv + g;"),
+    "append_slot_from_position": ("long row = ((long)b * J->W + t % J->W) * J->Hkv + kvh;",
+                                  "long row = ((long)b * J->W + (t + 1) % J->W) * J->Hkv + kvh;"),
 }
 
 
