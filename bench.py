@@ -351,6 +351,74 @@ def run_ours(args, rank, world, local_rank):
                            "peak_source": peak_src}}
     del dq, dk, dv
 
+    # ---- paged decode: the ring_decode shapes with the cache in 256-row pages
+    pcfg = inputs.PAGED_CONFIGS["paged_decode"]
+    pq, pkp, pvp, ptab, ppos = inputs.paged_inputs(pcfg, device=dev)
+    ptab, ppos = ptab.to(dev), ppos.to(dev)
+    pout = torch.empty_like(pq)
+    pstep = lambda: swa.swa_decode_paged(pq, pkp, pvp, ptab, ppos, pcfg.page_size, pcfg.W,
+                                         out=pout, stream=stream)
+    pms = time_device(pstep, args.steps, args.warmup, flush, stream)
+    p_ms = sum(pms) / len(pms)
+    pvalid = torch.clamp(ppos + 1, max=pcfg.W)
+    p_bytes = int(pvalid.sum().item()) * pcfg.Hkv * pcfg.D * 2 * 2 + 2 * pq.numel() * 2
+    paged = {"workload": pcfg.name, "ms": p_ms, "gbs": p_bytes / p_ms / 1e6,
+             "roofline": {"bound": "hbm", "achieved": p_bytes / p_ms / 1e6,
+                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": p_bytes / p_ms / 1e6 / peaks["hbm_gbs"], "traffic": None,
+                          "peak_source": peak_src}}
+    del pq, pkp, pvp
+
+    # ---- chunked append: 64-token chunks entering a 4096-slot ring
+    acfg = inputs.APPEND_CONFIGS["ring_append"]
+    aq, akn, avn, akr, avr, apos = inputs.append_inputs(acfg, device=dev)
+    apos = apos.to(dev)
+    aout = torch.empty_like(aq)
+    # every step appends the same chunk at the same positions: the ring is
+    # updated in place, so later steps read other values but do the same work
+    astep = lambda: swa.swa_append(aq, akn, avn, akr, avr, apos, out=aout, stream=stream)
+    ams = time_device(astep, args.steps, args.warmup, flush, stream)
+    a_ms = sum(ams) / len(ams)
+    a_pairs = acfg.H * sum(min(acfg.W, int(p0) + c + 1)
+                           for p0 in apos.tolist() for c in range(acfg.C))
+    a_flops = 4.0 * acfg.D * a_pairs
+    a_bytes = (acfg.B * min(acfg.W, acfg.C + acfg.W) * acfg.Hkv * acfg.D * 2 * 2
+               + (aq.numel() + aout.numel() + 2 * akn.numel()) * 2)
+    alu_peak = 2.0 * 128 * 148 * 1.965e9 / 1e12  # fp32 FMA lanes x SMs x max clock
+    append = {"workload": acfg.name, "ms": a_ms, "tflops": a_flops / a_ms / 1e9,
+              "gbs": a_bytes / a_ms / 1e6,
+              "roofline": {"bound": "alu", "achieved": a_flops / a_ms / 1e9, "peak": alu_peak,
+                           "unit": "TFLOP/s", "frac": a_flops / a_ms / 1e9 / alu_peak,
+                           "traffic": None, "peak_source": "derived (fp32 FMA rate)"}}
+    del aq, akn, avn, akr, avr
+
+    # ---- a hybrid per-layer schedule on the prefill shapes: plain causal
+    # windows below, growing dilation in the middle, a full causal layer every
+    # four layers and attention-sink tokens; each layer has its own tensors
+    sched = [(4095, 0, 1, ()), (4095, 0, 1, ()), (2047, 0, 2, ()), (-1, 0, 1, ()),
+             (1023, 0, 4, ()), (511, 0, 8, ()), (4095, 0, 1, (0, 1, 2, 3)), (-1, 0, 1, ())]
+    lay = []
+    for li, (L_, R_, d_, G_) in enumerate(sched):
+        lq = inputs.normal((cfg.B, cfg.N, cfg.H, cfg.D), 3000 + li, 0, torch.bfloat16, dev)
+        lk = inputs.normal((cfg.B, cfg.N, cfg.Hkv, cfg.D), 3000 + li, 1, torch.bfloat16, dev)
+        lv = inputs.normal((cfg.B, cfg.N, cfg.Hkv, cfg.D), 3000 + li, 2, torch.bfloat16, dev)
+        lay.append(dict(q=lq, k=lk, v=lv, out=torch.empty_like(lq),
+                        lse=torch.empty(cfg.B, cfg.H, cfg.N, device=dev), win_left=L_,
+                        win_right=R_, dilation=d_,
+                        global_idx=(torch.tensor(G_, dtype=torch.int32, device=dev) if G_
+                                    else None)))
+    lstep = lambda: swa.swa_forward_layers(lay, stream=stream)
+    lms = time_device(lstep, max(1, args.steps // 8), args.warmup, flush, stream)
+    l_ms = sum(lms) / len(lms)
+    l_flops = sum(4.0 * cfg.D * in_window_pairs(cfg.N, L_, R_, d_, 0, G_, cfg.B, cfg.H)
+                  for L_, R_, d_, G_ in sched)
+    layers = {"workload": "hybrid 8-layer schedule on mistral_causal_prefill shapes",
+              "layers": [{"win_left": L_, "win_right": R_, "dilation": d_, "global": list(G_)}
+                         for L_, R_, d_, G_ in sched],
+              "ms": l_ms, "tflops": l_flops / l_ms / 1e9,
+              "frac_tensor": l_flops / l_ms / 1e9 / peaks["bf16_tflops"]}
+    del lay
+
     # ---- the other forward workloads (parity cases; reported for context)
     others = {}
     for name in ("longformer_global", "dilated_token", "dilated_block"):
@@ -403,6 +471,9 @@ def run_ours(args, rank, world, local_rank):
                          "algorithmic_bytes": alg_bytes},
             "clocks": clk.summary(t_timed0, t_timed1),
             "decode": decode,
+            "paged_decode": paged,
+            "append": append,
+            "layers": layers,
             "others": others,
         }
         if not args.no_cpu_baseline:

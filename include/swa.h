@@ -110,6 +110,38 @@ SWA_API int swa_forward_ex(const void* q, const void* k, const void* v, void* ou
                            int n_global, float scale, void* stream);
 
 /*
+ * One layer of a per-layer window schedule (see swa_forward_layers).  Every
+ * field means what the argument of the same name means for swa_forward_ex.
+ */
+typedef struct swa_layer {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;
+  int win_left;
+  int win_right;
+  int dilation;
+  int dilation_block;
+  const int32_t* global_idx;
+  int n_global;
+  float scale;
+} swa_layer;
+
+/*
+ * swa_forward_layers -- swa_forward_ex for each of n_layers layers, in
+ * order, on `stream` ("空洞滑窗机制" page, §三: models mix plain windows in
+ * the lower layers, growing dilation in the middle ones and a global layer
+ * every few layers or a few always-visible "attention sink" tokens).  All
+ * layers share B, H, Hkv, N, D; each brings its own tensors, window,
+ * dilation, global tokens and scale.  Every layer is validated before the
+ * first launch: on an invalid layer nothing is launched, its index is
+ * stored in *bad_layer (if not NULL) and its status is returned.
+ */
+SWA_API int swa_forward_layers(const swa_layer* layers, int n_layers, int B, int H, int Hkv,
+                               int N, int D, int* bad_layer, void* stream);
+
+/*
  * swa_forward_f32 -- the same operation in fp32 (q, k, v, out are float*),
  * computed with fp32 FFMA on CUDA cores (no TF32), for callers that need
  * fp32 accuracy.  D in {32, 64, 96, 128}; any dilation_block >= 0.
@@ -178,6 +210,61 @@ SWA_API int swa_decode_noalloc(const void* q, const void* k_ring, const void* v_
 /* swa_decode_noalloc_scratch_bytes -- size of swa_decode_noalloc's fixed
    device array, per GPU. */
 SWA_API size_t swa_decode_noalloc_scratch_bytes(void);
+
+/*
+ * swa_decode_paged -- swa_decode over a paged KV cache ("空洞滑窗机制"
+ * page, §四: the cache is managed in PagedAttention-style pages, and pages
+ * that fall out of the window can be released).
+ *   k_pages, v_pages  [num_pages * page_size, Hkv, D] bf16, device: the page
+ *                     pool; page p holds rows [p * page_size, (p+1) * page_size)
+ *   block_table       [B, max_pages] int32, device: token t of sequence b is
+ *                     row t % page_size of page block_table[b, t / page_size]
+ *   pos               [B] int64, device: position of the new token (>= 0);
+ *                     its k/v are already in the pool
+ *   q, out            [B, H, D] bf16; lse [B, H] fp32 natural log (may be NULL)
+ * The query attends positions max(0, pos-W+1) .. pos.  Only table entries
+ * for those positions are read; an entry outside [0, num_pages), or a
+ * logical page >= max_pages, reads as zero keys (a caller error, never an
+ * out-of-bounds access).  page_size must be a positive multiple of 64;
+ * D in {64, 128}; H % Hkv == 0, H / Hkv <= 8; scale <= 0 means 1/sqrt(D).
+ * Workspace, streams and graphs as for swa_decode.
+ */
+SWA_API int swa_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* out,
+                             float* lse, const int32_t* block_table, const int64_t* pos, int B,
+                             int H, int Hkv, int D, int page_size, int num_pages, int max_pages,
+                             int W, float scale, void* stream);
+
+/*
+ * swa_paged_window -- host-only: the logical pages [*first_page,
+ * *last_page] that a decode at `pos` with window W reads; every page below
+ * *first_page has left the window and can be returned to the pool (and
+ * stays out: later tokens only move the window forward).  Returns
+ * SWA_ERR_ARG for pos < 0, W < 1 or page_size < 1.
+ */
+SWA_API int swa_paged_window(int64_t pos, int W, int page_size, int64_t* first_page,
+                             int64_t* last_page);
+
+/*
+ * swa_append -- a chunk of C new tokens per sequence enters a ring-buffer
+ * KV cache (aiqz.cc page, "推理优化策略": streaming inference; page
+ * "大模型窗口扩展技术" §3.1: position t lives in slot t % W).
+ *   q      [B, C, H, D] bf16: the chunk's queries
+ *   k_new, v_new [B, C, Hkv, D] bf16: the chunk's keys and values
+ *   k_ring, v_ring [B, W, Hkv, D] bf16: the cache holding positions < pos0;
+ *          updated in place: slot (pos0 + c) % W receives token c (of a
+ *          chunk longer than W only the last W tokens stay)
+ *   pos0   [B] int64, device: position of the chunk's first token (>= 0)
+ *   out    [B, C, H, D] bf16; lse [B, H, C] fp32 (may be NULL)
+ * Token c (position p = pos0 + c) attends positions max(0, p-W+1) .. p,
+ * taking positions >= pos0 from the chunk and the others from the ring as
+ * it was before the call.  W must be a positive multiple of 64; 1 <= C <=
+ * 65535; D in {64, 128}; H % Hkv == 0, H / Hkv <= 8; scale <= 0 means
+ * 1/sqrt(D).  Two launches on `stream` (attention, then the ring update).
+ * Workspace, streams and graphs as for swa_decode.
+ */
+SWA_API int swa_append(const void* q, const void* k_new, const void* v_new, void* k_ring,
+                       void* v_ring, void* out, float* lse, const int64_t* pos0, int B, int C,
+                       int H, int Hkv, int D, int W, float scale, void* stream);
 
 /*
  * swa_device_error -- synchronises `stream`, then reports (and clears) a

@@ -11,14 +11,18 @@ torch CUDA tensors, shapes and sizes are taken from them.
 from .binding import (  # noqa: F401
     SwaError,
     library_path,
+    swa_append,
     swa_decode,
     swa_decode_ex,
     swa_decode_noalloc,
     swa_decode_noalloc_scratch_bytes,
+    swa_decode_paged,
     swa_device_error,
     swa_forward,
     swa_forward_ex,
     swa_forward_f32,
+    swa_forward_layers,
+    swa_paged_window,
     swa_release,
     swa_schedule,
     swa_selftest_timeout,

@@ -30,6 +30,20 @@ _lib.swa_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
 _lib.swa_decode_noalloc.restype = _I
 _lib.swa_decode_noalloc_scratch_bytes.argtypes = []
 _lib.swa_decode_noalloc_scratch_bytes.restype = ctypes.c_size_t
+_lib.swa_decode_paged.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                                  _F, _P]
+_lib.swa_paged_window.argtypes = [ctypes.c_int64, _I, _I, _P, _P]
+_lib.swa_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
+
+
+class SwaLayer(ctypes.Structure):
+    """struct swa_layer of include/swa.h."""
+    _fields_ = [("q", _P), ("k", _P), ("v", _P), ("out", _P), ("lse", _P),
+                ("win_left", _I), ("win_right", _I), ("dilation", _I), ("dilation_block", _I),
+                ("global_idx", _P), ("n_global", _I), ("scale", _F)]
+
+
+_lib.swa_forward_layers.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P]
 _lib.swa_device_error.argtypes = [_P]
 _lib.swa_selftest_timeout.argtypes = [_I, _P]
 _lib.swa_schedule.argtypes = [_I, _I, _I, _I, _I, _P, _I]
@@ -38,6 +52,7 @@ _lib.swa_status_string.argtypes = [_I]
 _lib.swa_status_string.restype = ctypes.c_char_p
 _lib.swa_version.argtypes = []
 for _fn in ("swa_forward", "swa_forward_ex", "swa_forward_f32", "swa_decode", "swa_decode_ex",
+            "swa_decode_paged", "swa_paged_window", "swa_append", "swa_forward_layers",
             "swa_device_error", "swa_selftest_timeout", "swa_schedule", "swa_release",
             "swa_version"):
     getattr(_lib, _fn).restype = _I
@@ -127,6 +142,39 @@ def swa_forward_ex(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dilat
     return out
 
 
+def swa_forward_layers(layers, stream=None):
+    """A per-layer window schedule (C: swa_forward_layers).  `layers` is a list
+    of dicts with q, k, v (bf16 [B, N, H|Hkv, D], the same shapes in every
+    layer), and optionally out, lse, win_left, win_right, dilation,
+    dilation_block, global_idx, scale.  Returns the list of outputs."""
+    if not layers:
+        return []
+    arr = (SwaLayer * len(layers))()
+    outs, keep = [], []
+    shape = None
+    for i, L in enumerate(layers):
+        B, N, H, Hkv, D, out, gi, ng = _fwd_common(L["q"], L["k"], L["v"], L.get("out"),
+                                                    L.get("lse"), L.get("global_idx"),
+                                                    torch.bfloat16)
+        if shape is None:
+            shape = (B, N, H, Hkv, D)
+        elif shape != (B, N, H, Hkv, D):
+            raise ValueError(f"layer {i}: shapes differ from layer 0")
+        outs.append(out)
+        keep.append(gi)
+        arr[i] = SwaLayer(L["q"].data_ptr(), L["k"].data_ptr(), L["v"].data_ptr(), out.data_ptr(),
+                          None if L.get("lse") is None else L["lse"].data_ptr(),
+                          int(L.get("win_left", -1)), int(L.get("win_right", -1)),
+                          int(L.get("dilation", 1)), int(L.get("dilation_block", 0)),
+                          None if gi is None else gi.data_ptr(), ng, float(L.get("scale", 0.0)))
+    B, N, H, Hkv, D = shape
+    bad = ctypes.c_int(-1)
+    st = _lib.swa_forward_layers(ctypes.cast(arr, _P), len(layers), B, H, Hkv, N, D,
+                                 ctypes.byref(bad), _stream(stream))
+    _check(st, f"swa_forward_layers (layer {bad.value})")
+    return outs
+
+
 def swa_forward_f32(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dilation=1,
                     dilation_block=0, global_idx=None, scale=0.0, stream=None):
     """fp32 SWA forward on CUDA cores (C: swa_forward_f32)."""
@@ -188,6 +236,71 @@ def swa_decode_noalloc(q, k_ring, v_ring, pos, out, stream=None):
 def swa_decode_noalloc_scratch_bytes() -> int:
     """Bytes of the fixed device array swa_decode_noalloc uses (per GPU)."""
     return int(_lib.swa_decode_noalloc_scratch_bytes())
+
+
+def swa_decode_paged(q, k_pages, v_pages, block_table, pos, page_size, W, out=None, lse=None,
+                     scale=0.0, stream=None):
+    """Decode over a paged KV cache (C: swa_decode_paged).  q [B, H, D];
+    k_pages/v_pages [num_pages * page_size, Hkv, D]; block_table [B, max_pages]
+    int32; pos [B] int64.  Returns out [B, H, D]."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_pages, "k_pages", torch.bfloat16, 3)
+    _need(v_pages, "v_pages", torch.bfloat16, 3)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(pos, "pos", torch.int64, 1)
+    B, H, D = q.shape
+    rows, Hkv = k_pages.shape[0], k_pages.shape[1]
+    if (k_pages.shape[2] != D or v_pages.shape != k_pages.shape or pos.shape != (B,)
+            or block_table.shape[0] != B or rows % int(page_size) != 0):
+        raise ValueError("k_pages/v_pages [num_pages * page_size, Hkv, D], block_table [B, *], "
+                         "pos [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 3)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 2)
+    _check(_lib.swa_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(out), _ptr(lse),
+                                 _ptr(block_table), _ptr(pos), B, H, Hkv, D, int(page_size),
+                                 rows // int(page_size), block_table.shape[1], int(W),
+                                 float(scale), _stream(stream)), "swa_decode_paged")
+    return out
+
+
+def swa_paged_window(pos: int, W: int, page_size: int):
+    """Host-only: (first_page, last_page) of the logical pages a decode at
+    `pos` reads; pages below first_page can be released (C: swa_paged_window)."""
+    first, last = ctypes.c_int64(), ctypes.c_int64()
+    _check(_lib.swa_paged_window(int(pos), int(W), int(page_size), ctypes.byref(first),
+                                 ctypes.byref(last)), "swa_paged_window")
+    return first.value, last.value
+
+
+def swa_append(q, k_new, v_new, k_ring, v_ring, pos0, out=None, lse=None, scale=0.0,
+               stream=None):
+    """A chunk of C tokens enters the ring cache (C: swa_append).  q [B, C, H, D];
+    k_new/v_new [B, C, Hkv, D]; k_ring/v_ring [B, W, Hkv, D] (updated in place);
+    pos0 [B] int64.  Returns out [B, C, H, D]."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k_new, "k_new", torch.bfloat16, 4)
+    _need(v_new, "v_new", torch.bfloat16, 4)
+    _need(k_ring, "k_ring", torch.bfloat16, 4)
+    _need(v_ring, "v_ring", torch.bfloat16, 4)
+    _need(pos0, "pos0", torch.int64, 1)
+    B, C, H, D = q.shape
+    W, Hkv = k_ring.shape[1], k_ring.shape[2]
+    if (k_new.shape != (B, C, Hkv, D) or v_new.shape != k_new.shape
+            or k_ring.shape != (B, W, Hkv, D) or v_ring.shape != k_ring.shape
+            or pos0.shape != (B,)):
+        raise ValueError("k_new/v_new [B, C, Hkv, D], k_ring/v_ring [B, W, Hkv, D], pos0 [B]")
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", torch.bfloat16, 4)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, 3)
+    _check(_lib.swa_append(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ring), _ptr(v_ring),
+                           _ptr(out), _ptr(lse), _ptr(pos0), B, C, H, Hkv, D, W, float(scale),
+                           _stream(stream)), "swa_append")
+    return out
 
 
 def swa_device_error(stream=None) -> int:

@@ -123,15 +123,26 @@ float resolve_scale(float scale, int D) {
 
 extern "C" {
 
-SWA_API int swa_forward_ex(const void* q, const void* k, const void* v, void* out, float* lse,
-                           int B, int H, int Hkv, int N, int D, int win_left, int win_right,
-                           int dilation, int dilation_block, const int32_t* global_idx,
-                           int n_global, float scale, void* stream) {
+namespace {
+int check_forward_bf16(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                       int H, int Hkv, int N, int D, int dilation, int dilation_block,
+                       const int32_t* global_idx, int n_global) {
   int st = check_forward_args(q, k, v, out, lse, B, H, Hkv, N, D, dilation, dilation_block,
                               global_idx, n_global);
   if (st != SWA_OK) return st;
   if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
   if (dilation_block > 1 && dilation_block != kBlockRows) return SWA_ERR_UNSUPPORTED;
+  return SWA_OK;
+}
+}  // namespace
+
+SWA_API int swa_forward_ex(const void* q, const void* k, const void* v, void* out, float* lse,
+                           int B, int H, int Hkv, int N, int D, int win_left, int win_right,
+                           int dilation, int dilation_block, const int32_t* global_idx,
+                           int n_global, float scale, void* stream) {
+  int st = check_forward_bf16(q, k, v, out, lse, B, H, Hkv, N, D, dilation, dilation_block,
+                              global_idx, n_global);
+  if (st != SWA_OK) return st;
   if (B == 0 || N == 0) return SWA_OK;
   const float sc = resolve_scale(scale, D);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -150,6 +161,32 @@ SWA_API int swa_forward(const void* q, const void* k, const void* v, void* out, 
                         void* stream) {
   return swa_forward_ex(q, k, v, out, lse, B, H, Hkv, N, D, win_left, win_right, dilation, 0,
                         global_idx, n_global, scale, stream);
+}
+
+SWA_API int swa_forward_layers(const swa_layer* layers, int n_layers, int B, int H, int Hkv,
+                               int N, int D, int* bad_layer, void* stream) {
+  if (bad_layer) *bad_layer = -1;
+  if (n_layers < 0 || (n_layers > 0 && !layers)) return SWA_ERR_ARG;
+  for (int i = 0; i < n_layers; ++i) {
+    const swa_layer& L = layers[i];
+    const int st = check_forward_bf16(L.q, L.k, L.v, L.out, L.lse, B, H, Hkv, N, D, L.dilation,
+                                      L.dilation_block, L.global_idx, L.n_global);
+    if (st != SWA_OK) {
+      if (bad_layer) *bad_layer = i;
+      return st;
+    }
+  }
+  for (int i = 0; i < n_layers; ++i) {
+    const swa_layer& L = layers[i];
+    const int st = swa_forward_ex(L.q, L.k, L.v, L.out, L.lse, B, H, Hkv, N, D, L.win_left,
+                                  L.win_right, L.dilation, L.dilation_block, L.global_idx,
+                                  L.n_global, L.scale, stream);
+    if (st != SWA_OK) {
+      if (bad_layer) *bad_layer = i;
+      return st;
+    }
+  }
+  return SWA_OK;
 }
 
 SWA_API int swa_forward_f32(const float* q, const float* k, const float* v, float* out,
@@ -206,6 +243,53 @@ SWA_API int swa_decode_noalloc(const void* q, const void* k_ring, const void* v_
 }
 
 SWA_API size_t swa_decode_noalloc_scratch_bytes(void) { return noalloc_scratch_bytes(); }
+
+SWA_API int swa_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* out,
+                             float* lse, const int32_t* block_table, const int64_t* pos, int B,
+                             int H, int Hkv, int D, int page_size, int num_pages, int max_pages,
+                             int W, float scale, void* stream) {
+  if (B < 0 || H <= 0 || Hkv <= 0 || D <= 0 || W <= 0 || page_size <= 0 || num_pages <= 0 ||
+      max_pages <= 0)
+    return SWA_ERR_ARG;
+  if (H % Hkv != 0) return SWA_ERR_ARG;
+  if (!q || !k_pages || !v_pages || !out || !block_table || !pos) return SWA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(pos) & 7u) || (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return SWA_ERR_ALIGN;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (H / Hkv > 8 || page_size % 64 != 0) return SWA_ERR_UNSUPPORTED;
+  if (B == 0) return SWA_OK;
+  return launch_decode_paged(q, k_pages, v_pages, out, lse, block_table, pos, B, H, Hkv, D,
+                             page_size, num_pages, max_pages, W, resolve_scale(scale, D),
+                             static_cast<cudaStream_t>(stream));
+}
+
+SWA_API int swa_paged_window(int64_t pos, int W, int page_size, int64_t* first_page,
+                             int64_t* last_page) {
+  if (pos < 0 || W < 1 || page_size < 1 || !first_page || !last_page) return SWA_ERR_ARG;
+  const int64_t first = pos - W + 1 < 0 ? 0 : pos - W + 1;
+  *first_page = first / page_size;
+  *last_page = pos / page_size;
+  return SWA_OK;
+}
+
+SWA_API int swa_append(const void* q, const void* k_new, const void* v_new, void* k_ring,
+                       void* v_ring, void* out, float* lse, const int64_t* pos0, int B, int C,
+                       int H, int Hkv, int D, int W, float scale, void* stream) {
+  if (B < 0 || C < 0 || H <= 0 || Hkv <= 0 || D <= 0 || W <= 0) return SWA_ERR_ARG;
+  if (H % Hkv != 0) return SWA_ERR_ARG;
+  if (!q || !k_new || !v_new || !k_ring || !v_ring || !out || !pos0) return SWA_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_ring) ||
+      !aligned16(v_ring) || !aligned16(out) || (reinterpret_cast<uintptr_t>(pos0) & 7u) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return SWA_ERR_ALIGN;
+  if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
+  if (H / Hkv > 8 || W % 64 != 0 || C > 65535) return SWA_ERR_UNSUPPORTED;
+  if (B == 0 || C == 0) return SWA_OK;
+  return launch_append(q, k_new, v_new, k_ring, v_ring, out, lse, pos0, B, C, H, Hkv, D, W,
+                       resolve_scale(scale, D), static_cast<cudaStream_t>(stream));
+}
 
 SWA_API int swa_device_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)

@@ -45,6 +45,13 @@ size_t noalloc_scratch_bytes();
 
 int launch_timeout_selftest(int limit_us, cudaStream_t stream);
 
+int launch_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* out,
+                        float* lse, const int32_t* table, const int64_t* pos, int B, int H,
+                        int Hkv, int D, int page_size, int num_pages, int max_pages, int W,
+                        float scale, cudaStream_t stream);
+int launch_append(const void* q, const void* k_new, const void* v_new, void* k_ring, void* v_ring,
+                  void* out, float* lse, const int64_t* pos0, int B, int C, int H, int Hkv, int D,
+                  int W, float scale, cudaStream_t stream);
 void release_workspaces();
 
 }  // namespace swa

@@ -6,7 +6,13 @@
 //    slot t % W; aiqz.cc page, "推理优化策略": the cache rolls like a
 //    conveyor belt, old entries are overwritten);
 //  * global query rows: a global token attends every key (aiqz.cc page,
-//    "全局注意力token"); causal problems clip it to keys <= its position.
+//    "全局注意力token"); causal problems clip it to keys <= its position;
+//  * paged decode: the cache lives in fixed-size pages found through a block
+//    table, so pages that leave the window can be released ("空洞滑窗机制"
+//    page, §四, KV cache management with PagedAttention);
+//  * chunked append: C new tokens attend the ring history and the chunk
+//    itself, each over its own window (aiqz.cc page, "推理优化策略":
+//    streaming inference).
 //
 // The work is HBM-bound (each key/value byte is used for a handful of
 // flops), so the kernel is built for bandwidth: one CTA streams a chunk of
@@ -36,8 +42,12 @@ constexpr int kComputeWarps = 4;
 constexpr int kThreadsR = (kComputeWarps + 1) * 32;
 
 struct RowParams {
-  CUtensorMap tmK;
+  CUtensorMap tmK;   // decode: ring; global rows: sequence; paged: page pool
   CUtensorMap tmV;
+  CUtensorMap tmKn;  // chunked append: the chunk's new keys / values
+  CUtensorMap tmVn;
+  const int32_t* table;  // paged: block table [B, max_pages]
+  int page_size, max_pages;
   const uint16_t* q;
   uint16_t* out;
   float* lse;
@@ -47,7 +57,7 @@ struct RowParams {
   float* ws_ml;
   int* cnt;
   int* err;
-  int mode;  // 0: decode, 1: global rows
+  int mode;  // 0: decode, 1: global rows, 2: paged decode, 3: chunked append
   int B, H, Hkv, N, W, grp, ng, causal;
   int rows_per_cta, nrowchunks;
   int chunk, nsplit;
@@ -112,7 +122,9 @@ __device__ __forceinline__ float reduce8_transposed(float (&v)[NQ], int t, int* 
   return w[0];
 }
 
-template <int D, int NQ>
+// MODE: 0 ring decode, 1 global rows, 2 paged decode, 3 chunked append
+// (compile-time, so each user's kernel carries only its own addressing).
+template <int D, int NQ, int MODE>
 __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
     swa_rowattn_kernel(const __grid_constant__ RowParams p) {
   using S = RSmem<D, NQ>;
@@ -131,9 +143,13 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
   const int split = blockIdx.x;
   const int gi = blockIdx.y;  // query set
 
-  // ---- the query set: kv head, batch, query vectors and their key limits
+  // ---- the query set: kv head, batch, query vectors and their key sets.
+  // Keys are walked by an index idx in [0, max_limit).  Key positions are
+  // kept relative to tA (32-bit): rel(idx) = idx below seg_n, idx + off_b
+  // from seg_n on (the chunk of an append); slot s sees the keys with
+  // lo_r[s] <= rel <= hi_r[s] (and, below seg_n, rel < a_end_r).
   int b, g, rowchunk = 0;
-  if (p.mode == 0) {
+  if (MODE == 0 || MODE == 2) {
     g = gi % p.Hkv;
     b = gi / p.Hkv;
   } else {
@@ -141,32 +157,68 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
     g = (gi / p.nrowchunks) % p.Hkv;
     b = gi / (p.nrowchunks * p.Hkv);
   }
-  // per slot: query row offset and key limit (keys [0, limit))
+  long long tA = 0;
+  int seg_n = 0x7fffffff, off_b = 0, a_end_r = 0x7fffffff;
   long qoff[NQ];
-  int limit[NQ];
+  int lo_r[NQ], hi_r[NQ];
   int max_limit = 0;
+  if (MODE == 2) {
+    const long long ps = p.pos[b];
+    const long long start = ps - p.W + 1 < 0 ? 0 : ps - p.W + 1;
+    tA = start & ~(long long)(kRows - 1);
+    const long long lim = ps + 1 - tA;
+    max_limit = lim < 0 ? 0 : (int)lim;
+  } else if (MODE == 3) {
+    const long long pos0 = p.pos[b];
+    const long long r0 = (long long)rowchunk * p.rows_per_cta;
+    const long long start = pos0 + r0 - p.W + 1 < 0 ? 0 : pos0 + r0 - p.W + 1;
+    tA = start & ~(long long)(kRows - 1);
+    const long long na = pos0 > tA ? ((pos0 - tA + kRows - 1) / kRows) * kRows : 0;
+    seg_n = (int)na;
+    a_end_r = (int)(pos0 - tA);
+    off_b = (int)(pos0 - na - tA);
+    const long long last = r0 + p.rows_per_cta < p.N ? r0 + p.rows_per_cta : p.N;
+    max_limit = (int)(na + last);
+  }
 #pragma unroll
   for (int s = 0; s < NQ; ++s) {
     const int hsub = s % p.grp, rsub = s / p.grp;
     const int h = g * p.grp + hsub;
     qoff[s] = -1;
-    limit[s] = 0;
+    lo_r[s] = 0;
+    hi_r[s] = -1;
     if (rsub < p.rows_per_cta) {
-      if (p.mode == 0) {
+      if (MODE == 0) {
         long long ps = p.pos[b];
-        limit[s] = ps + 1 < (long long)p.W ? (int)(ps + 1) : p.W;
+        const int limit = ps + 1 < (long long)p.W ? (int)(ps + 1) : p.W;
+        hi_r[s] = limit - 1;
         qoff[s] = ((long)b * p.H + h) * D;
+        max_limit = limit > max_limit ? limit : max_limit;
+      } else if (MODE == 2) {
+        const long long ps = p.pos[b];
+        lo_r[s] = (int)((ps - p.W + 1 < 0 ? 0 : ps - p.W + 1) - tA);
+        hi_r[s] = (int)(ps - tA);
+        qoff[s] = ((long)b * p.H + h) * D;
+      } else if (MODE == 3) {
+        const int c = rowchunk * p.rows_per_cta + rsub;
+        if (c < p.N) {
+          const long long pc = p.pos[b] + c;
+          lo_r[s] = (int)((pc - p.W + 1 < 0 ? 0 : pc - p.W + 1) - tA);
+          hi_r[s] = (int)(pc - tA);
+          qoff[s] = (((long)b * p.N + c) * p.H + h) * D;
+        }
       } else {
         const int j = rowchunk * p.rows_per_cta + rsub;
         if (j < p.ng) {
           int i = p.G[j];
           i = i < 0 ? 0 : (i >= p.N ? p.N - 1 : i);
-          limit[s] = p.causal ? i + 1 : p.N;
+          const int limit = p.causal ? i + 1 : p.N;
+          hi_r[s] = limit - 1;
           qoff[s] = (((long)b * p.N + i) * p.H + h) * D;
+          max_limit = limit > max_limit ? limit : max_limit;
         }
       }
     }
-    max_limit = limit[s] > max_limit ? limit[s] : max_limit;
   }
   const int key0 = split * p.chunk;
   int nk = max_limit - key0;
@@ -198,6 +250,10 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
     if (lane == 0) {
       prefetch_tensormap(&p.tmK);
       prefetch_tensormap(&p.tmV);
+      if (MODE == 3) {
+        prefetch_tensormap(&p.tmKn);
+        prefetch_tensormap(&p.tmVn);
+      }
       for (int k = 0; k < n_stages; ++k) {
         const int st = k % kStagesR;
         if (k >= kStagesR &&
@@ -205,10 +261,33 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
           break;
         uint8_t* kb = smem + st * S::kStage;
         uint8_t* vb = kb + S::kTile;
+        // source of the 64 key rows [idx0, idx0 + 64): a row of the ring /
+        // sequence, a page of the pool, or rows of the chunk.  Rows past a
+        // tensor's end (or a page id past the pool) read as zeros and are
+        // masked below.
+        const int idx0 = key0 + k * kRows;
+        const CUtensorMap* mk = &p.tmK;
+        const CUtensorMap* mv = &p.tmV;
+        int row = idx0, bc = b;
+        if (MODE == 2) {
+          const long long t0 = tA + idx0;
+          const long long lp = t0 / p.page_size;
+          const long long page = lp < p.max_pages ? p.table[(long)b * p.max_pages + lp] : -1;
+          row = page < 0 ? -kRows : (int)(page * p.page_size + t0 % p.page_size);
+          bc = 0;
+        } else if (MODE == 3) {
+          if (idx0 < seg_n) {
+            row = (int)((tA + idx0) % p.W);
+          } else {
+            row = idx0 - seg_n;
+            mk = &p.tmKn;
+            mv = &p.tmVn;
+          }
+        }
         mbar_arrive_expect_tx(&full[st], S::kStage);
         for (int cc = 0; cc < D / 64; ++cc) {
-          tma_load_4d(kb + cc * (kRows * 128), &p.tmK, &full[st], cc * 64, g, key0 + k * kRows, b);
-          tma_load_4d(vb + cc * (kRows * 128), &p.tmV, &full[st], cc * 64, g, key0 + k * kRows, b);
+          tma_load_4d(kb + cc * (kRows * 128), mk, &full[st], cc * 64, g, row, bc);
+          tma_load_4d(vb + cc * (kRows * 128), mv, &full[st], cc * 64, g, row, bc);
         }
       }
     }
@@ -271,12 +350,21 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
         // after the reduction lanes t with t % (8 / NQ) == 0 hold distinct
         // slots; each writes its (row, slot) score
         if ((t8 & (8 / NQ - 1)) == 0) {
-          const int key = key0 + k * kRows + r;
-          int lim = 0;
+          const int idx = key0 + k * kRows + r;
+          const int rel = idx < seg_n ? idx : idx + off_b;
+          int lo = lo_r[0], hi = hi_r[0];  // decode, paged: one sequence per set
+          if (MODE == 1 || MODE == 3) {
 #pragma unroll
-          for (int s = 0; s < NQ; ++s)
-            if (s == myslot) lim = limit[s];
-          sc[r * NQ + myslot] = key < lim ? tot : -INFINITY;
+            for (int s = 1; s < NQ; ++s)
+              if (s == myslot) {
+                lo = lo_r[s];
+                hi = hi_r[s];
+              }
+          }
+          const bool ok = (MODE == 0 || MODE == 1)
+                              ? idx <= hi
+                              : (rel >= lo && rel <= hi && (idx >= seg_n || rel < a_end_r));
+          sc[r * NQ + myslot] = ok ? tot : -INFINITY;
         }
       }
       named_sync(1, kComputeWarps * 32);
@@ -387,7 +475,7 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
       const float lv = (sc[s] + __log2f(sc[NQ + s])) * 0.69314718055994531f;
       const long row = qoff[s] / D;  // decode: b*H + h; global: (b*N + i)*H + h
       long li;
-      if (p.mode == 0) li = row;
+      if (MODE == 0 || MODE == 2) li = row;
       else {
         const int h = (int)(row % p.H);
         const long bi = row / p.H;
@@ -449,7 +537,7 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
     const float lv = (Ms[s] + __log2f(Ls[s])) * 0.69314718055994531f;
     const long row = qoff[s] / D;
     long li;
-    if (p.mode == 0) li = row;
+    if (MODE == 0 || MODE == 2) li = row;
     else {
       const int h = (int)(row % p.H);
       const long bi = row / p.H;
@@ -461,7 +549,8 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
 }
 
 // ------------------------------------------------------------ workspaces
-// Per device and per user (0: decode, 1: global rows): split counters and
+// Per device and per user (0: decode, 1: global rows, 2: paged decode,
+// 3: chunked append): split counters and
 // split partials in separate buffers.  Every merge resets its counter to
 // zero, so between complete calls all counters are zero; the counter buffer
 // is zeroed whenever it is (re)allocated and is never overlapped by the
@@ -473,7 +562,7 @@ struct Workspace {
   size_t part_bytes = 0;
 };
 constexpr int kMaxDev = 64;
-Workspace g_ws[kMaxDev][2];
+Workspace g_ws[kMaxDev][4];  // users: decode, global rows, paged, append
 std::mutex g_ws_mu;
 
 bool get_workspace(int which, size_t cnt_bytes, size_t part_bytes, cudaStream_t stream,
@@ -515,28 +604,41 @@ bool get_workspace(int which, size_t cnt_bytes, size_t part_bytes, cudaStream_t 
   return true;
 }
 
-template <int D, int NQ>
+template <int D, int NQ, int MODE>
 int launch_rows(RowParams& p, int nsets, cudaStream_t stream) {
   using S = RSmem<D, NQ>;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(swa_rowattn_kernel<D, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             S::kAlloc) != cudaSuccess)
+    if (cudaFuncSetAttribute(swa_rowattn_kernel<D, NQ, MODE>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) != cudaSuccess)
       return SWA_ERR_CUDA;
     attr = true;
   }
   dim3 grid(p.nsplit, nsets);
-  swa_rowattn_kernel<D, NQ><<<grid, kThreadsR, S::kAlloc, stream>>>(p);
+  swa_rowattn_kernel<D, NQ, MODE><<<grid, kThreadsR, S::kAlloc, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
+// decode and paged decode serve a GQA group (1, 2, 4 or 8 query vectors);
+// global rows and chunked append always fill 8 slots
 template <int D>
 int dispatch_nq(RowParams& p, int nq, int nsets, cudaStream_t stream) {
+  if (p.mode == 1) return nq == 8 ? launch_rows<D, 8, 1>(p, nsets, stream) : SWA_ERR_UNSUPPORTED;
+  if (p.mode == 3) return nq == 8 ? launch_rows<D, 8, 3>(p, nsets, stream) : SWA_ERR_UNSUPPORTED;
+  if (p.mode == 0) {
+    switch (nq) {
+      case 1: return launch_rows<D, 1, 0>(p, nsets, stream);
+      case 2: return launch_rows<D, 2, 0>(p, nsets, stream);
+      case 4: return launch_rows<D, 4, 0>(p, nsets, stream);
+      case 8: return launch_rows<D, 8, 0>(p, nsets, stream);
+      default: return SWA_ERR_UNSUPPORTED;
+    }
+  }
   switch (nq) {
-    case 1: return launch_rows<D, 1>(p, nsets, stream);
-    case 2: return launch_rows<D, 2>(p, nsets, stream);
-    case 4: return launch_rows<D, 4>(p, nsets, stream);
-    case 8: return launch_rows<D, 8>(p, nsets, stream);
+    case 1: return launch_rows<D, 1, 2>(p, nsets, stream);
+    case 2: return launch_rows<D, 2, 2>(p, nsets, stream);
+    case 4: return launch_rows<D, 4, 2>(p, nsets, stream);
+    case 8: return launch_rows<D, 8, 2>(p, nsets, stream);
     default: return SWA_ERR_UNSUPPORTED;
   }
 }
@@ -573,6 +675,23 @@ int run(RowParams& p, int D, int nq, int nsets, int which, cudaStream_t stream) 
   if (D == 128) return dispatch_nq<128>(p, nq, nsets, stream);
   if (D == 64) return dispatch_nq<64>(p, nq, nsets, stream);
   return SWA_ERR_UNSUPPORTED;
+}
+
+// Writes the chunk's keys and values into their ring slots (pos0 + c) % W,
+// 16 bytes per thread.  grid (ceil(row_vecs / 256), C - c_first, B).
+__global__ void ring_store_kernel(const uint4* __restrict__ k_new, const uint4* __restrict__ v_new,
+                                  uint4* __restrict__ k_ring, uint4* __restrict__ v_ring,
+                                  const int64_t* __restrict__ pos0, int C, int W, int row_vecs,
+                                  int c_first) {
+  const int b = blockIdx.z, c = c_first + (int)blockIdx.y;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  const long long p0 = pos0[b];
+  if (i >= row_vecs || p0 < 0) return;
+  const long long slot = (p0 + c) % W;
+  const long src = ((long)b * C + c) * row_vecs + i;
+  const long dst = ((long)b * W + slot) * row_vecs + i;
+  k_ring[dst] = k_new[src];
+  v_ring[dst] = v_new[src];
 }
 
 }  // namespace
@@ -636,10 +755,92 @@ int launch_global_rows(const void* q, const void* k, const void* v, void* out, f
   return run(p, D, nq, B * Hkv * p.nrowchunks, 1, stream);
 }
 
+int launch_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* out,
+                        float* lse, const int32_t* table, const int64_t* pos, int B, int H,
+                        int Hkv, int D, int page_size, int num_pages, int max_pages, int W,
+                        float scale, cudaStream_t stream) {
+  RowParams p;
+  std::memset(&p, 0, sizeof(p));
+  const long long rows = (long long)num_pages * page_size;
+  if (rows > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  if (encode_kv(&p.tmK, k_pages, D, Hkv, (int)rows, 1) != SWA_OK ||
+      encode_kv(&p.tmV, v_pages, D, Hkv, (int)rows, 1) != SWA_OK)
+    return SWA_ERR_CUDA;
+  p.q = static_cast<const uint16_t*>(q);
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.pos = pos;
+  p.table = table;
+  p.page_size = page_size;
+  p.max_pages = max_pages;
+  p.err = device_error_word();
+  if (!p.err) return SWA_ERR_CUDA;
+  p.mode = 2;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.W = W;
+  p.grp = H / Hkv;
+  p.rows_per_cta = 1;
+  p.nrowchunks = 1;
+  // the window's keys, from a 64-aligned start: at most W + 63 indices,
+  // split into near-equal multiples of 64 of about 1024 keys
+  const int span = W + kRows;
+  p.nsplit = (span + 1023) / 1024;
+  p.chunk = (((span + p.nsplit - 1) / p.nsplit) + kRows - 1) / kRows * kRows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int nq = pow2_at_least(p.grp);
+  return run(p, D, nq, B * Hkv, 2, stream);
+}
+
+int launch_append(const void* q, const void* k_new, const void* v_new, void* k_ring, void* v_ring,
+                  void* out, float* lse, const int64_t* pos0, int B, int C, int H, int Hkv, int D,
+                  int W, float scale, cudaStream_t stream) {
+  RowParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (encode_kv(&p.tmK, k_ring, D, Hkv, W, B) != SWA_OK ||
+      encode_kv(&p.tmV, v_ring, D, Hkv, W, B) != SWA_OK ||
+      encode_kv(&p.tmKn, k_new, D, Hkv, C, B) != SWA_OK ||
+      encode_kv(&p.tmVn, v_new, D, Hkv, C, B) != SWA_OK)
+    return SWA_ERR_CUDA;
+  p.q = static_cast<const uint16_t*>(q);
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.pos = pos0;
+  p.err = device_error_word();
+  if (!p.err) return SWA_ERR_CUDA;
+  p.mode = 3;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.N = C;
+  p.W = W;
+  p.grp = H / Hkv;
+  const int nq = 8;
+  p.rows_per_cta = nq / p.grp;  // query tokens per CTA (8 query vectors)
+  p.nrowchunks = (C + p.rows_per_cta - 1) / p.rows_per_cta;
+  // history (at most W + 64 indices from a 64-aligned start) then the chunk
+  const int span = W + kRows + C;
+  p.nsplit = (span + 1023) / 1024;
+  p.chunk = (((span + p.nsplit - 1) / p.nsplit) + kRows - 1) / kRows * kRows;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int st = run(p, D, nq, B * Hkv * p.nrowchunks, 3, stream);
+  if (st != SWA_OK) return st;
+  // then the new tokens enter the ring (after every query has read the
+  // slots they overwrite); of a chunk longer than W only the last W stay
+  const int c_first = C > W ? C - W : 0;
+  const int row_vecs = Hkv * D / 8;
+  dim3 grid((row_vecs + 255) / 256, C - c_first, B);
+  ring_store_kernel<<<grid, 256, 0, stream>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+      static_cast<uint4*>(k_ring), static_cast<uint4*>(v_ring), pos0, C, W, row_vecs, c_first);
+  return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
 void release_workspaces() {
   std::lock_guard<std::mutex> lk(g_ws_mu);
   for (int d = 0; d < kMaxDev; ++d)
-    for (int w = 0; w < 2; ++w) {
+    for (int w = 0; w < 4; ++w) {
       Workspace& ws = g_ws[d][w];
       if (!ws.cnt && !ws.part) continue;
       int cur = 0;

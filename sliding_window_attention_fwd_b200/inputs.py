@@ -130,3 +130,87 @@ def decode_inputs(cfg: DecodeConfig, device="cpu"):
     vr = normal((cfg.B, cfg.W, cfg.Hkv, cfg.D), cfg.seed, 2, torch.bfloat16, device)
     pos = uniform_int(cfg.B, cfg.pos_lo, cfg.pos_hi, cfg.seed, 3)
     return q, kr, vr, pos
+
+
+@dataclass
+class PagedConfig:
+    """Decode over a paged cache: page_size-row pages of a shared pool, each
+    sequence's live window scattered over randomly chosen physical pages;
+    logical pages that left the window are marked -1 (evicted)."""
+    name: str
+    B: int
+    H: int
+    Hkv: int
+    D: int
+    W: int
+    page_size: int
+    pos_lo: int
+    pos_hi: int
+    seed: int = 7
+
+
+@dataclass
+class AppendConfig:
+    """A chunk of C new tokens per sequence entering a W-slot ring cache."""
+    name: str
+    B: int
+    C: int
+    H: int
+    Hkv: int
+    D: int
+    W: int
+    pos_lo: int
+    pos_hi: int
+    seed: int = 8
+
+
+PAGED_CONFIGS = {
+    # the ring_decode workload's shapes with the cache in 256-row pages
+    "paged_decode": PagedConfig("paged_decode", B=64, H=32, Hkv=8, D=128, W=4096, page_size=256,
+                                pos_lo=4096, pos_hi=131072, seed=1007),
+    "small_paged": PagedConfig("small_paged", B=5, H=8, Hkv=2, D=128, W=300, page_size=64,
+                               pos_lo=0, pos_hi=1000, seed=2008),
+}
+
+APPEND_CONFIGS = {
+    # chunked prefill / streaming: 64-token chunks into a Mistral-sized ring
+    "ring_append": AppendConfig("ring_append", B=8, C=64, H=32, Hkv=8, D=128, W=4096,
+                                pos_lo=4096, pos_hi=131072, seed=1009),
+    "small_append": AppendConfig("small_append", B=4, C=37, H=8, Hkv=2, D=128, W=256,
+                                 pos_lo=0, pos_hi=600, seed=2010),
+}
+
+
+def paged_inputs(cfg: PagedConfig, device="cpu"):
+    """(q [B,H,D], k_pages, v_pages [P*page_size,Hkv,D], block_table [B,max_pages]
+    int32, pos [B] int64).  The pool holds exactly the pages of the live
+    windows, assigned to sequences in a seeded random order."""
+    pos = uniform_int(cfg.B, cfg.pos_lo, cfg.pos_hi, cfg.seed, 3)
+    ps = cfg.page_size
+    first = [max(0, int(p) - cfg.W + 1) // ps for p in pos]
+    last = [int(p) // ps for p in pos]
+    n_live = [l - f + 1 for f, l in zip(first, last)]
+    P = sum(n_live)
+    perm = torch.randperm(P, generator=_gen(cfg.seed, 4, "cpu"))
+    max_pages = max(last) + 1
+    table = torch.full((cfg.B, max_pages), -1, dtype=torch.int32)
+    k = 0
+    for b in range(cfg.B):
+        for lp in range(first[b], last[b] + 1):
+            table[b, lp] = int(perm[k])
+            k += 1
+    q = normal((cfg.B, cfg.H, cfg.D), cfg.seed, 0, torch.bfloat16, device)
+    kp = normal((P * ps, cfg.Hkv, cfg.D), cfg.seed, 1, torch.bfloat16, device)
+    vp = normal((P * ps, cfg.Hkv, cfg.D), cfg.seed, 2, torch.bfloat16, device)
+    return q, kp, vp, table, pos
+
+
+def append_inputs(cfg: AppendConfig, device="cpu"):
+    """(q [B,C,H,D], k_new, v_new [B,C,Hkv,D], k_ring, v_ring [B,W,Hkv,D], pos0 [B])."""
+    q = normal((cfg.B, cfg.C, cfg.H, cfg.D), cfg.seed, 0, torch.bfloat16, device)
+    kn = normal((cfg.B, cfg.C, cfg.Hkv, cfg.D), cfg.seed, 1, torch.bfloat16, device)
+    vn = normal((cfg.B, cfg.C, cfg.Hkv, cfg.D), cfg.seed, 2, torch.bfloat16, device)
+    kr = normal((cfg.B, cfg.W, cfg.Hkv, cfg.D), cfg.seed, 3, torch.bfloat16, device)
+    vr = normal((cfg.B, cfg.W, cfg.Hkv, cfg.D), cfg.seed, 4, torch.bfloat16, device)
+    pos0 = uniform_int(cfg.B, cfg.pos_lo, cfg.pos_hi, cfg.seed, 5)
+    return q, kn, vn, kr, vr, pos0

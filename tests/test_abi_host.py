@@ -86,3 +86,77 @@ def test_decode_validation():
 
 def test_selftest_rejects_bad_limit():
     assert L.swa_selftest_timeout(0, None) == ARG
+
+
+def test_paged_validation():
+    def pg(**kw):
+        return L.swa_decode_paged(kw.get("q", A), A, A, A, kw.get("lse", None), kw.get("tab", A),
+                                  kw.get("pos", A), kw.get("B", 2), kw.get("H", 32),
+                                  kw.get("Hkv", 8), kw.get("D", 128), kw.get("ps", 256),
+                                  kw.get("npages", 16), kw.get("maxp", 8), kw.get("W", 4096),
+                                  0.0, None)
+    assert pg(H=32, Hkv=3) == ARG
+    assert pg(ps=0) == ARG
+    assert pg(npages=0) == ARG
+    assert pg(tab=None) == ARG
+    assert pg(tab=A + 2) == ALIGN
+    assert pg(pos=A + 4) == ALIGN
+    assert pg(ps=96) == UNSUP       # pages must hold whole 64-row boxes
+    assert pg(H=32, Hkv=2) == UNSUP  # GQA group of 16
+    assert pg(D=96) == UNSUP
+    assert pg(B=0) == OK
+
+
+def test_append_validation():
+    def ap(**kw):
+        return L.swa_append(kw.get("q", A), A, A, A, A, A, None, kw.get("pos", A), kw.get("B", 2),
+                            kw.get("C", 16), kw.get("H", 32), kw.get("Hkv", 8), kw.get("D", 128),
+                            kw.get("W", 4096), 0.0, None)
+    assert ap(C=-1) == ARG
+    assert ap(W=0) == ARG
+    assert ap(pos=None) == ARG
+    assert ap(q=A + 8) == ALIGN
+    assert ap(W=100) == UNSUP       # ring slots of a 64-row box must not wrap
+    assert ap(C=70000) == UNSUP
+    assert ap(C=0) == OK
+    assert ap(B=0) == OK
+
+
+@pytest.mark.parametrize("pos,W,ps", [(0, 1, 64), (5000, 4096, 256), (4095, 4096, 256),
+                                      (131071, 4096, 64), (10, 4096, 128), (256, 1, 256)])
+def test_paged_window_is_exactly_the_pages_of_the_key_set(pos, W, ps):
+    """Pages below first hold no position of the decode's key set (the oracle's
+    key list for the causal window), page first and last hold its ends."""
+    import oracle
+    first, last = swa.swa_paged_window(pos, W, ps)
+    lo = max(0, pos - W + 1)
+    if pos < 20000:
+        keys = oracle.key_set(pos, pos + 1, W - 1, 0)
+        assert min(keys) == lo and max(keys) == pos
+    assert first == lo // ps and last == pos // ps
+    assert first * ps <= lo < (first + 1) * ps
+
+
+def test_paged_window_rejects_bad_arguments():
+    with pytest.raises(swa.SwaError):
+        swa.swa_paged_window(-1, 10, 64)
+    with pytest.raises(swa.SwaError):
+        swa.swa_paged_window(5, 0, 64)
+
+
+def test_layers_validation_names_the_bad_layer():
+    """An invalid layer anywhere in the schedule stops it before any launch."""
+    from sliding_window_attention_fwd_b200.binding import SwaLayer
+    good = SwaLayer(A, A, A, A, None, 8, 8, 1, 0, None, 0, 0.0)
+    bad_d = SwaLayer(A, A, A, A, None, 8, 8, 0, 0, None, 0, 0.0)      # dilation 0
+    bad_al = SwaLayer(A, A, A + 8, A, None, 8, 8, 1, 0, None, 0, 0.0)  # misaligned v
+    for layers, code, idx in [([good, good, bad_d], ARG, 2), ([good, bad_al, good], ALIGN, 1),
+                              ([bad_d], ARG, 0)]:
+        arr = (SwaLayer * len(layers))(*layers)
+        bad = ctypes.c_int(-7)
+        st = L.swa_forward_layers(ctypes.cast(arr, ctypes.c_void_p), len(layers), 1, 4, 2, 64, 128,
+                                  ctypes.byref(bad), None)
+        assert st == code and bad.value == idx
+    bad = ctypes.c_int(-7)
+    assert L.swa_forward_layers(None, 0, 1, 4, 2, 64, 128, ctypes.byref(bad), None) == OK
+    assert L.swa_forward_layers(None, 2, 1, 4, 2, 64, 128, ctypes.byref(bad), None) == ARG
