@@ -55,6 +55,9 @@ def _load():
         lib.oracle_append.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I,
                                       ctypes.c_double, I]
         lib.oracle_append.restype = None
+        lib.oracle_backward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, I, P, I,
+                                        ctypes.c_double, I]
+        lib.oracle_backward.restype = None
         _lib = lib
     return _lib
 
@@ -181,3 +184,24 @@ def append(q, k_ring, v_ring, k_new, v_new, pos0, scale=None, threads=None):
                       _ptr(lse), B, C, H, Hkv, D, W, float(scale),
                       int(threads or default_threads()))
     return out, lse
+
+
+def backward(q, k, v, dout, win_left, win_right, dilation=1, dilation_block=0, global_idx=(),
+             scale=None, threads=None):
+    """fp64 gradients (dq [B,N,H,D], dk, dv [B,N,Hkv,D]) of the forward for an
+    upstream gradient dout [B,N,H,D]."""
+    lib = _load()
+    q, k, v, do = _f32(q), _f32(k), _f32(v), _f32(dout)
+    B, N, H, D = q.shape
+    Hkv = k.shape[2]
+    G = np.ascontiguousarray(np.asarray(global_idx, dtype=np.int32))
+    if scale is None or scale <= 0:
+        scale = 1.0 / np.sqrt(D)
+    dq = np.zeros((B, N, H, D), dtype=np.float64)
+    dk = np.zeros((B, N, Hkv, D), dtype=np.float64)
+    dv = np.zeros((B, N, Hkv, D), dtype=np.float64)
+    lib.oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv), B, H,
+                        Hkv, N, D, int(win_left), int(win_right), int(dilation),
+                        int(dilation_block), _ptr(G), len(G), float(scale),
+                        int(threads or default_threads()))
+    return dq, dk, dv

@@ -403,6 +403,118 @@ void oracle_append(const float* q, const float* k_ring, const float* v_ring,
   free(jobs);
 }
 
+/*
+ * Backward oracle: gradients of the forward definition above with respect to
+ * q, k and v, for an upstream gradient dout = dL/dout.  The pages use the
+ * method in training but print no backward pass, so this is the derivative
+ * of the definition written out (plain calculus, fp64), row by row over the
+ * same key sets:
+ *   P_ij  = exp(s_ij - lse_i),       s_ij = scale * q_i . k_j,  j in K(i)
+ *   dV_j += P_ij dO_i
+ *   dP_ij = dO_i . v_j,              D_i = sum_j P_ij dP_ij  (= dO_i . out_i)
+ *   dS_ij = P_ij (dP_ij - D_i)
+ *   dQ_i  = scale * sum_j dS_ij k_j, dK_j += scale * dS_ij q_i
+ * q, dout [B,N,H,D]; k, v [B,N,Hkv,D] (fp32); dq [B,N,H,D], dk, dv
+ * [B,N,Hkv,D] (fp64).  Work is split by (b, kv head) so the dk / dv sums of
+ * a GQA group stay in one thread.
+ */
+typedef struct {
+  const float *q, *k, *v, *dout;
+  double *dq, *dk, *dv;
+  int B, H, Hkv, N, D, L, R, d, bs, ng;
+  const int* G;
+  double scale;
+  int tid, nthreads;
+} bwd_job;
+
+static void* bwd_worker(void* arg) {
+  bwd_job* J = (bwd_job*)arg;
+  const int D = J->D;
+  int* keys = (int*)malloc(sizeof(int) * (size_t)(J->N + J->ng + 1));
+  double* s = (double*)malloc(sizeof(double) * (size_t)(J->N + J->ng + 1));
+  double* dp = (double*)malloc(sizeof(double) * (size_t)(J->N + J->ng + 1));
+  double* o = (double*)malloc(sizeof(double) * (size_t)D);
+  int grp = J->H / J->Hkv;
+  long kvs = (long)J->Hkv * D;
+  for (int64_t u = J->tid; u < (int64_t)J->B * J->Hkv; u += J->nthreads) {
+    int b = (int)(u / J->Hkv), g = (int)(u % J->Hkv);
+    const float* kb = J->k + ((long)b * J->N * J->Hkv + g) * D;
+    const float* vb = J->v + ((long)b * J->N * J->Hkv + g) * D;
+    double* dkb = J->dk + ((long)b * J->N * J->Hkv + g) * D;
+    double* dvb = J->dv + ((long)b * J->N * J->Hkv + g) * D;
+    for (int h = g * grp; h < (g + 1) * grp; ++h) {
+      for (int i = 0; i < J->N; ++i) {
+        int nk = oracle_key_set(i, J->N, J->L, J->R, J->d, J->bs, J->G, J->ng, keys);
+        long row = ((long)b * J->N + i) * J->H + h;
+        const float* qi = J->q + row * D;
+        const float* doi = J->dout + row * D;
+        double m = -INFINITY;
+        for (int t = 0; t < nk; ++t) {
+          const float* kr = kb + (long)keys[t] * kvs;
+          double acc = 0.0;
+          for (int c = 0; c < D; ++c) acc += (double)qi[c] * (double)kr[c];
+          s[t] = J->scale * acc;
+          if (s[t] > m) m = s[t];
+        }
+        double l = 0.0;
+        for (int t = 0; t < nk; ++t) l += exp(s[t] - m);
+        double lse = m + log(l);
+        /* P (in s), out_i, D_i */
+        for (int c = 0; c < D; ++c) o[c] = 0.0;
+        for (int t = 0; t < nk; ++t) {
+          s[t] = exp(s[t] - lse);
+          const float* vr = vb + (long)keys[t] * kvs;
+          for (int c = 0; c < D; ++c) o[c] += s[t] * (double)vr[c];
+        }
+        double Di = 0.0;
+        for (int c = 0; c < D; ++c) Di += (double)doi[c] * o[c];
+        double* dqi = J->dq + row * D;
+        for (int t = 0; t < nk; ++t) {
+          const float* kr = kb + (long)keys[t] * kvs;
+          const float* vr = vb + (long)keys[t] * kvs;
+          double a = 0.0;
+          for (int c = 0; c < D; ++c) a += (double)doi[c] * (double)vr[c];
+          dp[t] = a;
+          double ds = s[t] * (dp[t] - Di);
+          double* dkr = dkb + (long)keys[t] * kvs;
+          double* dvr = dvb + (long)keys[t] * kvs;
+          for (int c = 0; c < D; ++c) {
+            dqi[c] += J->scale * ds * (double)kr[c];
+            dkr[c] += J->scale * ds * (double)qi[c];
+            dvr[c] += s[t] * (double)doi[c];
+          }
+        }
+      }
+    }
+  }
+  free(keys);
+  free(s);
+  free(dp);
+  free(o);
+  return NULL;
+}
+
+void oracle_backward(const float* q, const float* k, const float* v, const float* dout,
+                     double* dq, double* dk, double* dv, int B, int H, int Hkv, int N, int D,
+                     int win_left, int win_right, int dilation, int dilation_block,
+                     const int* G, int n_global, double scale, int nthreads) {
+  if (nthreads < 1) nthreads = 1;
+  memset(dq, 0, sizeof(double) * (size_t)B * N * H * D);
+  memset(dk, 0, sizeof(double) * (size_t)B * N * Hkv * D);
+  memset(dv, 0, sizeof(double) * (size_t)B * N * Hkv * D);
+  pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)nthreads);
+  bwd_job* jobs = (bwd_job*)malloc(sizeof(bwd_job) * (size_t)nthreads);
+  for (int t = 0; t < nthreads; ++t) {
+    bwd_job J = {q, k, v, dout, dq, dk, dv, B, H, Hkv, N, D, win_left, win_right, dilation,
+                 dilation_block, n_global, G, scale, t, nthreads};
+    jobs[t] = J;
+    pthread_create(&th[t], NULL, bwd_worker, &jobs[t]);
+  }
+  for (int t = 0; t < nthreads; ++t) pthread_join(th[t], NULL);
+  free(th);
+  free(jobs);
+}
+
 #ifdef __cplusplus
 }
 #endif
