@@ -419,6 +419,23 @@ def run_ours(args, rank, world, local_rank):
               "frac_tensor": l_flops / l_ms / 1e9 / peaks["bf16_tflops"]}
     del lay
 
+    # ---- backward (dq, dk, dv) of the prefill workload, on CUDA cores
+    bdo = inputs.normal((cfg.B, cfg.N, cfg.H, cfg.D), cfg.seed, 9, torch.bfloat16, dev)
+    step()  # out and lse of the forward for these inputs
+    torch.cuda.synchronize()
+    bgrads = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+    bstep = lambda: swa.swa_backward(q, k, v, out, bdo, lse, cfg.win_left, cfg.win_right,
+                                     dq=bgrads[0], dk=bgrads[1], dv=bgrads[2], stream=stream)
+    bms = time_device(bstep, max(2, args.steps // 40), 1, flush, stream)
+    b_ms = sum(bms) / len(bms)
+    b_flops = 10.0 * cfg.D * pairs  # QK^T recompute, dP, dV, dQ, dK: 5 products of 2*D
+    backward = {"workload": cfg.name, "ms": b_ms, "tflops": b_flops / b_ms / 1e9,
+                "roofline": {"bound": "alu", "achieved": b_flops / b_ms / 1e9,
+                             "peak": alu_peak, "unit": "TFLOP/s",
+                             "frac": b_flops / b_ms / 1e9 / alu_peak, "traffic": None,
+                             "peak_source": "derived (fp32 FMA rate)"}}
+    del bdo, bgrads
+
     # ---- the other forward workloads (parity cases; reported for context)
     others = {}
     for name in ("longformer_global", "dilated_token", "dilated_block"):
@@ -474,6 +491,7 @@ def run_ours(args, rank, world, local_rank):
             "paged_decode": paged,
             "append": append,
             "layers": layers,
+            "backward": backward,
             "others": others,
         }
         if not args.no_cpu_baseline:

@@ -142,6 +142,27 @@ SWA_API int swa_forward_layers(const swa_layer* layers, int n_layers, int B, int
                                int N, int D, int* bad_layer, void* stream);
 
 /*
+ * swa_backward -- gradients of swa_forward_ex with respect to q, k and v.
+ * The pages train with the method but print no backward pass; this is the
+ * derivative of the forward definition over the same key sets, with
+ * P = exp(s - lse) recomputed from the forward's lse:
+ *   dV_j = sum_i P_ij dO_i,  dS_ij = P_ij (dO_i . v_j - dO_i . out_i),
+ *   dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i.
+ *   q, dout, out, dq [B, N, H, D] bf16; k, v, dk, dv [B, N, Hkv, D] bf16;
+ *   lse [B, H, N] fp32 (natural log) and out as written by swa_forward_ex
+ *   for the same arguments; all device memory, 16-byte aligned.
+ * Window arguments as for swa_forward_ex.  Runs on CUDA cores (fp32 math):
+ * one warp per (batch, row, kv head) with dk / dv summed in a library-owned
+ * fp32 workspace (2 * B * N * Hkv * D floats, kept until swa_release), then
+ * rounded to bf16.  D in {64, 128}; H / Hkv <= 8.
+ */
+SWA_API int swa_backward(const void* q, const void* k, const void* v, const void* out,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int Hkv, int N, int D, int win_left, int win_right, int dilation,
+                         int dilation_block, const int32_t* global_idx, int n_global,
+                         float scale, void* stream);
+
+/*
  * swa_forward_f32 -- the same operation in fp32 (q, k, v, out are float*),
  * computed with fp32 FFMA on CUDA cores (no TF32), for callers that need
  * fp32 accuracy.  D in {32, 64, 96, 128}; any dilation_block >= 0.

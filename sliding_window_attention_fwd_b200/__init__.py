@@ -12,6 +12,7 @@ from .binding import (  # noqa: F401
     SwaError,
     library_path,
     swa_append,
+    swa_backward,
     swa_decode,
     swa_decode_ex,
     swa_decode_noalloc,

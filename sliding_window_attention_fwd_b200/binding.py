@@ -44,6 +44,8 @@ class SwaLayer(ctypes.Structure):
 
 
 _lib.swa_forward_layers.argtypes = [_P, _I, _I, _I, _I, _I, _I, _P, _P]
+_lib.swa_backward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                              _I, _P, _I, _F, _P]
 _lib.swa_device_error.argtypes = [_P]
 _lib.swa_selftest_timeout.argtypes = [_I, _P]
 _lib.swa_schedule.argtypes = [_I, _I, _I, _I, _I, _P, _I]
@@ -53,6 +55,7 @@ _lib.swa_status_string.restype = ctypes.c_char_p
 _lib.swa_version.argtypes = []
 for _fn in ("swa_forward", "swa_forward_ex", "swa_forward_f32", "swa_decode", "swa_decode_ex",
             "swa_decode_paged", "swa_paged_window", "swa_append", "swa_forward_layers",
+            "swa_backward",
             "swa_device_error", "swa_selftest_timeout", "swa_schedule", "swa_release",
             "swa_version"):
     getattr(_lib, _fn).restype = _I
@@ -173,6 +176,27 @@ def swa_forward_layers(layers, stream=None):
                                  ctypes.byref(bad), _stream(stream))
     _check(st, f"swa_forward_layers (layer {bad.value})")
     return outs
+
+
+def swa_backward(q, k, v, out, dout, lse, win_left=-1, win_right=-1, dilation=1,
+                 dilation_block=0, global_idx=None, scale=0.0, dq=None, dk=None, dv=None,
+                 stream=None):
+    """Gradients (dq, dk, dv) of swa_forward_ex (C: swa_backward); out and lse
+    are the forward's outputs for the same arguments."""
+    B, N, H, Hkv, D, out, gi, ng = _fwd_common(q, k, v, out, lse, global_idx, torch.bfloat16)
+    _need(dout, "dout", torch.bfloat16, 4)
+    if lse is None:
+        raise ValueError("lse (from the forward) is required")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, n, torch.bfloat16, 4)
+    _check(_lib.swa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                             _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, D, int(win_left),
+                             int(win_right), int(dilation), int(dilation_block), _ptr(gi), ng,
+                             float(scale), _stream(stream)), "swa_backward")
+    return dq, dk, dv
 
 
 def swa_forward_f32(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dilation=1,

@@ -189,6 +189,25 @@ SWA_API int swa_forward_layers(const swa_layer* layers, int n_layers, int B, int
   return SWA_OK;
 }
 
+SWA_API int swa_backward(const void* q, const void* k, const void* v, const void* out,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int Hkv, int N, int D, int win_left, int win_right, int dilation,
+                         int dilation_block, const int32_t* global_idx, int n_global,
+                         float scale, void* stream) {
+  int st = check_forward_bf16(q, k, v, const_cast<void*>(out), nullptr, B, H, Hkv, N, D, dilation,
+                              dilation_block, global_idx, n_global);
+  if (st != SWA_OK) return st;
+  if (!dout || !lse || !dq || !dk || !dv) return SWA_ERR_ARG;
+  if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return SWA_ERR_ALIGN;
+  if (H / Hkv > 8) return SWA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) return SWA_OK;
+  return launch_backward(q, k, v, out, dout, lse, dq, dk, dv, B, H, Hkv, N, D, win_left,
+                         win_right, dilation, dilation_block, global_idx, n_global,
+                         resolve_scale(scale, D), static_cast<cudaStream_t>(stream));
+}
+
 SWA_API int swa_forward_f32(const float* q, const float* k, const float* v, float* out,
                             float* lse, int B, int H, int Hkv, int N, int D, int win_left,
                             int win_right, int dilation, int dilation_block,
@@ -348,6 +367,7 @@ SWA_API int swa_schedule(int N, int win_left, int win_right, int dilation, int d
 
 SWA_API int swa_release(void) {
   release_workspaces();
+  release_backward_workspace();
   return SWA_OK;
 }
 

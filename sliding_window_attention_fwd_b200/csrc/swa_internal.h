@@ -53,5 +53,10 @@ int launch_append(const void* q, const void* k_new, const void* v_new, void* k_r
                   void* out, float* lse, const int64_t* pos0, int B, int C, int H, int Hkv, int D,
                   int W, float scale, cudaStream_t stream);
 void release_workspaces();
+int launch_backward(const void* q, const void* k, const void* v, const void* out,
+                    const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                    int H, int Hkv, int N, int D, int L, int R, int d, int bs, const int32_t* G,
+                    int ng, float scale, cudaStream_t stream);
+void release_backward_workspace();
 
 }  // namespace swa
