@@ -37,6 +37,36 @@ struct BwdParams {
 
 __device__ __forceinline__ float bf(uint16_t x) { return __uint_as_float((uint32_t)x << 16); }
 
+// NV contiguous bf16 values (NV = 2 or 4) -> fp32
+template <int NV>
+__device__ __forceinline__ void load_bf(const uint16_t* src, float (&x)[NV]) {
+  if (NV == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(src);
+    x[0] = __uint_as_float(w.x << 16);
+    x[NV > 1 ? 1 : 0] = __uint_as_float(w.x & 0xFFFF0000u);
+    x[NV > 2 ? 2 : 0] = __uint_as_float(w.y << 16);
+    x[NV > 3 ? 3 : 0] = __uint_as_float(w.y & 0xFFFF0000u);
+  } else {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(src);
+    x[0] = __uint_as_float(w << 16);
+    x[NV > 1 ? 1 : 0] = __uint_as_float(w & 0xFFFF0000u);
+  }
+}
+
+// adds NV contiguous floats with one vector reduction (no return value)
+template <int NV>
+__device__ __forceinline__ void red_add(float* dst, const float (&x)[NV]) {
+  if (NV == 4) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(x[0]),
+                 "f"(x[NV > 1 ? 1 : 0]), "f"(x[NV > 2 ? 2 : 0]), "f"(x[NV > 3 ? 3 : 0])
+                 : "memory");
+  } else {
+    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(dst), "f"(x[0]),
+                 "f"(x[NV > 1 ? 1 : 0])
+                 : "memory");
+  }
+}
+
 __device__ __forceinline__ bool is_global(const int32_t* G, int ng, int i) {
   int lo = 0, hi = ng - 1;
   while (lo <= hi) {
@@ -78,19 +108,23 @@ __global__ void __launch_bounds__(128) swa_bwd_rows_kernel(BwdParams p) {
   const float kLog2e = 1.4426950408889634f;
   const float c2 = p.scale * kLog2e;
 
+  // lane owns the NV contiguous columns [NV * lane, NV * lane + NV)
+  const int c0 = NV * lane;
   float qv[NQ][NV], dov[NQ][NV], dq[NQ][NV], lse2[NQ], Dsum[NQ];
 #pragma unroll
   for (int s = 0; s < NQ; ++s) {
     const bool ok = s < p.grp;
     const int h = g * p.grp + (ok ? s : 0);
     const long row = (((long)b * p.N + i) * p.H + h) * p.D;
+    float ov[NV];
+    load_bf<NV>(p.q + row + c0, qv[s]);
+    load_bf<NV>(p.dout + row + c0, dov[s]);
+    load_bf<NV>(p.out + row + c0, ov);
     float dsum = 0.f;
 #pragma unroll
     for (int t = 0; t < NV; ++t) {
-      const int c = lane + 32 * t;
-      qv[s][t] = ok ? bf(p.q[row + c]) : 0.f;
-      dov[s][t] = ok ? bf(p.dout[row + c]) : 0.f;
-      dsum = fmaf(dov[s][t], ok ? bf(p.out[row + c]) : 0.f, dsum);
+      if (!ok) qv[s][t] = dov[s][t] = 0.f;
+      dsum = fmaf(dov[s][t], ov[t], dsum);
       dq[s][t] = 0.f;
     }
 #pragma unroll
@@ -99,18 +133,15 @@ __global__ void __launch_bounds__(128) swa_bwd_rows_kernel(BwdParams p) {
     lse2[s] = ok ? p.lse[((long)b * p.H + h) * p.N + i] * kLog2e : INFINITY;
   }
   const long kv_stride = (long)p.Hkv * p.D;
-  const uint16_t* kb = p.k + ((long)b * p.N * p.Hkv + g) * p.D;
-  const uint16_t* vb = p.v + ((long)b * p.N * p.Hkv + g) * p.D;
-  float* dkb = p.dk_acc + ((long)b * p.N * p.Hkv + g) * p.D;
-  float* dvb = p.dv_acc + ((long)b * p.N * p.Hkv + g) * p.D;
+  const uint16_t* kb = p.k + ((long)b * p.N * p.Hkv + g) * p.D + c0;
+  const uint16_t* vb = p.v + ((long)b * p.N * p.Hkv + g) * p.D + c0;
+  float* dkb = p.dk_acc + ((long)b * p.N * p.Hkv + g) * p.D + c0;
+  float* dvb = p.dv_acc + ((long)b * p.N * p.Hkv + g) * p.D + c0;
 
   auto visit = [&](int j) {
     float kv[NV], vv[NV];
-#pragma unroll
-    for (int t = 0; t < NV; ++t) {
-      kv[t] = bf(kb[(long)j * kv_stride + lane + 32 * t]);
-      vv[t] = bf(vb[(long)j * kv_stride + lane + 32 * t]);
-    }
+    load_bf<NV>(kb + (long)j * kv_stride, kv);
+    load_bf<NV>(vb + (long)j * kv_stride, vv);
     float sc[NQ], dp[NQ];
 #pragma unroll
     for (int s = 0; s < NQ; ++s) {
@@ -145,10 +176,9 @@ __global__ void __launch_bounds__(128) swa_bwd_rows_kernel(BwdParams p) {
       }
     }
 #pragma unroll
-    for (int t = 0; t < NV; ++t) {
-      atomicAdd(dkb + (long)j * kv_stride + lane + 32 * t, dk[t] * p.scale);
-      atomicAdd(dvb + (long)j * kv_stride + lane + 32 * t, dv[t]);
-    }
+    for (int t = 0; t < NV; ++t) dk[t] *= p.scale;
+    red_add<NV>(dkb + (long)j * kv_stride, dk);
+    red_add<NV>(dvb + (long)j * kv_stride, dv);
   };
 
   // the key set of row i, walked as the forward walks it
@@ -189,10 +219,10 @@ __global__ void __launch_bounds__(128) swa_bwd_rows_kernel(BwdParams p) {
   for (int s = 0; s < NQ; ++s) {
     if (s >= p.grp) continue;
     const int h = g * p.grp + s;
-    uint16_t* drow = p.dq + (((long)b * p.N + i) * p.H + h) * p.D;
+    uint16_t* drow = p.dq + (((long)b * p.N + i) * p.H + h) * p.D + c0;
 #pragma unroll
     for (int t = 0; t < NV; ++t)
-      drow[lane + 32 * t] = __bfloat16_as_ushort(__float2bfloat16_rn(dq[s][t] * p.scale));
+      drow[t] = __bfloat16_as_ushort(__float2bfloat16_rn(dq[s][t] * p.scale));
   }
 }
 
