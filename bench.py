@@ -294,6 +294,9 @@ def run_ours(args, rank, world, local_rank):
     if args.only == "decode":
         run_decode_only(args, swa, inputs, dev, stream, flush)
         return
+    if args.only in ("paged", "append", "backward"):
+        run_next_only(args, swa, inputs, dev, stream, flush)
+        return
     barrier()
     with ClockSampler(local_rank, clock_path) as clk:
         barrier()
@@ -510,6 +513,35 @@ def run_decode_only(args, swa, inputs, dev, stream, flush):
     print(json.dumps({"only": "decode", "ms_per_step": sum(dms) / len(dms)}), flush=True)
 
 
+def run_next_only(args, swa, inputs, dev, stream, flush):
+    """One next-row workload alone (used for profiling captures)."""
+    import torch
+    if args.only == "paged":
+        c = inputs.PAGED_CONFIGS["paged_decode"]
+        q, kp, vp, tab, pos = inputs.paged_inputs(c, device=dev)
+        tab, pos = tab.to(dev), pos.to(dev)
+        o = torch.empty_like(q)
+        fn = lambda: swa.swa_decode_paged(q, kp, vp, tab, pos, c.page_size, c.W, out=o,
+                                          stream=stream)
+    elif args.only == "append":
+        c = inputs.APPEND_CONFIGS["ring_append"]
+        q, kn, vn, kr, vr, pos = inputs.append_inputs(c, device=dev)
+        pos = pos.to(dev)
+        o = torch.empty_like(q)
+        fn = lambda: swa.swa_append(q, kn, vn, kr, vr, pos, out=o, stream=stream)
+    else:
+        c = inputs.CONFIGS["mistral_causal_prefill"]
+        q, k, v, _ = inputs.forward_inputs(c, device=dev)
+        do = inputs.normal((c.B, c.N, c.H, c.D), c.seed, 9, torch.bfloat16, dev)
+        lse = torch.empty(c.B, c.H, c.N, device=dev)
+        o = swa.swa_forward(q, k, v, None, lse, c.win_left, c.win_right, stream=stream)
+        g = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+        fn = lambda: swa.swa_backward(q, k, v, o, do, lse, c.win_left, c.win_right, dq=g[0],
+                                      dk=g[1], dv=g[2], stream=stream)
+    ms = time_device(fn, args.steps, args.warmup, flush, stream)
+    print(json.dumps({"only": args.only, "ms_per_step": sum(ms) / len(ms)}), flush=True)
+
+
 def torch_empty_like(t):
     import torch
     return torch.empty_like(t)
@@ -562,7 +594,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "forward", "decode"],
+    ap.add_argument("--only", default="all",
+                    choices=["all", "forward", "decode", "paged", "append", "backward"],
                     help="run one workload alone (profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
