@@ -35,8 +35,6 @@ struct BwdParams {
   float scale;
 };
 
-__device__ __forceinline__ float bf(uint16_t x) { return __uint_as_float((uint32_t)x << 16); }
-
 // NV contiguous bf16 values (NV = 2 or 4) -> fp32
 template <int NV>
 __device__ __forceinline__ void load_bf(const uint16_t* src, float (&x)[NV]) {

@@ -623,8 +623,12 @@ int launch_rows(RowParams& p, int nsets, cudaStream_t stream) {
 // global rows and chunked append always fill 8 slots
 template <int D>
 int dispatch_nq(RowParams& p, int nq, int nsets, cudaStream_t stream) {
-  if (p.mode == 1) return nq == 8 ? launch_rows<D, 8, 1>(p, nsets, stream) : SWA_ERR_UNSUPPORTED;
-  if (p.mode == 3) return nq == 8 ? launch_rows<D, 8, 3>(p, nsets, stream) : SWA_ERR_UNSUPPORTED;
+  if (p.mode == 1)
+    return nq == 8 ? launch_rows<D, 8, 1>(p, nsets, stream)
+                   : (nq == 4 ? launch_rows<D, 4, 1>(p, nsets, stream) : SWA_ERR_UNSUPPORTED);
+  if (p.mode == 3)
+    return nq == 8 ? launch_rows<D, 8, 3>(p, nsets, stream)
+                   : (nq == 4 ? launch_rows<D, 4, 3>(p, nsets, stream) : SWA_ERR_UNSUPPORTED);
   if (p.mode == 0) {
     switch (nq) {
       case 1: return launch_rows<D, 1, 0>(p, nsets, stream);
@@ -746,7 +750,7 @@ int launch_global_rows(const void* q, const void* k, const void* v, void* out, f
   p.grp = H / Hkv;
   p.ng = ng;
   p.causal = causal ? 1 : 0;
-  const int nq = 8;
+  const int nq = p.grp <= 4 ? 4 : 8;
   p.rows_per_cta = nq / p.grp;
   p.nrowchunks = (ng + p.rows_per_cta - 1) / p.rows_per_cta;
   p.chunk = 512;
@@ -816,8 +820,8 @@ int launch_append(const void* q, const void* k_new, const void* v_new, void* k_r
   p.N = C;
   p.W = W;
   p.grp = H / Hkv;
-  const int nq = 8;
-  p.rows_per_cta = nq / p.grp;  // query tokens per CTA (8 query vectors)
+  const int nq = p.grp <= 4 ? 4 : 8;
+  p.rows_per_cta = nq / p.grp;  // query tokens per CTA
   p.nrowchunks = (C + p.rows_per_cta - 1) / p.rows_per_cta;
   // history (at most W + 64 indices from a 64-aligned start) then the chunk
   const int span = W + kRows + C;
