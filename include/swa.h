@@ -1,6 +1,7 @@
 /*
- * swa.h -- C ABI of libswa.so: sliding-window attention (SWA) forward and
- * ring-buffer decode on NVIDIA B200 (sm_100a).
+ * swa.h -- C ABI of libswa.so: sliding-window attention (SWA) on NVIDIA
+ * B200 (sm_100a): forward (also over a per-layer schedule), backward,
+ * ring-buffer and paged-cache decode, and chunked append into a ring.
  *
  * Every call is asynchronous on the CUDA stream passed as `stream` (a
  * cudaStream_t as void*; NULL = the legacy default stream).  All pointers
@@ -86,9 +87,12 @@ typedef enum {
  * 0 = causal).  dilation >= 1.  global_idx: device int32 array of n_global
  * entries (NULL iff n_global == 0).  scale <= 0 selects 1/sqrt(D) (the
  * "softmax_scale None" default on page "别再只加Mask了", §3).
- * B == 0 or N == 0 is a no-op returning SWA_OK.  The call allocates no
- * device memory.  Entries of global_idx outside [0, N) are clamped when
- * read (no out-of-bounds access) but then the result is unspecified.
+ * B == 0 or N == 0 is a no-op returning SWA_OK.  Without global tokens the
+ * call allocates no device memory; with them, the global query rows use the
+ * library-owned split workspace of the row kernel (allocated on the first
+ * such call on a device, kept until swa_release).  Entries of global_idx
+ * outside [0, N) are clamped when read (no out-of-bounds access) but then
+ * the result is unspecified.
  */
 SWA_API int swa_forward(const void* q, const void* k, const void* v, void* out,
                         float* lse, int B, int H, int Hkv, int N, int D,
@@ -321,7 +325,9 @@ SWA_API int swa_selftest_timeout(int limit_us, void* stream);
 SWA_API int swa_schedule(int N, int win_left, int win_right, int dilation,
                          int dilation_block, int32_t* tile_out, int cap);
 
-/* swa_release -- frees library-owned workspaces on the current device. */
+/* swa_release -- frees every library-owned workspace (the row kernel's
+   split workspaces and the backward's accumulators) on every device that
+   has one, after synchronising that device; later calls allocate again. */
 SWA_API int swa_release(void);
 
 /* swa_status_string -- static text for a status code. */
