@@ -73,6 +73,13 @@ struct FwdParams {
   int qtile_prefix[kMaxClasses + 1];
   int Mv[kMaxClasses];
   float scale_log2;
+  // Query window (chunked append; pos0 == NULL otherwise): the Mq query
+  // rows are local rows 0..Mq-1 of q / out / lse ([B, Mq, H, D] /
+  // [B, H, Mq]) and sit at virtual rows q0.. of the key sequence, whose
+  // row v holds position pos0[b] - (win - 1) + v; rows of negative
+  // positions (v < win - 1 - pos0[b]) are masked.
+  const int64_t* pos0;
+  int q0, Mq, win;
 };
 
 template <int D, int NSLOT, int NSTREAM>
@@ -97,7 +104,9 @@ struct Cfg {
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
-template <int D, int NSLOT, int NSTREAM>
+// QWIN: the query window of a chunked append (compile-time, so the plain
+// forward carries none of its row mapping).
+template <int D, int NSLOT, int NSTREAM, bool QWIN>
 __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     swa_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
   using C = Cfg<D, NSLOT, NSTREAM>;
@@ -147,7 +156,18 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
   }
   const Geometry g = make_geometry(p.N, p.L, p.R, p.d, p.bs);
   const int Mv = p.Mv[cl];
-  const TileRange tr = tile_range(g, Mv, qt);
+  constexpr bool qwin = QWIN;
+  const int Mq = qwin ? p.Mq : Mv;  // query rows (local)
+  const int q0 = qwin ? p.q0 : 0;   // virtual row of local query row 0
+  const int qm0 = q0 + qt * kTileM;
+  const int qm1 = q0 + min(qt * kTileM + kTileM - 1, Mq - 1);
+  const TileRange tr = tile_range_rows(g, Mv, qm0, qm1);
+  int lo_b = 0;  // first key row holding a real position (query window only)
+  if (qwin) {
+    const long long pb = p.pos0[b];
+    const long long lb = (long long)(p.win - 1) - pb;
+    lo_b = lb <= 0 ? 0 : (lb > Mv ? Mv : (int)lb);
+  }
   const int n_band = tr.kv_end - tr.kv_begin;
   const int n_gtiles = (p.n_global + kTileN - 1) / kTileN;
   const int n_tiles = n_band + n_gtiles;
@@ -359,11 +379,12 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     const uint32_t tS = tmem + 128u * slot + lane_off;
     const uint32_t tO = tmem + 256u + 128u * slot + lane_off;
     const int h = head[slot];
-    const int m_row = qt * kTileM + r;
-    const bool row_valid = m_row < Mv && slot_ok[slot];
-    const int klo = key_lo(g, m_row);
-    const int khi = key_hi(g, m_row, Mv);
-    const int i_phys = (int)phys_row(g, c, m_row);
+    const int m_row = qt * kTileM + r;  // local query row
+    const bool row_valid = m_row < Mq && slot_ok[slot];
+    const int m_v = q0 + m_row;         // its virtual row among the keys
+    const int klo = max(key_lo(g, m_v), lo_b);
+    const int khi = key_hi(g, m_v, Mv);
+    const int i_phys = (int)phys_row(g, c, m_v);
     const bool causal = p.R == 0;
     // band of the row in physical positions, for the global-key test
     const int glo = p.L < 0 ? -0x40000000
@@ -379,7 +400,8 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
 
     float m_pend = -INFINITY;  // max seen but not yet adopted (adopted next tile)
     int int_lo, int_hi;        // key tiles that need no element mask
-    interior_tiles(g, Mv, qt, &int_lo, &int_hi);
+    interior_tiles_rows(g, Mv, qm0, &int_lo, &int_hi);
+    if (lo_b > 0 || qt * kTileM + kTileM > Mq) int_hi = int_lo - 1;  // mask every tile
 
     // the 64 score columns of key half hf (TMEM -> registers)
     auto read_half = [&](int hf, float (&sv)[64]) {
@@ -571,7 +593,8 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
       const float inv = 1.f / l;
-      uint16_t* orow = p.out + (((size_t)b * p.N + i_phys) * p.H + h) * D;
+      const size_t orow_i = qwin ? (size_t)b * Mq + m_row : (size_t)b * p.N + i_phys;
+      uint16_t* orow = p.out + (orow_i * p.H + h) * D;
 #pragma unroll
       for (int j = 0; j < D / 32; ++j) {
         uint32_t v[32];
@@ -590,7 +613,8 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
         }
       }
       if (row_valid && p.lse)
-        p.lse[((size_t)b * p.H + h) * p.N + i_phys] = (m_used + __log2f(l)) * 0.69314718055994531f;
+        p.lse[((size_t)b * p.H + h) * (qwin ? Mq : p.N) + (qwin ? m_row : i_phys)] =
+            (m_used + __log2f(l)) * 0.69314718055994531f;
     }
   }
 
@@ -614,11 +638,13 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
 template <int D, int NSLOT, int NSTREAM>
 int launch_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
                 int Hkv, int N, int L, int R, int d, int bs, const int32_t* G, int ng,
-                float scale, cudaStream_t stream) {
+                float scale, cudaStream_t stream, const QueryWindow* qw) {
   using C = Cfg<D, NSLOT, NSTREAM>;
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM>,
+    if (cudaFuncSetAttribute(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess ||
+        cudaFuncSetAttribute(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, true>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess)
       return SWA_ERR_CUDA;
     attr_set = true;
@@ -651,7 +677,14 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
     p.qtile_prefix[0] = 0;
     for (int cl = 0; cl < p.nclass; ++cl) {
       p.Mv[cl] = class_valid_rows(geo, c0 + cl);
-      p.qtile_prefix[cl + 1] = p.qtile_prefix[cl] + (p.Mv[cl] + kTileM - 1) / kTileM;
+      const int rows_q = qw ? qw->Mq : p.Mv[cl];
+      p.qtile_prefix[cl + 1] = p.qtile_prefix[cl] + (rows_q + kTileM - 1) / kTileM;
+    }
+    if (qw) {
+      p.pos0 = qw->pos0;
+      p.q0 = qw->q0;
+      p.Mq = qw->Mq;
+      p.win = qw->win;
     }
     const uint32_t box[4] = {64, 1, (uint32_t)kBlockRows, 1};
     const int nmaps = block_mode ? 1 : p.nclass;
@@ -661,8 +694,10 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
       const uint64_t rstep = block_mode ? 1 : (uint64_t)d;
       const size_t qoff = block_mode ? 0 : (size_t)cc * H * D;
       const size_t kvoff = block_mode ? 0 : (size_t)cc * Hkv * D;
-      const uint64_t dq[4] = {(uint64_t)D, (uint64_t)H, rows, (uint64_t)B};
-      const uint64_t sq[3] = {(uint64_t)D * 2, rstep * H * D * 2, (uint64_t)N * H * D * 2};
+      const uint64_t qrows = qw ? (uint64_t)qw->Mq : rows;
+      const uint64_t qN = qw ? (uint64_t)qw->Mq : (uint64_t)N;
+      const uint64_t dq[4] = {(uint64_t)D, (uint64_t)H, qrows, (uint64_t)B};
+      const uint64_t sq[3] = {(uint64_t)D * 2, rstep * H * D * 2, qN * H * D * 2};
       const uint64_t dk[4] = {(uint64_t)D, (uint64_t)Hkv, rows, (uint64_t)B};
       const uint64_t sk[3] = {(uint64_t)D * 2, rstep * Hkv * D * 2, (uint64_t)N * Hkv * D * 2};
       void* qb = (void*)(static_cast<const uint16_t*>(q) + qoff);
@@ -679,7 +714,12 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
     const long grid = (long)p.qtile_prefix[p.nclass] * B * ((H + NSLOT - 1) / NSLOT);
     if (grid <= 0) continue;
     if (grid > 0x7fffffffL) return SWA_ERR_UNSUPPORTED;
-    swa_fwd_sm100_kernel<D, NSLOT, NSTREAM><<<(unsigned)grid, C::kThreads, C::kAlloc, stream>>>(p);
+    if (qw)
+      swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, true><<<(unsigned)grid, C::kThreads, C::kAlloc,
+                                                      stream>>>(p);
+    else
+      swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, false><<<(unsigned)grid, C::kThreads, C::kAlloc,
+                                                       stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
   }
   return SWA_OK;
@@ -692,21 +732,21 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
 // per CTA otherwise.
 int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                      int H, int Hkv, int N, int D, int L, int R, int d, int bs, const int32_t* G,
-                     int ng, float scale, cudaStream_t stream) {
+                     int ng, float scale, cudaStream_t stream, const QueryWindow* qw) {
   const bool gqa_pair = (H / Hkv) % 2 == 0;
   if (D == 128) {
     if (gqa_pair)
       return launch_impl<128, 2, 1>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
-                                    stream);
+                                    stream, qw);
     return launch_impl<128, 1, 1>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
-                                  stream);
+                                  stream, qw);
   }
   if (D == 64) {
     if (gqa_pair)
       return launch_impl<64, 2, 1>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
-                                   stream);
+                                   stream, qw);
     return launch_impl<64, 2, 2>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
-                                 stream);
+                                 stream, qw);
   }
   return SWA_ERR_UNSUPPORTED;
 }

@@ -22,9 +22,18 @@ int launch_fwd_f32(const float* q, const float* k, const float* v, float* out, f
                    int B, int H, int Hkv, int N, int D, int L, int R, int d, int bs,
                    const int32_t* G, int ng, float scale, cudaStream_t stream);
 
+// Query window of the forward (chunked append): the Mq query rows are the
+// local rows of q / out / lse and sit at virtual rows q0.. of the key
+// sequence, whose row v holds position pos0[b] - (win - 1) + v (device
+// array; rows of negative positions are masked).
+struct QueryWindow {
+  const int64_t* pos0;
+  int q0, Mq, win;
+};
 int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, float* lse,
                      int B, int H, int Hkv, int N, int D, int L, int R, int d, int bs,
-                     const int32_t* G, int ng, float scale, cudaStream_t stream);
+                     const int32_t* G, int ng, float scale, cudaStream_t stream,
+                     const QueryWindow* qw = nullptr);
 
 // Dense rows for global queries: every global row i attends keys
 // [0, N) (causal: [0, i]); overwrites those rows of out / lse.

@@ -550,7 +550,8 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
 
 // ------------------------------------------------------------ workspaces
 // Per device and per user (0: decode, 1: global rows, 2: paged decode,
-// 3: chunked append): split counters and
+// 3: chunked append, 4: the staged key sequence of a tensor-core append):
+// split counters and
 // split partials in separate buffers.  Every merge resets its counter to
 // zero, so between complete calls all counters are zero; the counter buffer
 // is zeroed whenever it is (re)allocated and is never overlapped by the
@@ -562,7 +563,7 @@ struct Workspace {
   size_t part_bytes = 0;
 };
 constexpr int kMaxDev = 64;
-Workspace g_ws[kMaxDev][4];  // users: decode, global rows, paged, append
+Workspace g_ws[kMaxDev][5];  // users: decode, global rows, paged, append, append staging
 std::mutex g_ws_mu;
 
 bool get_workspace(int which, size_t cnt_bytes, size_t part_bytes, cudaStream_t stream,
@@ -698,6 +699,38 @@ __global__ void ring_store_kernel(const uint4* __restrict__ k_new, const uint4* 
   v_ring[dst] = v_new[src];
 }
 
+// Stages the key / value sequence of a chunked append for the tensor-core
+// forward: row v holds position pos0[b] - (W - 1) + v, taken from the ring
+// (slot position % W) below pos0 and from the chunk from pos0 on; rows of
+// negative positions are zeros (the forward masks them).  16 B per thread.
+__global__ void append_stage_kernel(const uint4* __restrict__ k_ring,
+                                    const uint4* __restrict__ v_ring,
+                                    const uint4* __restrict__ k_new,
+                                    const uint4* __restrict__ v_new, uint4* __restrict__ ks,
+                                    uint4* __restrict__ vs, const int64_t* __restrict__ pos0,
+                                    int B, int C, int W, int Nv, int row_vecs) {
+  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= (long long)B * Nv * row_vecs) return;
+  const int i = (int)(t % row_vecs);
+  const int v = (int)((t / row_vecs) % Nv);
+  const int b = (int)(t / ((long long)row_vecs * Nv));
+  const long long p0 = pos0[b];
+  const long long pos = p0 - (W - 1) + v;
+  uint4 kk = make_uint4(0u, 0u, 0u, 0u), vv = kk;
+  if (pos >= p0) {
+    const long src = ((long)b * C + (pos - p0)) * row_vecs + i;
+    kk = k_new[src];
+    vv = v_new[src];
+  } else if (pos >= 0) {
+    const long src = ((long)b * W + pos % W) * row_vecs + i;
+    kk = k_ring[src];
+    vv = v_ring[src];
+  }
+  const long dst = ((long)b * Nv + v) * row_vecs + i;
+  ks[dst] = kk;
+  vs[dst] = vv;
+}
+
 }  // namespace
 
 int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* out, float* lse,
@@ -797,9 +830,63 @@ int launch_decode_paged(const void* q, const void* k_pages, const void* v_pages,
   return run(p, D, nq, B * Hkv, 2, stream);
 }
 
+namespace {
+// The new tokens enter the ring (launched after every query has read the
+// slots they overwrite); of a chunk longer than W only the last W stay.
+int ring_store(const void* k_new, const void* v_new, void* k_ring, void* v_ring,
+               const int64_t* pos0, int B, int C, int Hkv, int D, int W, cudaStream_t stream) {
+  const int c_first = C > W ? C - W : 0;
+  const int row_vecs = Hkv * D / 8;
+  dim3 grid((row_vecs + 255) / 256, C - c_first, B);
+  ring_store_kernel<<<grid, 256, 0, stream>>>(
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+      static_cast<uint4*>(k_ring), static_cast<uint4*>(v_ring), pos0, C, W, row_vecs, c_first);
+  return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+}  // namespace
+
+namespace {
+// Chunks of 32 tokens and more: stage the chunk's key sequence contiguously
+// (ring history below pos0, then the chunk) and run the tcgen05 forward
+// over it with a causal window of W keys, its queries being the last C
+// rows.  Shorter chunks would leave most of a 128-row query tile idle and
+// take the row kernel below.
+int append_attention_tc(const void* q, const void* k_new, const void* v_new, const void* k_ring,
+                        const void* v_ring, void* out, float* lse, const int64_t* pos0, int B,
+                        int C, int H, int Hkv, int D, int W, float scale, cudaStream_t stream) {
+  const long long Nv = (long long)W - 1 + C;
+  if (Nv > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  const size_t half = (size_t)B * Nv * Hkv * D * 2;
+  int* cnt = nullptr;
+  void* part = nullptr;
+  if (!get_workspace(4, 256, 2 * half, stream, &cnt, &part)) return SWA_ERR_NOMEM;
+  uint8_t* ks = static_cast<uint8_t*>(part);
+  uint8_t* vs = ks + half;
+  const int row_vecs = Hkv * D / 8;
+  const long long n = (long long)B * Nv * row_vecs;
+  const long long blocks = (n + 255) / 256;
+  if (blocks > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  append_stage_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+      static_cast<const uint4*>(k_ring), static_cast<const uint4*>(v_ring),
+      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
+      reinterpret_cast<uint4*>(ks), reinterpret_cast<uint4*>(vs), pos0, B, C, W, (int)Nv,
+      row_vecs);
+  if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
+  const QueryWindow qw{pos0, W - 1, C, W};
+  return launch_fwd_sm100(q, ks, vs, out, lse, B, H, Hkv, (int)Nv, D, W - 1, 0, 1, 0, nullptr, 0,
+                          scale, stream, &qw);
+}
+}  // namespace
+
 int launch_append(const void* q, const void* k_new, const void* v_new, void* k_ring, void* v_ring,
                   void* out, float* lse, const int64_t* pos0, int B, int C, int H, int Hkv, int D,
                   int W, float scale, cudaStream_t stream) {
+  if (C >= 32) {
+    const int st = append_attention_tc(q, k_new, v_new, k_ring, v_ring, out, lse, pos0, B, C, H,
+                                       Hkv, D, W, scale, stream);
+    if (st != SWA_OK) return st;
+    return ring_store(k_new, v_new, k_ring, v_ring, pos0, B, C, Hkv, D, W, stream);
+  }
   RowParams p;
   std::memset(&p, 0, sizeof(p));
   if (encode_kv(&p.tmK, k_ring, D, Hkv, W, B) != SWA_OK ||
@@ -830,21 +917,13 @@ int launch_append(const void* q, const void* k_new, const void* v_new, void* k_r
   p.scale_log2 = scale * 1.4426950408889634f;
   const int st = run(p, D, nq, B * Hkv * p.nrowchunks, 3, stream);
   if (st != SWA_OK) return st;
-  // then the new tokens enter the ring (after every query has read the
-  // slots they overwrite); of a chunk longer than W only the last W stay
-  const int c_first = C > W ? C - W : 0;
-  const int row_vecs = Hkv * D / 8;
-  dim3 grid((row_vecs + 255) / 256, C - c_first, B);
-  ring_store_kernel<<<grid, 256, 0, stream>>>(
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
-      static_cast<uint4*>(k_ring), static_cast<uint4*>(v_ring), pos0, C, W, row_vecs, c_first);
-  return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+  return ring_store(k_new, v_new, k_ring, v_ring, pos0, B, C, Hkv, D, W, stream);
 }
 
 void release_workspaces() {
   std::lock_guard<std::mutex> lk(g_ws_mu);
   for (int d = 0; d < kMaxDev; ++d)
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < 5; ++w) {
       Workspace& ws = g_ws[d][w];
       if (!ws.cnt && !ws.part) continue;
       int cur = 0;

@@ -107,11 +107,9 @@ struct TileRange {
   int kv_begin, kv_end;  // kv tiles [begin, end) of the class
 };
 
-// KV tiles needed by query tile qt of a class with Mv valid rows.
-SWA_HD TileRange tile_range(const Geometry& g, int Mv, int qt) {
-  int m0 = qt * kTileM;
-  int m1 = m0 + kTileM - 1;
-  if (m1 > Mv - 1) m1 = Mv - 1;
+// KV tiles needed by the query rows [m0, m1] of a class whose keys are its
+// Mv valid rows.
+SWA_HD TileRange tile_range_rows(const Geometry& g, int Mv, int m0, int m1) {
   int lo = key_lo(g, m0);
   if (lo < 0) lo = 0;
   int hi = key_hi(g, m1, Mv);
@@ -123,13 +121,20 @@ SWA_HD TileRange tile_range(const Geometry& g, int Mv, int qt) {
   return r;
 }
 
-// KV tiles [*lo, *hi] of query tile qt whose every (row, key) pair is inside
-// the window and in range, so they need no element mask (empty when
-// *lo > *hi).  Key bounds are monotone in the row, so the keys every row of
-// the tile sees are [key_lo(last row), key_hi(first row)], and those tiles
-// form one contiguous run.
-SWA_HD void interior_tiles(const Geometry& g, int Mv, int qt, int* lo, int* hi) {
-  const int m0 = qt * kTileM;
+// KV tiles needed by query tile qt of a class with Mv valid rows.
+SWA_HD TileRange tile_range(const Geometry& g, int Mv, int qt) {
+  int m0 = qt * kTileM;
+  int m1 = m0 + kTileM - 1;
+  if (m1 > Mv - 1) m1 = Mv - 1;
+  return tile_range_rows(g, Mv, m0, m1);
+}
+
+// KV tiles [*lo, *hi] of the 128 query rows [m0, m0 + 127] whose every
+// (row, key) pair is inside the window and in range, so they need no
+// element mask (empty when *lo > *hi).  Key bounds are monotone in the row,
+// so the keys every row sees are [key_lo(last row), key_hi(first row)], and
+// those tiles form one contiguous run.
+SWA_HD void interior_tiles_rows(const Geometry& g, int Mv, int m0, int* lo, int* hi) {
   const int m1 = m0 + kTileM - 1;
   *lo = 1;
   *hi = 0;
@@ -140,6 +145,11 @@ SWA_HD void interior_tiles(const Geometry& g, int Mv, int qt, int* lo, int* hi) 
   if (b > Mv - 1) b = Mv - 1;
   *lo = (a + kTileN - 1) / kTileN;
   *hi = (b + 1) / kTileN - 1;
+}
+
+// The same for query tile qt of a class with Mv valid rows.
+SWA_HD void interior_tiles(const Geometry& g, int Mv, int qt, int* lo, int* hi) {
+  interior_tiles_rows(g, Mv, qt * kTileM, lo, hi);
 }
 
 }  // namespace swa
