@@ -10,6 +10,12 @@
  * returns.  Arguments are validated on the host before anything is
  * launched: on failure the call returns a negative swa_status and launches
  * nothing.  No call synchronises the stream; swa_device_error() does.
+ * Library-owned device workspaces (split partials of the decode / global
+ * row / paged / append kernels, the staged keys of a long append, the
+ * backward's accumulators) are one per device and per use: two calls that
+ * use the same one must not run on the device at the same time, whichever
+ * streams they are on.  Workspaces grow on demand (the growing call
+ * synchronises its stream first) and are freed by swa_release().
  *
  * Definitions (page title, section):
  *  - Window and output: "滑动窗口注意力" (bmjup.com/post/11897), section
