@@ -27,6 +27,26 @@ def test_pair_counts_match_oracle_key_sets(N, L, R, d, bs, G):
     assert bench.in_window_pairs(N, L, R, d, bs, G) == ref
 
 
+@pytest.mark.parametrize("N,L,R,d,G", [
+    # the layer kinds of the bench's hybrid schedule, shrunk: causal dilated
+    # windows, a full causal layer, a causal window with attention sinks
+    (300, 63, 0, 2, ()), (300, 31, 0, 4, ()), (300, -1, 0, 1, ()), (300, 100, 0, 1, (0, 1, 2, 3)),
+])
+def test_schedule_pair_counts_match_oracle(N, L, R, d, G):
+    ref = sum(len(oracle.key_set(i, N, L, R, d, 0, G)) for i in range(N))
+    assert bench.in_window_pairs(N, L, R, d, 0, G) == ref
+
+
+def test_append_pair_count_matches_oracle():
+    """The append FLOP count: token c at position p0 + c sees min(W, p0 + c + 1)
+    keys -- the size of the oracle's causal key set of that position."""
+    W = 64
+    for p0 in (0, 10, 63, 64, 200):
+        for c in range(5):
+            p = p0 + c
+            assert min(W, p + 1) == len(oracle.key_set(p, p + 1, W - 1, 0))
+
+
 def test_workload_pair_counts():
     assert bench.in_window_pairs(8192, 4095, 0, 1, 0, (), 1, 32) == 805_371_904
     assert bench.in_window_pairs(4096, 256, 256, 1, 0, range(0, 4096, 512), 4, 12) == 100_475_520
