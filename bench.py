@@ -289,8 +289,10 @@ def run_ours(args, rank, world, local_rank):
     def max_over_ranks(x):
         return reduce_max(x, world, dev)
 
-    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-    clock_path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{rank}.csv") if rank == 0 else None
+    clock_path = None
+    if args.clock_log and rank == 0:
+        os.makedirs(os.path.dirname(os.path.abspath(args.clock_log)), exist_ok=True)
+        clock_path = args.clock_log
     if args.only == "decode":
         run_decode_only(args, swa, inputs, dev, stream, flush)
         return
@@ -596,6 +598,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clock-log", default=None,
+                    help="also write the clock samples of the timed region to this CSV file")
     ap.add_argument("--only", default="all",
                     choices=["all", "forward", "decode", "paged", "append", "backward"],
                     help="run one workload alone (profiling captures)")
