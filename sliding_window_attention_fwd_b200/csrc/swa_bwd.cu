@@ -94,6 +94,48 @@ __device__ __forceinline__ bool in_band(const BwdParams& p, int i, int j) {
   return true;
 }
 
+// Sums each of the K values (K a power of two, 2..16) over the 32 lanes of
+// the warp and returns all K sums to every lane, with K - 1 + (5 - log2 K)
+// exchanges for the reduction and K for the broadcast (a plain butterfly
+// per value takes 5 K).  Reduction: at each of the first log2 K levels a
+// lane keeps the half of its values selected by its lane bit and sends the
+// other half to its partner; after them lane l holds a partial sum of one
+// value, which the remaining levels complete.  Broadcast: every sum is read
+// from a lane that holds it.
+template <int K>
+__device__ __forceinline__ void warp_allreduce(float (&v)[K], int lane) {
+  constexpr int kLog = K == 2 ? 1 : (K == 4 ? 2 : (K == 8 ? 3 : 4));
+  static_assert((1 << kLog) == K, "K must be 2, 4, 8 or 16");
+  float w[K];
+#pragma unroll
+  for (int i = 0; i < K; ++i) w[i] = v[i];
+#pragma unroll
+  for (int lvl = 0; lvl < kLog; ++lvl) {
+    const int o = 16 >> lvl;
+    const int h = K >> (lvl + 1);
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < K / 2; ++i) {
+      if (i < h) {
+        const float send = upper ? w[i] : w[i + h];
+        const float keep = upper ? w[i + h] : w[i];
+        w[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16 >> kLog; o > 0; o >>= 1) w[0] += __shfl_xor_sync(0xffffffffu, w[0], o);
+  // the sum of value t sits in the lanes whose bits (4 - l) spell t's bits
+  // (kLog - 1 - l), l = 0 .. kLog - 1
+#pragma unroll
+  for (int t = 0; t < K; ++t) {
+    int owner = 0;
+#pragma unroll
+    for (int l = 0; l < kLog; ++l) owner |= ((t >> (kLog - 1 - l)) & 1) << (4 - l);
+    v[t] = __shfl_sync(0xffffffffu, w[0], owner);
+  }
+}
+
 template <int NV, int NQ>  // NV = D / 32 values per lane; NQ = query heads per warp
 __global__ void __launch_bounds__(128) swa_bwd_rows_kernel(BwdParams p) {
   const long warp = (long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
@@ -140,7 +182,7 @@ __global__ void __launch_bounds__(128) swa_bwd_rows_kernel(BwdParams p) {
     float kv[NV], vv[NV];
     load_bf<NV>(kb + (long)j * kv_stride, kv);
     load_bf<NV>(vb + (long)j * kv_stride, vv);
-    float sc[NQ], dp[NQ];
+    float red[2 * NQ];  // scores, then dO . v, of every head
 #pragma unroll
     for (int s = 0; s < NQ; ++s) {
       float a = 0.f, e = 0.f;
@@ -149,16 +191,16 @@ __global__ void __launch_bounds__(128) swa_bwd_rows_kernel(BwdParams p) {
         a = fmaf(qv[s][t], kv[t], a);
         e = fmaf(dov[s][t], vv[t], e);
       }
-      sc[s] = a;
-      dp[s] = e;
+      red[s] = a;
+      red[NQ + s] = e;
     }
+    warp_allreduce<2 * NQ>(red, lane);
+    float sc[NQ], dp[NQ];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-      for (int s = 0; s < NQ; ++s) {
-        sc[s] += __shfl_xor_sync(0xffffffffu, sc[s], o);
-        dp[s] += __shfl_xor_sync(0xffffffffu, dp[s], o);
-      }
+    for (int s = 0; s < NQ; ++s) {
+      sc[s] = red[s];
+      dp[s] = red[NQ + s];
+    }
     float dk[NV], dv[NV];
 #pragma unroll
     for (int t = 0; t < NV; ++t) dk[t] = dv[t] = 0.f;
