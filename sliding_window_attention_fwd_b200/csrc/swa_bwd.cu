@@ -16,6 +16,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "swa_internal.h"
 
@@ -178,47 +179,72 @@ __global__ void __launch_bounds__(128) swa_bwd_rows_kernel(BwdParams p) {
   float* dkb = p.dk_acc + ((long)b * p.N * p.Hkv + g) * p.D + c0;
   float* dvb = p.dv_acc + ((long)b * p.N * p.Hkv + g) * p.D + c0;
 
+  // gradient contributions of NK key rows js[0..NK) (NK = 1 or 2; two rows
+  // give two independent dependency chains and one shared reduction)
+  auto visit_n = [&](auto nk_tag, const int (&js)[2]) {
+    constexpr int NK = decltype(nk_tag)::value;
+    float kv[NK][NV], vv[NK][NV];
+#pragma unroll
+    for (int u = 0; u < NK; ++u) {
+      load_bf<NV>(kb + (long)js[u] * kv_stride, kv[u]);
+      load_bf<NV>(vb + (long)js[u] * kv_stride, vv[u]);
+    }
+    float red[2 * NQ * NK];  // per key: scores, then dO . v, of every head
+#pragma unroll
+    for (int u = 0; u < NK; ++u)
+#pragma unroll
+      for (int s = 0; s < NQ; ++s) {
+        float a = 0.f, e = 0.f;
+#pragma unroll
+        for (int t = 0; t < NV; ++t) {
+          a = fmaf(qv[s][t], kv[u][t], a);
+          e = fmaf(dov[s][t], vv[u][t], e);
+        }
+        red[2 * NQ * u + s] = a;
+        red[2 * NQ * u + NQ + s] = e;
+      }
+    warp_allreduce<2 * NQ * NK>(red, lane);
+#pragma unroll
+    for (int u = 0; u < NK; ++u) {
+      float dk[NV], dv[NV];
+#pragma unroll
+      for (int t = 0; t < NV; ++t) dk[t] = dv[t] = 0.f;
+#pragma unroll
+      for (int s = 0; s < NQ; ++s) {
+        const float P = exp2f(red[2 * NQ * u + s] * c2 - lse2[s]);  // 0 for unused slots
+        const float ds = P * (red[2 * NQ * u + NQ + s] - Dsum[s]);
+#pragma unroll
+        for (int t = 0; t < NV; ++t) {
+          dq[s][t] = fmaf(ds, kv[u][t], dq[s][t]);
+          dk[t] = fmaf(ds, qv[s][t], dk[t]);
+          dv[t] = fmaf(P, dov[s][t], dv[t]);
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < NV; ++t) dk[t] *= p.scale;
+      red_add<NV>(dkb + (long)js[u] * kv_stride, dk);
+      red_add<NV>(dvb + (long)js[u] * kv_stride, dv);
+    }
+  };
   auto visit = [&](int j) {
-    float kv[NV], vv[NV];
-    load_bf<NV>(kb + (long)j * kv_stride, kv);
-    load_bf<NV>(vb + (long)j * kv_stride, vv);
-    float red[2 * NQ];  // scores, then dO . v, of every head
-#pragma unroll
-    for (int s = 0; s < NQ; ++s) {
-      float a = 0.f, e = 0.f;
-#pragma unroll
-      for (int t = 0; t < NV; ++t) {
-        a = fmaf(qv[s][t], kv[t], a);
-        e = fmaf(dov[s][t], vv[t], e);
-      }
-      red[s] = a;
-      red[NQ + s] = e;
-    }
-    warp_allreduce<2 * NQ>(red, lane);
-    float sc[NQ], dp[NQ];
-#pragma unroll
-    for (int s = 0; s < NQ; ++s) {
-      sc[s] = red[s];
-      dp[s] = red[NQ + s];
-    }
-    float dk[NV], dv[NV];
-#pragma unroll
-    for (int t = 0; t < NV; ++t) dk[t] = dv[t] = 0.f;
-#pragma unroll
-    for (int s = 0; s < NQ; ++s) {
-      const float P = exp2f(sc[s] * c2 - lse2[s]);  // 0 for unused slots
-      const float ds = P * (dp[s] - Dsum[s]);
-#pragma unroll
-      for (int t = 0; t < NV; ++t) {
-        dq[s][t] = fmaf(ds, kv[t], dq[s][t]);
-        dk[t] = fmaf(ds, qv[s][t], dk[t]);
-        dv[t] = fmaf(P, dov[s][t], dv[t]);
+    const int js[2] = {j, j};
+    visit_n(std::integral_constant<int, 1>(), js);
+  };
+  // pairs of keys where the reduction stays within 16 values
+  constexpr bool kPairs = NQ <= 4;
+  int pend = -1;
+  auto visit_paired = [&](int j) {
+    if constexpr (!kPairs) {
+      visit(j);
+    } else {
+      if (pend < 0) {
+        pend = j;
+      } else {
+        const int js[2] = {pend, j};
+        visit_n(std::integral_constant<int, 2>(), js);
+        pend = -1;
       }
     }
-#pragma unroll
-    for (int t = 0; t < NV; ++t) dk[t] *= p.scale;
-    red_add<NV>(dkb + (long)j * kv_stride, dk);
-    red_add<NV>(dvb + (long)j * kv_stride, dv);
   };
 
   // the key set of row i, walked as the forward walks it
@@ -244,8 +270,10 @@ __global__ void __launch_bounds__(128) swa_bwd_rows_kernel(BwdParams p) {
       for (long kk = klo; kk <= khi; ++kk) {
         const long j = i + kk * p.d;
         if (j < 0 || j > jmax) continue;
-        visit((int)j);
+        visit_paired((int)j);
       }
+      if (pend >= 0) visit(pend);
+      pend = -1;
     }
     for (int t = 0; t < p.n_global; ++t) {
       int j = p.G[t];
