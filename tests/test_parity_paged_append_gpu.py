@@ -135,6 +135,9 @@ def test_append_configs(swa, name):
     (2, 17, 4, 4, 64, 192, [190, 400]),            # MHA, chunk wraps the ring
     (2, 9, 16, 2, 128, 64, [60, 2]),               # GQA 8
     (3, 64, 8, 4, 64, 256, [255, 256, 1]),         # GQA 2, D = 64
+    (2, 40, 4, 4, 64, 128, [100, 3]),              # MHA, D = 64, tensor-core path
+    (1, 33, 2, 2, 128, 64, [70]),                  # MHA, D = 128, tensor-core path
+    (2, 130, 6, 2, 128, 192, [5, 1000]),           # GQA 3, two query tiles
 ])
 def test_append_shapes(swa, B, C, H, Hkv, D, W, pos0):
     q = inputs.normal((B, C, H, D), C + W, 0)
