@@ -106,6 +106,8 @@ SMALL_BF16 = [
     (1, 2000, 2, 2, 128, 20, 30, 16, 0, None),     # d > 8 classes per launch
     (1, 1344, 2, 1, 64, 128, 128, 4, 64, None),    # block-level dilation
     (1, 1000, 2, 2, 64, 128, 0, 2, 64, [3, 500]),  # block, causal, ragged, globals
+    (1, 500, 8, 1, 128, 64, 64, 1, 0, [0, 250]),   # globals with a GQA group of 8
+    (1, 400, 8, 2, 64, 40, 0, 1, 0, [5, 399]),     # globals, GQA 4, causal, last row global
 ]
 
 
