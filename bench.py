@@ -204,6 +204,32 @@ class ClockSampler:
                 "samples": len(sel)}
 
 
+def run_others(args, swa, inputs, dev, stream, flush, peaks):
+    """The remaining forward workloads (Longformer globals, token and block
+    dilation), each timed alone with the L2 flushed before every step."""
+    import torch
+    others = {}
+    for name in ("longformer_global", "dilated_token", "dilated_block"):
+        c = inputs.CONFIGS[name]
+        oq, ok_, ov, oG = inputs.forward_inputs(c, device=dev)
+        oG = oG.to(dev) if len(oG) else None
+        oo = torch.empty_like(oq)
+        ol = torch.empty(c.B, c.H, c.N, dtype=torch.float32, device=dev)
+        fn = lambda: swa.swa_forward_ex(oq, ok_, ov, oo, ol, c.win_left, c.win_right, c.dilation,
+                                        c.dilation_block, oG, c.scale, stream)
+        oms = time_device(fn, args.steps, args.warmup, flush, stream)
+        m = sum(oms) / len(oms)
+        pr = in_window_pairs(c.N, c.win_left, c.win_right, c.dilation, c.dilation_block,
+                             [] if oG is None else oG.cpu().numpy(), c.B, c.H)
+        fl = 4.0 * c.D * pr
+        by = (oq.numel() * 2 + ok_.numel() * 2) * 2 + ol.numel() * 4
+        others[name] = {"ms": m, "tflops": fl / m / 1e9, "gbs": by / m / 1e6,
+                        "frac_tensor": fl / m / 1e9 / peaks["bf16_tflops"],
+                        "frac_hbm": by / m / 1e6 / peaks["hbm_gbs"]}
+        del oq, ok_, ov, oo, ol
+    return others
+
+
 def time_device(fn, steps, warmup, flush, stream):
     """Per-step device time (ms) with CUDA events on `stream`; L2 flushed before each step."""
     import torch
@@ -298,6 +324,11 @@ def run_ours(args, rank, world, local_rank):
         return
     if args.only in ("paged", "append", "backward"):
         run_next_only(args, swa, inputs, dev, stream, flush)
+        return
+    if args.only == "others":
+        others = run_others(args, swa, inputs, dev, stream, flush, peaks)
+        assert swa.swa_device_error(stream) == 0
+        print(json.dumps({"only": "others", **others}), flush=True)
         return
     barrier()
     with ClockSampler(local_rank, clock_path) as clk:
@@ -444,25 +475,7 @@ def run_ours(args, rank, world, local_rank):
     del bdo, bgrads
 
     # ---- the other forward workloads (parity cases; reported for context)
-    others = {}
-    for name in ("longformer_global", "dilated_token", "dilated_block"):
-        c = inputs.CONFIGS[name]
-        oq, ok_, ov, oG = inputs.forward_inputs(c, device=dev)
-        oG = oG.to(dev) if len(oG) else None
-        oo = torch.empty_like(oq)
-        ol = torch.empty(c.B, c.H, c.N, dtype=torch.float32, device=dev)
-        fn = lambda: swa.swa_forward_ex(oq, ok_, ov, oo, ol, c.win_left, c.win_right, c.dilation,
-                                        c.dilation_block, oG, c.scale, stream)
-        oms = time_device(fn, args.steps, args.warmup, flush, stream)
-        m = sum(oms) / len(oms)
-        pr = in_window_pairs(c.N, c.win_left, c.win_right, c.dilation, c.dilation_block,
-                             [] if oG is None else oG.cpu().numpy(), c.B, c.H)
-        fl = 4.0 * c.D * pr
-        by = (oq.numel() * 2 + ok_.numel() * 2) * 2 + ol.numel() * 4
-        others[name] = {"ms": m, "tflops": fl / m / 1e9, "gbs": by / m / 1e6,
-                        "frac_tensor": fl / m / 1e9 / peaks["bf16_tflops"],
-                        "frac_hbm": by / m / 1e6 / peaks["hbm_gbs"]}
-        del oq, ok_, ov, oo, ol
+    others = run_others(args, swa, inputs, dev, stream, flush, peaks)
     assert swa.swa_device_error(stream) == 0
 
     if rank == 0:
@@ -601,7 +614,8 @@ def main():
     ap.add_argument("--clock-log", default=None,
                     help="also write the clock samples of the timed region to this CSV file")
     ap.add_argument("--only", default="all",
-                    choices=["all", "forward", "decode", "paged", "append", "backward"],
+                    choices=["all", "forward", "decode", "paged", "append", "backward",
+                             "others"],
                     help="run one workload alone (profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
