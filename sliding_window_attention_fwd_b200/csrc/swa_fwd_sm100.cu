@@ -640,15 +640,12 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
                 int Hkv, int N, int L, int R, int d, int bs, const int32_t* G, int ng,
                 float scale, cudaStream_t stream, const QueryWindow* qw) {
   using C = Cfg<D, NSLOT, NSTREAM>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess ||
-        cudaFuncSetAttribute(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, true>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess)
-      return SWA_ERR_CUDA;
-    attr_set = true;
-  }
+  static std::atomic<unsigned long long> attr_plain{0}, attr_qwin{0};
+  if (!smem_attr_once(reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, false>),
+                      C::kAlloc, attr_plain) ||
+      !smem_attr_once(reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, true>),
+                      C::kAlloc, attr_qwin))
+    return SWA_ERR_CUDA;
   int* err = device_error_word();
   if (!err) return SWA_ERR_CUDA;
   const Geometry geo = make_geometry(N, L, R, d, bs);

@@ -4,11 +4,28 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "swa.h"
 
 namespace swa {
+
+// Raises a kernel's dynamic shared memory limit to `bytes` on the current
+// device.  The attribute belongs to the kernel's instance on each device,
+// so it is set once per device (devices 0-63 are remembered in `done`;
+// higher ordinals set it on every call).  False on a CUDA error.
+inline bool smem_attr_once(const void* kernel, int bytes, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  const unsigned long long bit = dev >= 0 && dev < 64 ? 1ull << dev : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  if (bit) done.fetch_or(bit, std::memory_order_acq_rel);
+  return true;
+}
 
 // Device error word of the current device (bounded waits write into it).
 int* device_error_word();

@@ -608,13 +608,10 @@ bool get_workspace(int which, size_t cnt_bytes, size_t part_bytes, cudaStream_t 
 template <int D, int NQ, int MODE>
 int launch_rows(RowParams& p, int nsets, cudaStream_t stream) {
   using S = RSmem<D, NQ>;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(swa_rowattn_kernel<D, NQ, MODE>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, S::kAlloc) != cudaSuccess)
-      return SWA_ERR_CUDA;
-    attr = true;
-  }
+  static std::atomic<unsigned long long> attr{0};
+  if (!smem_attr_once(reinterpret_cast<const void*>(swa_rowattn_kernel<D, NQ, MODE>), S::kAlloc,
+                      attr))
+    return SWA_ERR_CUDA;
   dim3 grid(p.nsplit, nsets);
   swa_rowattn_kernel<D, NQ, MODE><<<grid, kThreadsR, S::kAlloc, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
