@@ -16,6 +16,11 @@
  * use the same one must not run on the device at the same time, whichever
  * streams they are on.  Workspaces grow on demand (the growing call
  * synchronises its stream first) and are freed by swa_release().
+ * Every call runs on the calling thread's current CUDA device, and the
+ * stream must belong to that device.  What the library keeps (workspaces,
+ * the device error word, kernel shared-memory limits) is kept per device
+ * (ordinals 0-63), so one process may drive several GPUs, one current
+ * device at a time.
  *
  * Definitions (page title, section):
  *  - Window and output: "滑动窗口注意力" (bmjup.com/post/11897), section
