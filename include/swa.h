@@ -98,6 +98,8 @@ typedef enum {
  * 0 = causal).  dilation >= 1.  global_idx: device int32 array of n_global
  * entries (NULL iff n_global == 0).  scale <= 0 selects 1/sqrt(D) (the
  * "softmax_scale None" default on page "别再只加Mask了", §3).
+ * With global tokens the GQA group H / Hkv must be <= 8 (else
+ * SWA_ERR_UNSUPPORTED).
  * B == 0 or N == 0 is a no-op returning SWA_OK.  Without global tokens the
  * call allocates no device memory; with them, the global query rows use the
  * library-owned split workspace of the row kernel (allocated on the first

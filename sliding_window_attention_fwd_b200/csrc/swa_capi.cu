@@ -132,6 +132,9 @@ int check_forward_bf16(const void* q, const void* k, const void* v, void* out, f
   if (st != SWA_OK) return st;
   if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
   if (dilation_block > 1 && dilation_block != kBlockRows) return SWA_ERR_UNSUPPORTED;
+  // the global query rows run on the row kernel, which serves up to 8
+  // query heads per kv head
+  if (n_global > 0 && H / Hkv > 8) return SWA_ERR_UNSUPPORTED;
   return SWA_OK;
 }
 }  // namespace
