@@ -596,6 +596,10 @@ def run_reference(args, rank, world):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cfg.name, "B": cfg.B, "N": cfg.N, "H": cfg.H, "Hkv": cfg.Hkv,
                        "D": cfg.D, "window": "causal, j in [i-4095, i]",
+                       "in_window_pairs": int(cnt.sum()) * cfg.B * cfg.H,
+                       "flops_per_step": 4.0 * cfg.D * int(cnt.sum()) * cfg.B * cfg.H,
+                       "l2": "host run: no device cache to flush",
+                       "parallelism": "rank 0 alone, on the host cores",
                        "sample_rows_per_step": n},
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                              "sample": f"{n} random query rows per step, fp64"},
