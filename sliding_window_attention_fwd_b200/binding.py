@@ -94,13 +94,28 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
-def _need(t, name, dtype, ndim):
+def _need(t, name, dtype, ndim, shape=None):
+    """Checks dtype, rank and (if given) the exact shape.  The library
+    receives bare pointers, so a buffer of the wrong size must be caught
+    here."""
     if t.dtype != dtype:
         raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
     if t.dim() != ndim:
         raise ValueError(f"{name}: expected {ndim} dims, got shape {tuple(t.shape)}")
-    if not t.is_cuda or not t.is_contiguous():
-        raise ValueError(f"{name}: must be a contiguous CUDA tensor")
+    if shape is not None and tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _placed(ref, **tensors):
+    """Every given tensor (None skipped) must be a contiguous CUDA tensor on
+    ref's device, where the call then runs."""
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name}: must be a contiguous CUDA tensor")
+        if t.device != ref.device:
+            raise ValueError(f"{name}: on {t.device}, expected {ref.device} like the queries")
 
 
 def _fwd_common(q, k, v, out, lse, global_idx, dtype):
@@ -113,15 +128,16 @@ def _fwd_common(q, k, v, out, lse, global_idx, dtype):
         raise ValueError("k and v must be [B, N, Hkv, D] matching q [B, N, H, D]")
     if out is None:
         out = torch.empty_like(q)
-    _need(out, "out", dtype, 4)
+    _need(out, "out", dtype, 4, (B, N, H, D))
     if lse is not None:
-        _need(lse, "lse", torch.float32, 3)
+        _need(lse, "lse", torch.float32, 3, (B, H, N))
     ng = 0
     if global_idx is not None and global_idx.numel() > 0:
         _need(global_idx, "global_idx", torch.int32, 1)
         ng = global_idx.numel()
     else:
         global_idx = None
+    _placed(q, q=q, k=k, v=v, out=out, lse=lse, global_idx=global_idx)
     return B, N, H, Hkv, D, out, global_idx, ng
 
 
@@ -129,9 +145,10 @@ def swa_forward(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dilation
                 global_idx=None, scale=0.0, stream=None):
     """bf16 SWA forward (C: swa_forward).  Returns out."""
     B, N, H, Hkv, D, out, gi, ng = _fwd_common(q, k, v, out, lse, global_idx, torch.bfloat16)
-    _check(_lib.swa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N, D,
-                            int(win_left), int(win_right), int(dilation), _ptr(gi), ng,
-                            float(scale), _stream(stream)), "swa_forward")
+    with torch.cuda.device(q.device):
+        _check(_lib.swa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N, D,
+                                int(win_left), int(win_right), int(dilation), _ptr(gi), ng,
+                                float(scale), _stream(stream)), "swa_forward")
     return out
 
 
@@ -139,9 +156,11 @@ def swa_forward_ex(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dilat
                    dilation_block=0, global_idx=None, scale=0.0, stream=None):
     """bf16 SWA forward with block-level dilation (C: swa_forward_ex)."""
     B, N, H, Hkv, D, out, gi, ng = _fwd_common(q, k, v, out, lse, global_idx, torch.bfloat16)
-    _check(_lib.swa_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N, D,
-                               int(win_left), int(win_right), int(dilation), int(dilation_block),
-                               _ptr(gi), ng, float(scale), _stream(stream)), "swa_forward_ex")
+    with torch.cuda.device(q.device):
+        _check(_lib.swa_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N,
+                                   D, int(win_left), int(win_right), int(dilation),
+                                   int(dilation_block), _ptr(gi), ng, float(scale),
+                                   _stream(stream)), "swa_forward_ex")
     return out
 
 
@@ -161,8 +180,11 @@ def swa_forward_layers(layers, stream=None):
                                                     torch.bfloat16)
         if shape is None:
             shape = (B, N, H, Hkv, D)
+            dev0 = L["q"].device
         elif shape != (B, N, H, Hkv, D):
             raise ValueError(f"layer {i}: shapes differ from layer 0")
+        elif L["q"].device != dev0:
+            raise ValueError(f"layer {i}: on {L['q'].device}, layer 0 on {dev0}")
         outs.append(out)
         keep.append(gi)
         arr[i] = SwaLayer(L["q"].data_ptr(), L["k"].data_ptr(), L["v"].data_ptr(), out.data_ptr(),
@@ -172,8 +194,9 @@ def swa_forward_layers(layers, stream=None):
                           None if gi is None else gi.data_ptr(), ng, float(L.get("scale", 0.0)))
     B, N, H, Hkv, D = shape
     bad = ctypes.c_int(-1)
-    st = _lib.swa_forward_layers(ctypes.cast(arr, _P), len(layers), B, H, Hkv, N, D,
-                                 ctypes.byref(bad), _stream(stream))
+    with torch.cuda.device(dev0):
+        st = _lib.swa_forward_layers(ctypes.cast(arr, _P), len(layers), B, H, Hkv, N, D,
+                                     ctypes.byref(bad), _stream(stream))
     _check(st, f"swa_forward_layers (layer {bad.value})")
     return outs
 
@@ -183,19 +206,21 @@ def swa_backward(q, k, v, out, dout, lse, win_left=-1, win_right=-1, dilation=1,
                  stream=None):
     """Gradients (dq, dk, dv) of swa_forward_ex (C: swa_backward); out and lse
     are the forward's outputs for the same arguments."""
-    B, N, H, Hkv, D, out, gi, ng = _fwd_common(q, k, v, out, lse, global_idx, torch.bfloat16)
-    _need(dout, "dout", torch.bfloat16, 4)
-    if lse is None:
-        raise ValueError("lse (from the forward) is required")
+    if out is None or lse is None:
+        raise ValueError("out and lse (from the forward) are required")
+    _need(dout, "dout", torch.bfloat16, 4, q.shape)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
-        _need(t, n, torch.bfloat16, 4)
-    _check(_lib.swa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
-                             _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, D, int(win_left),
-                             int(win_right), int(dilation), int(dilation_block), _ptr(gi), ng,
-                             float(scale), _stream(stream)), "swa_backward")
+    for t, n, ref in ((dq, "dq", q), (dk, "dk", k), (dv, "dv", v)):
+        _need(t, n, torch.bfloat16, 4, ref.shape)
+    B, N, H, Hkv, D, out, gi, ng = _fwd_common(q, k, v, out, lse, global_idx, torch.bfloat16)
+    _placed(q, dout=dout, dq=dq, dk=dk, dv=dv)
+    with torch.cuda.device(q.device):
+        _check(_lib.swa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                                 _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, N, D, int(win_left),
+                                 int(win_right), int(dilation), int(dilation_block), _ptr(gi),
+                                 ng, float(scale), _stream(stream)), "swa_backward")
     return dq, dk, dv
 
 
@@ -203,10 +228,11 @@ def swa_forward_f32(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dila
                     dilation_block=0, global_idx=None, scale=0.0, stream=None):
     """fp32 SWA forward on CUDA cores (C: swa_forward_f32)."""
     B, N, H, Hkv, D, out, gi, ng = _fwd_common(q, k, v, out, lse, global_idx, torch.float32)
-    _check(_lib.swa_forward_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N,
-                                D, int(win_left), int(win_right), int(dilation),
-                                int(dilation_block), _ptr(gi), ng, float(scale),
-                                _stream(stream)), "swa_forward_f32")
+    with torch.cuda.device(q.device):
+        _check(_lib.swa_forward_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv,
+                                    N, D, int(win_left), int(win_right), int(dilation),
+                                    int(dilation_block), _ptr(gi), ng, float(scale),
+                                    _stream(stream)), "swa_forward_f32")
     return out
 
 
@@ -221,15 +247,17 @@ def _dec_common(q, k_ring, v_ring, out, pos):
         raise ValueError("k_ring/v_ring must be [B, W, Hkv, D] and pos [B]")
     if out is None:
         out = torch.empty_like(q)
-    _need(out, "out", torch.bfloat16, 3)
+    _need(out, "out", torch.bfloat16, 3, (B, H, D))
     return B, H, Hkv, D, W, out
 
 
 def swa_decode(q, k_ring, v_ring, pos, out=None, stream=None):
     """Ring-buffer decode (C: swa_decode).  Returns out [B, H, D]."""
     B, H, Hkv, D, W, out = _dec_common(q, k_ring, v_ring, out, pos)
-    _check(_lib.swa_decode(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(out), _ptr(pos), B, H, Hkv,
-                           D, W, _stream(stream)), "swa_decode")
+    _placed(q, q=q, k_ring=k_ring, v_ring=v_ring, pos=pos, out=out)
+    with torch.cuda.device(q.device):
+        _check(_lib.swa_decode(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(out), _ptr(pos), B, H,
+                               Hkv, D, W, _stream(stream)), "swa_decode")
     return out
 
 
@@ -237,10 +265,12 @@ def swa_decode_ex(q, k_ring, v_ring, pos, out=None, lse=None, scale=0.0, stream=
     """Ring-buffer decode that also writes lse [B, H] (C: swa_decode_ex)."""
     B, H, Hkv, D, W, out = _dec_common(q, k_ring, v_ring, out, pos)
     if lse is not None:
-        _need(lse, "lse", torch.float32, 2)
-    _check(_lib.swa_decode_ex(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(out), _ptr(lse),
-                              _ptr(pos), B, H, Hkv, D, W, float(scale), _stream(stream)),
-           "swa_decode_ex")
+        _need(lse, "lse", torch.float32, 2, (B, H))
+    _placed(q, q=q, k_ring=k_ring, v_ring=v_ring, pos=pos, out=out, lse=lse)
+    with torch.cuda.device(q.device):
+        _check(_lib.swa_decode_ex(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(out), _ptr(lse),
+                                  _ptr(pos), B, H, Hkv, D, W, float(scale), _stream(stream)),
+               "swa_decode_ex")
     return out
 
 
@@ -251,9 +281,14 @@ def swa_decode_noalloc(q, k_ring, v_ring, pos, out, stream=None):
     fixed array inside the library, shared by all calls on a device, so calls
     must not overlap on the GPU.  `out` must be given (nothing is allocated
     here either)."""
+    if out is None:
+        raise ValueError("out is required (nothing is allocated here)")
     B, H, Hkv, D, W, out = _dec_common(q, k_ring, v_ring, out, pos)
-    _check(_lib.swa_decode_noalloc(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(out), _ptr(pos),
-                                   B, H, Hkv, D, W, _stream(stream)), "swa_decode_noalloc")
+    _placed(q, q=q, k_ring=k_ring, v_ring=v_ring, pos=pos, out=out)
+    with torch.cuda.device(q.device):
+        _check(_lib.swa_decode_noalloc(_ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(out),
+                                       _ptr(pos), B, H, Hkv, D, W, _stream(stream)),
+               "swa_decode_noalloc")
     return out
 
 
@@ -280,13 +315,16 @@ def swa_decode_paged(q, k_pages, v_pages, block_table, pos, page_size, W, out=No
                          "pos [B]")
     if out is None:
         out = torch.empty_like(q)
-    _need(out, "out", torch.bfloat16, 3)
+    _need(out, "out", torch.bfloat16, 3, (B, H, D))
     if lse is not None:
-        _need(lse, "lse", torch.float32, 2)
-    _check(_lib.swa_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(out), _ptr(lse),
-                                 _ptr(block_table), _ptr(pos), B, H, Hkv, D, int(page_size),
-                                 rows // int(page_size), block_table.shape[1], int(W),
-                                 float(scale), _stream(stream)), "swa_decode_paged")
+        _need(lse, "lse", torch.float32, 2, (B, H))
+    _placed(q, q=q, k_pages=k_pages, v_pages=v_pages, block_table=block_table, pos=pos, out=out,
+            lse=lse)
+    with torch.cuda.device(q.device):
+        _check(_lib.swa_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(out), _ptr(lse),
+                                     _ptr(block_table), _ptr(pos), B, H, Hkv, D, int(page_size),
+                                     rows // int(page_size), block_table.shape[1], int(W),
+                                     float(scale), _stream(stream)), "swa_decode_paged")
     return out
 
 
@@ -318,12 +356,15 @@ def swa_append(q, k_new, v_new, k_ring, v_ring, pos0, out=None, lse=None, scale=
         raise ValueError("k_new/v_new [B, C, Hkv, D], k_ring/v_ring [B, W, Hkv, D], pos0 [B]")
     if out is None:
         out = torch.empty_like(q)
-    _need(out, "out", torch.bfloat16, 4)
+    _need(out, "out", torch.bfloat16, 4, (B, C, H, D))
     if lse is not None:
-        _need(lse, "lse", torch.float32, 3)
-    _check(_lib.swa_append(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ring), _ptr(v_ring),
-                           _ptr(out), _ptr(lse), _ptr(pos0), B, C, H, Hkv, D, W, float(scale),
-                           _stream(stream)), "swa_append")
+        _need(lse, "lse", torch.float32, 3, (B, H, C))
+    _placed(q, q=q, k_new=k_new, v_new=v_new, k_ring=k_ring, v_ring=v_ring, pos0=pos0, out=out,
+            lse=lse)
+    with torch.cuda.device(q.device):
+        _check(_lib.swa_append(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_ring), _ptr(v_ring),
+                               _ptr(out), _ptr(lse), _ptr(pos0), B, C, H, Hkv, D, W,
+                               float(scale), _stream(stream)), "swa_append")
     return out
 
 
