@@ -127,6 +127,38 @@ def test_bruteforce_mask(case):
     np.testing.assert_allclose(l1, l2, atol=1e-12, rtol=0)
 
 
+try:
+    from hypothesis import given, settings, strategies as st
+except ImportError:  # pragma: no cover - hypothesis is part of the test image
+    given = None
+
+
+if given is not None:
+    @settings(max_examples=80, deadline=None, derandomize=True)
+    @given(data=st.data())
+    def test_bruteforce_mask_random(data):
+        """The same brute-force pin over randomly drawn problems: any window
+        kind, dilation, block size, GQA group, global set and scale."""
+        N = data.draw(st.integers(1, 70), "N")
+        Hkv = data.draw(st.integers(1, 2), "Hkv")
+        H = Hkv * data.draw(st.sampled_from([1, 2, 3]), "group")
+        D = data.draw(st.sampled_from([4, 8]), "D")
+        L = data.draw(st.integers(-1, 24), "L")
+        R = data.draw(st.integers(-1, 24), "R")
+        d = data.draw(st.integers(1, 5), "d")
+        bs = data.draw(st.sampled_from([0, 2, 4, 8]), "bs")
+        G = sorted(set(data.draw(st.lists(st.integers(0, N - 1), max_size=4), "G")))
+        scale = data.draw(st.sampled_from([None, 0.37]), "scale")
+        seed = data.draw(st.integers(0, 10_000), "seed")
+        q = _rand((1, N, H, D), seed)
+        k = _rand((1, N, Hkv, D), seed + 1)
+        v = _rand((1, N, Hkv, D), seed + 2)
+        o1, l1 = oracle.forward(q, k, v, L, R, d, bs, G, scale, threads=2)
+        o2, l2 = _brute(q, k, v, L, R, d, bs, G, scale)
+        np.testing.assert_allclose(o1, o2, atol=1e-12, rtol=0)
+        np.testing.assert_allclose(l1, l2, atol=1e-12, rtol=0)
+
+
 def test_wide_window_is_full_attention():
     N, D = 29, 8
     q, k, v = _rand((1, N, 1, D), 4), _rand((1, N, 1, D), 5), _rand((1, N, 1, D), 6)
