@@ -184,3 +184,65 @@ def test_planted_mistake_fails_a_pin(tmp_path, name, monkeypatch):
         except AssertionError:
             failed = True
     assert failed, f"mutant {name} passed every pin"
+
+
+try:
+    from hypothesis import given, settings, strategies as st
+except ImportError:  # pragma: no cover - hypothesis is part of the test image
+    given = None
+
+
+if given is not None:
+    @settings(max_examples=40, deadline=None, derandomize=True)
+    @given(data=st.data())
+    def test_paged_equals_forward_random(data):
+        """Paged decode = the forward oracle's causal window, over random
+        windows, page sizes, positions, GQA groups and page orders."""
+        B = data.draw(st.integers(1, 3), "B")
+        Hkv = data.draw(st.integers(1, 2), "Hkv")
+        H = Hkv * data.draw(st.sampled_from([1, 2, 4]), "group")
+        D = data.draw(st.sampled_from([8, 16]), "D")
+        N = data.draw(st.integers(1, 260), "N")
+        W = data.draw(st.integers(1, 300), "W")
+        ps = data.draw(st.sampled_from([8, 64, 96]), "page_size")
+        pos = np.array([data.draw(st.integers(0, N - 1), f"pos{b}") for b in range(B)])
+        rng = np.random.default_rng(data.draw(st.integers(0, 10_000), "seed"))
+        q, k, v = _seq(rng, B, N, H, Hkv, D)
+        first = np.maximum(0, pos - W + 1)
+        n_lp = (N + ps - 1) // ps
+        kp, vp, table = _pages_from_seq(rng, k, v, ps, n_lp, B * n_lp,
+                                        evict_before=(first // ps) * ps)
+        qd = np.stack([q[b, pos[b]] for b in range(B)])
+        o, l = oracle.decode_paged(qd, kp, vp, table, pos, ps, W)
+        rows = [(b, h, pos[b]) for b in range(B) for h in range(H)]
+        ro, rl = _forward_rows(q, k, v, W, rows)
+        assert np.isfinite(o).all()
+        np.testing.assert_allclose(o.reshape(B * H, D), ro, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l.reshape(B * H), rl, rtol=0, atol=1e-12)
+
+    @settings(max_examples=40, deadline=None, derandomize=True)
+    @given(data=st.data())
+    def test_append_equals_forward_random(data):
+        """Chunked append = the forward oracle on history + chunk, over random
+        windows, chunk lengths (also longer than the ring), start positions
+        (also inside the first window) and GQA groups."""
+        B = data.draw(st.integers(1, 2), "B")
+        Hkv = data.draw(st.integers(1, 2), "Hkv")
+        H = Hkv * data.draw(st.sampled_from([1, 3, 4]), "group")
+        D = data.draw(st.sampled_from([8, 16]), "D")
+        W = data.draw(st.integers(1, 96), "W")
+        C = data.draw(st.integers(1, 80), "C")
+        pos0 = np.array([data.draw(st.integers(0, 300), f"pos0_{b}") for b in range(B)])
+        rng = np.random.default_rng(data.draw(st.integers(0, 10_000), "seed"))
+        N = int(pos0.max()) + C
+        q, k, v = _seq(rng, B, N, H, Hkv, D)
+        kr, vr = _ring_from_seq(k, v, pos0, W)
+        qc = np.stack([q[b, pos0[b]:pos0[b] + C] for b in range(B)])
+        kn = np.stack([k[b, pos0[b]:pos0[b] + C] for b in range(B)])
+        vn = np.stack([v[b, pos0[b]:pos0[b] + C] for b in range(B)])
+        o, l = oracle.append(qc, kr, vr, kn, vn, pos0)
+        rows = [(b, h, pos0[b] + c) for b in range(B) for c in range(C) for h in range(H)]
+        ro, rl = _forward_rows(q, k, v, W, rows)
+        np.testing.assert_allclose(o.reshape(B * C * H, D), ro, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l.transpose(0, 2, 1).reshape(B * C * H), rl, rtol=0,
+                                   atol=1e-12)
