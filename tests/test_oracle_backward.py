@@ -9,7 +9,8 @@ the forward definition.  It is pinned by things other than itself:
     sum_j dV_j = sum over the group's query rows of dout (softmax rows sum to
     one, and the rows of dS sum to zero);
   * full attention (window wider than the sequence) equals torch autograd of
-    textbook softmax attention in fp64;
+    textbook softmax attention in fp64, and so does dense attention with the
+    key-set mask over randomly drawn windows;
 Planted mistakes in a copy of the C source each fail one of them.
 """
 import ctypes
@@ -94,6 +95,66 @@ def test_full_window_equals_autograd_softmax_attention():
     np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=0, atol=1e-12)
     np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=0, atol=1e-12)
     np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=0, atol=1e-12)
+
+
+def _allowed(N, L, R, d, bs, G):
+    """Pair-wise key-set predicate written from the definition (band, then
+    globals, then the causal cut), independent of the oracle's index lists."""
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    if bs > 1:
+        diff, lo, hi = j // bs - i // bs, -(L // bs) * d, (R // bs) * d
+    else:
+        diff, lo, hi = j - i, -L * d, R * d
+    ok = diff % d == 0
+    if L >= 0:
+        ok &= diff >= lo
+    if R >= 0:
+        ok &= diff <= hi
+    isg = np.zeros(N, dtype=bool)
+    isg[list(G)] = True
+    ok |= isg[None, :] | isg[:, None]
+    if R == 0:
+        ok &= j <= i
+    return ok
+
+
+try:
+    from hypothesis import given, settings, strategies as st
+except ImportError:  # pragma: no cover - hypothesis is part of the test image
+    given = None
+
+
+if given is not None:
+    @settings(max_examples=40, deadline=None, derandomize=True)
+    @given(data=st.data())
+    def test_masked_autograd_random(data):
+        """Over randomly drawn windows (band, causal, dilated, block-dilated,
+        global tokens, GQA) the oracle's gradients equal torch autograd of
+        dense fp64 attention with the key-set mask."""
+        N = data.draw(st.integers(1, 40), "N")
+        Hkv = data.draw(st.integers(1, 2), "Hkv")
+        H = Hkv * data.draw(st.sampled_from([1, 2, 3]), "group")
+        D = data.draw(st.sampled_from([4, 8]), "D")
+        L = data.draw(st.integers(-1, 12), "L")
+        R = data.draw(st.integers(-1, 12), "R")
+        d = data.draw(st.integers(1, 4), "d")
+        bs = data.draw(st.sampled_from([0, 2, 4]), "bs")
+        G = sorted(set(data.draw(st.lists(st.integers(0, N - 1), max_size=3), "G")))
+        rng = np.random.default_rng(data.draw(st.integers(0, 10_000), "seed"))
+        q, k, v, do = _rand(rng, 1, N, H, Hkv, D)
+        dq, dk, dv = oracle.backward(q, k, v, do, L, R, d, bs, G)
+        tq, tk, tv = (torch.tensor(a, dtype=torch.float64, requires_grad=True) for a in (q, k, v))
+        kk = tk.repeat_interleave(H // Hkv, dim=2)
+        vv = tv.repeat_interleave(H // Hkv, dim=2)
+        s = torch.einsum("bihd,bjhd->bhij", tq, kk) / np.sqrt(D)
+        mask = torch.tensor(_allowed(N, L, R, d, bs, G))
+        s = torch.where(mask, s, torch.tensor(float("-inf"), dtype=torch.float64))
+        out = torch.einsum("bhij,bjhd->bihd", torch.softmax(s, -1), vv)
+        (out * torch.tensor(do, dtype=torch.float64)).sum().backward()
+        np.testing.assert_allclose(dq, tq.grad.numpy(), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(dk, tk.grad.numpy(), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(dv, tv.grad.numpy(), rtol=0, atol=1e-11)
 
 
 MUTANTS = {
