@@ -1,7 +1,8 @@
 """The band-aware tile scheduler (host query swa_schedule) against the
 oracle's explicit key lists: the KV tiles of every query tile cover every
-key of every row, and exactly the tiles that are not wholly inside every
-row's window are flagged as edge tiles.  No GPU needed."""
+key of every row, the first and last of them hold a key (no tile is visited
+for nothing at either end), and exactly the tiles that are not wholly inside
+every row's window are flagged as edge tiles.  No GPU needed."""
 import numpy as np
 import pytest
 
@@ -44,6 +45,12 @@ CASES = [
 
 @pytest.mark.parametrize("case", CASES)
 def test_schedule_covers_window_and_flags_edges(case):
+    check_schedule(case, tight=True)
+
+
+def check_schedule(case, tight=False):
+    """Every key of every row lies in the listed tiles, the edge count is
+    exact, and (tight) the first and last listed tiles each hold a key."""
     N, L, R, d, bs = case
     recs = swa.swa_schedule(N, L, R, d, bs)
     cls = classes(N, d, bs)
@@ -63,6 +70,8 @@ def test_schedule_covers_window_and_flags_edges(case):
             needed.update(n // TILE for n in vk)
             full_rows[m] = set(vk)
         assert needed <= set(range(kb, ke)), (c, qt)
+        if tight:
+            assert (kb, ke - 1) == (min(needed), max(needed)), (c, qt)
         # a tile is full when all 128 rows and 128 keys exist and every row sees every key
         n_full = 0
         for t in range(kb, ke):
@@ -71,6 +80,20 @@ def test_schedule_covers_window_and_flags_edges(case):
                     keys <= full_rows[m] for m in ms):
                 n_full += 1
         assert n_edge == (ke - kb) - n_full, (c, qt)
+
+
+try:
+    from hypothesis import given, settings, strategies as st
+except ImportError:  # pragma: no cover - hypothesis is part of the test image
+    given = None
+
+
+if given is not None:
+    @settings(max_examples=30, deadline=None, derandomize=True)
+    @given(N=st.integers(1, 1200), L=st.integers(-1, 300), R=st.integers(-1, 300),
+           d=st.integers(1, 5), bs=st.sampled_from([0, 64]))
+    def test_schedule_random(N, L, R, d, bs):
+        check_schedule((N, L, R, d, bs), tight=True)
 
 
 def test_causal_mistral_tile_counts():
