@@ -488,6 +488,8 @@ def run_ours(args, rank, world, local_rank):
             "steps": args.steps,
             "warmup": args.warmup,
             "ms_per_step": step_ms,
+            "ms_median": statistics.median(ms),  # this rank's timed steps
+            "ms_min": min(ms),
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
