@@ -58,6 +58,28 @@ def test_bidirectional_truncated_window():
         assert list(ks) == list(range(first, last + 1))
 
 
+def test_receptive_fields_the_pages_print():
+    """Span of the key set after stacking layers: each layer's keys come from
+    the oracle's key sets, composed layer by layer (for the causal stacks the
+    reach of a contiguous band only depends on its first key)."""
+    for W, d, layers, span, tol in _rows(os.path.join(GOLDEN, "receptive_field.txt")):
+        if layers == 1:
+            w = (W - 1) // 2
+            ks = oracle.key_set(1000, 4000, w, w, dilation=d)
+            assert len(ks) == W and ks.max() - ks.min() + 1 == span
+            continue
+        N = layers * W + 10
+        i = N - 1
+        first = i
+        for _ in range(layers):
+            ks = oracle.key_set(first, N, W - 1, 0, dilation=d)
+            assert list(ks) == list(range(ks.min(), first + 1))  # contiguous, causal
+            first = int(ks.min())
+        reach = i - first + 1
+        assert reach == layers * (W - 1) + 1
+        assert abs(reach - span) <= tol
+
+
 # ------------------------------------------------------- brute force with mask
 def _brute(q, k, v, L, R, d=1, bs=0, G=(), scale=None):
     """Dense scores, then a band mask built pair by pair, then softmax."""
