@@ -297,7 +297,10 @@ SWA_API int swa_paged_window(int64_t pos, int W, int page_size, int64_t* first_p
  * taking positions >= pos0 from the chunk and the others from the ring as
  * it was before the call.  W must be a positive multiple of 64; 1 <= C <=
  * 65535; D in {64, 128}; H % Hkv == 0, H / Hkv <= 8; scale <= 0 means
- * 1/sqrt(D).  Two launches on `stream` (attention, then the ring update).
+ * 1/sqrt(D).  Launches on `stream`: for C >= 32 a staging copy (the
+ * window's history, de-rotated, followed by the chunk, into a library
+ * workspace), the tensor-core attention over it and the ring update; for
+ * shorter chunks the row-kernel attention and the ring update.
  * Workspace, streams and graphs as for swa_decode.
  */
 SWA_API int swa_append(const void* q, const void* k_new, const void* v_new, void* k_ring,
@@ -323,7 +326,7 @@ SWA_API int swa_selftest_timeout(int limit_us, void* stream);
 /*
  * swa_schedule -- host-only query of the band-aware tile scheduler (no GPU
  * needed).  For the forward problem (N, win_left, win_right, dilation,
- * dilation_block, n_global), writes one record of 6 int32 per query tile:
+ * dilation_block), writes one record of 6 int32 per query tile:
  *   { residue_class, q_tile, first_row, kv_tile_begin, kv_tile_end, n_edge }
  * where the 128-row query tile covers virtual rows [first_row,
  * first_row+128) of its residue class, it visits kv tiles [begin, end) of
