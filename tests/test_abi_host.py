@@ -29,6 +29,31 @@ def test_exports_every_declared_symbol():
         assert hasattr(lib, n), n
 
 
+def declared_parameter_counts():
+    """{name: number of parameters} of every SWA_API function in the header."""
+    text = open(HEADER).read()
+    out = {}
+    for m in re.finditer(r"SWA_API\s+[\w\s\*]+?\b(swa_\w+)\s*\(([^)]*)\)", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argtypes_match_the_header():
+    """Each ctypes prototype of the binding has as many arguments as the
+    header declares (a missing or extra one would shift every later
+    argument)."""
+    counts = declared_parameter_counts()
+    checked = 0
+    for name, n in counts.items():
+        fn = getattr(binding._lib, name)
+        if fn.argtypes is None:
+            continue
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+        checked += 1
+    assert checked >= 15
+
+
 def test_status_strings_and_version():
     assert swa.swa_status_string(0) == "ok"
     assert "aligned" in swa.swa_status_string(ALIGN)
