@@ -113,22 +113,54 @@ SWA_API int swa_forward(const void* q, const void* k, const void* v, void* out,
                         const int32_t* global_idx, int n_global, float scale,
                         void* stream);
 
+/* Element type of q, k, v and out in swa_params.dtype. */
+typedef enum {
+  SWA_DTYPE_BF16 = 0, /* bf16 tensors: the fused tcgen05 kernel (D 64 or 128) */
+  SWA_DTYPE_F32 = 1   /* fp32 tensors: the FFMA path of swa_forward_f32     */
+} swa_dtype;
+
 /*
- * swa_forward_ex -- swa_forward with block-level dilation.
- * dilation_block <= 1 is token-level dilation (identical to swa_forward);
- * dilation_block = Bs > 1 applies the dilation to whole Bs-token blocks
- * ("空洞滑窗机制" §四).  The fused kernel supports Bs = 64 (its tile is two
- * 64-row blocks); other Bs > 1 return SWA_ERR_UNSUPPORTED.
+ * Every argument of one forward call.  Each field means what the argument
+ * of the same name means for swa_forward; two more:
+ *   dilation_block  <= 1: token-level dilation (as swa_forward); Bs > 1:
+ *                   the dilation applies to whole Bs-token blocks
+ *                   ("空洞滑窗机制" §四), dense inside each block.  The bf16
+ *                   kernel supports Bs = 64 (its tile is two 64-row blocks;
+ *                   other Bs > 1 return SWA_ERR_UNSUPPORTED); the fp32 path
+ *                   any Bs.
+ *   dtype           a swa_dtype value: the element type of q, k, v, out.
+ * The struct is read during the call only.
  */
-SWA_API int swa_forward_ex(const void* q, const void* k, const void* v, void* out,
-                           float* lse, int B, int H, int Hkv, int N, int D,
-                           int win_left, int win_right, int dilation,
-                           int dilation_block, const int32_t* global_idx,
-                           int n_global, float scale, void* stream);
+typedef struct swa_params {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* out;
+  float* lse;
+  int B, H, Hkv, N, D;
+  int win_left;
+  int win_right;
+  int dilation;
+  int dilation_block;
+  const int32_t* global_idx;
+  int n_global;
+  float scale;
+  int dtype;
+} swa_params;
+
+/*
+ * swa_forward_ex -- the forward over a parameter block: swa_forward plus
+ * block-level dilation and a dtype selector (swa_forward is this call with
+ * dilation_block = 0 and dtype = SWA_DTYPE_BF16; swa_forward_f32 with
+ * dtype = SWA_DTYPE_F32).  p == NULL or an unknown dtype is SWA_ERR_ARG.
+ * Everything else (validation, errors, allocation) as for swa_forward or
+ * swa_forward_f32.
+ */
+SWA_API int swa_forward_ex(const swa_params* p, void* stream);
 
 /*
  * One layer of a per-layer window schedule (see swa_forward_layers).  Every
- * field means what the argument of the same name means for swa_forward_ex.
+ * field means what the field of the same name means in swa_params (bf16).
  */
 typedef struct swa_layer {
   const void* q;
@@ -230,9 +262,12 @@ SWA_API int swa_decode_ex(const void* q, const void* k_ring, const void* v_ring,
  * outputs.
  *
  * Limits and behaviour:
- *  - a problem whose split partials need more than the array holds (about
- *    B * Hkv * ceil(W / 512) * pow2(H/Hkv) * (D + 2) * 4 bytes) returns
- *    SWA_ERR_UNSUPPORTED and launches nothing;
+ *  - the array holds the split counters and the split partials: with
+ *    S = B * Hkv query sets, nsplit = ceil(W / 1024) key chunks per set and
+ *    nq = H/Hkv rounded up to a power of two, a problem with nsplit > 1
+ *    needs round_up(S * 4, 256) + S * nsplit * nq * (D + 2) * 4 bytes; one
+ *    that needs more than swa_decode_noalloc_scratch_bytes() returns
+ *    SWA_ERR_UNSUPPORTED and launches nothing (W <= 1024 needs none);
  *  - the first call on a device looks up the array's device address (once
  *    per device, with that device current); make that first call before
  *    any stream capture;

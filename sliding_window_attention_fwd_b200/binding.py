@@ -21,9 +21,9 @@ _I = ctypes.c_int
 _F = ctypes.c_float
 
 _lib.swa_forward.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _F, _P]
-_lib.swa_forward_ex.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I,
-                                _F, _P]
-_lib.swa_forward_f32.argtypes = _lib.swa_forward_ex.argtypes
+_lib.swa_forward_ex.argtypes = [_P, _P]
+_lib.swa_forward_f32.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I,
+                                 _F, _P]
 _lib.swa_decode.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
 _lib.swa_decode_ex.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]
 _lib.swa_decode_noalloc.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
@@ -34,6 +34,18 @@ _lib.swa_decode_paged.argtypes = [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I
                                   _F, _P]
 _lib.swa_paged_window.argtypes = [ctypes.c_int64, _I, _I, _P, _P]
 _lib.swa_append.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]
+
+
+SWA_DTYPE_BF16 = 0
+SWA_DTYPE_F32 = 1
+
+
+class SwaParams(ctypes.Structure):
+    """struct swa_params of include/swa.h."""
+    _fields_ = [("q", _P), ("k", _P), ("v", _P), ("out", _P), ("lse", _P),
+                ("B", _I), ("H", _I), ("Hkv", _I), ("N", _I), ("D", _I),
+                ("win_left", _I), ("win_right", _I), ("dilation", _I), ("dilation_block", _I),
+                ("global_idx", _P), ("n_global", _I), ("scale", _F), ("dtype", _I)]
 
 
 class SwaLayer(ctypes.Structure):
@@ -154,13 +166,19 @@ def swa_forward(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dilation
 
 def swa_forward_ex(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dilation=1,
                    dilation_block=0, global_idx=None, scale=0.0, stream=None):
-    """bf16 SWA forward with block-level dilation (C: swa_forward_ex)."""
-    B, N, H, Hkv, D, out, gi, ng = _fwd_common(q, k, v, out, lse, global_idx, torch.bfloat16)
+    """SWA forward with block-level dilation over a parameter block (C:
+    swa_forward_ex).  bf16 tensors take the tcgen05 kernel, fp32 tensors the
+    FFMA path (the block's dtype follows q)."""
+    dt = torch.float32 if q.dtype == torch.float32 else torch.bfloat16
+    B, N, H, Hkv, D, out, gi, ng = _fwd_common(q, k, v, out, lse, global_idx, dt)
+    prm = SwaParams(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                    None if lse is None else lse.data_ptr(), B, H, Hkv, N, D, int(win_left),
+                    int(win_right), int(dilation), int(dilation_block),
+                    None if gi is None else gi.data_ptr(), ng, float(scale),
+                    SWA_DTYPE_F32 if dt == torch.float32 else SWA_DTYPE_BF16)
     with torch.cuda.device(q.device):
-        _check(_lib.swa_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N,
-                                   D, int(win_left), int(win_right), int(dilation),
-                                   int(dilation_block), _ptr(gi), ng, float(scale),
-                                   _stream(stream)), "swa_forward_ex")
+        _check(_lib.swa_forward_ex(ctypes.c_void_p(ctypes.addressof(prm)), _stream(stream)),
+               "swa_forward_ex")
     return out
 
 

@@ -139,31 +139,80 @@ int check_forward_bf16(const void* q, const void* k, const void* v, void* out, f
 }
 }  // namespace
 
-SWA_API int swa_forward_ex(const void* q, const void* k, const void* v, void* out, float* lse,
-                           int B, int H, int Hkv, int N, int D, int win_left, int win_right,
-                           int dilation, int dilation_block, const int32_t* global_idx,
-                           int n_global, float scale, void* stream) {
-  int st = check_forward_bf16(q, k, v, out, lse, B, H, Hkv, N, D, dilation, dilation_block,
-                              global_idx, n_global);
+namespace {
+// The bf16 forward of one parameter block, validated by the caller.
+int forward_bf16(const swa_params& p, cudaStream_t s) {
+  if (p.B == 0 || p.N == 0) return SWA_OK;
+  const float sc = resolve_scale(p.scale, p.D);
+  int st = launch_fwd_sm100(p.q, p.k, p.v, p.out, p.lse, p.B, p.H, p.Hkv, p.N, p.D, p.win_left,
+                            p.win_right, p.dilation, p.dilation_block, p.global_idx, p.n_global,
+                            sc, s);
   if (st != SWA_OK) return st;
-  if (B == 0 || N == 0) return SWA_OK;
-  const float sc = resolve_scale(scale, D);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  st = launch_fwd_sm100(q, k, v, out, lse, B, H, Hkv, N, D, win_left, win_right, dilation,
-                        dilation_block, global_idx, n_global, sc, s);
-  if (st != SWA_OK) return st;
-  if (n_global > 0)
-    st = launch_global_rows(q, k, v, out, lse, B, H, Hkv, N, D, win_right == 0, global_idx,
-                            n_global, sc, s);
+  if (p.n_global > 0)
+    st = launch_global_rows(p.q, p.k, p.v, p.out, p.lse, p.B, p.H, p.Hkv, p.N, p.D,
+                            p.win_right == 0, p.global_idx, p.n_global, sc, s);
   return st;
+}
+
+int forward_f32(const swa_params& p, cudaStream_t s) {
+  int st = check_forward_args(p.q, p.k, p.v, p.out, p.lse, p.B, p.H, p.Hkv, p.N, p.D,
+                              p.dilation, p.dilation_block, p.global_idx, p.n_global);
+  if (st != SWA_OK) return st;
+  if (p.D != 32 && p.D != 64 && p.D != 96 && p.D != 128) return SWA_ERR_UNSUPPORTED;
+  if (p.B == 0 || p.N == 0) return SWA_OK;
+  return launch_fwd_f32(static_cast<const float*>(p.q), static_cast<const float*>(p.k),
+                        static_cast<const float*>(p.v), static_cast<float*>(p.out), p.lse, p.B,
+                        p.H, p.Hkv, p.N, p.D, p.win_left, p.win_right, p.dilation,
+                        p.dilation_block, p.global_idx, p.n_global,
+                        resolve_scale(p.scale, p.D), s);
+}
+
+swa_params make_params(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int H, int Hkv, int N, int D, int win_left, int win_right,
+                       int dilation, int dilation_block, const int32_t* global_idx,
+                       int n_global, float scale, int dtype) {
+  swa_params p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.out = out;
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.D = D;
+  p.win_left = win_left;
+  p.win_right = win_right;
+  p.dilation = dilation;
+  p.dilation_block = dilation_block;
+  p.global_idx = global_idx;
+  p.n_global = n_global;
+  p.scale = scale;
+  p.dtype = dtype;
+  return p;
+}
+}  // namespace
+
+SWA_API int swa_forward_ex(const swa_params* p, void* stream) {
+  if (!p) return SWA_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (p->dtype == SWA_DTYPE_F32) return forward_f32(*p, s);
+  if (p->dtype != SWA_DTYPE_BF16) return SWA_ERR_ARG;
+  const int st = check_forward_bf16(p->q, p->k, p->v, p->out, p->lse, p->B, p->H, p->Hkv, p->N,
+                                    p->D, p->dilation, p->dilation_block, p->global_idx,
+                                    p->n_global);
+  if (st != SWA_OK) return st;
+  return forward_bf16(*p, s);
 }
 
 SWA_API int swa_forward(const void* q, const void* k, const void* v, void* out, float* lse,
                         int B, int H, int Hkv, int N, int D, int win_left, int win_right,
                         int dilation, const int32_t* global_idx, int n_global, float scale,
                         void* stream) {
-  return swa_forward_ex(q, k, v, out, lse, B, H, Hkv, N, D, win_left, win_right, dilation, 0,
-                        global_idx, n_global, scale, stream);
+  const swa_params p = make_params(q, k, v, out, lse, B, H, Hkv, N, D, win_left, win_right,
+                                   dilation, 0, global_idx, n_global, scale, SWA_DTYPE_BF16);
+  return swa_forward_ex(&p, stream);
 }
 
 SWA_API int swa_forward_layers(const swa_layer* layers, int n_layers, int B, int H, int Hkv,
@@ -181,9 +230,10 @@ SWA_API int swa_forward_layers(const swa_layer* layers, int n_layers, int B, int
   }
   for (int i = 0; i < n_layers; ++i) {
     const swa_layer& L = layers[i];
-    const int st = swa_forward_ex(L.q, L.k, L.v, L.out, L.lse, B, H, Hkv, N, D, L.win_left,
-                                  L.win_right, L.dilation, L.dilation_block, L.global_idx,
-                                  L.n_global, L.scale, stream);
+    const swa_params p = make_params(L.q, L.k, L.v, L.out, L.lse, B, H, Hkv, N, D, L.win_left,
+                                     L.win_right, L.dilation, L.dilation_block, L.global_idx,
+                                     L.n_global, L.scale, SWA_DTYPE_BF16);
+    const int st = forward_bf16(p, static_cast<cudaStream_t>(stream));
     if (st != SWA_OK) {
       if (bad_layer) *bad_layer = i;
       return st;
@@ -216,14 +266,10 @@ SWA_API int swa_forward_f32(const float* q, const float* k, const float* v, floa
                             int win_right, int dilation, int dilation_block,
                             const int32_t* global_idx, int n_global, float scale,
                             void* stream) {
-  int st = check_forward_args(q, k, v, out, lse, B, H, Hkv, N, D, dilation, dilation_block,
-                              global_idx, n_global);
-  if (st != SWA_OK) return st;
-  if (D != 32 && D != 64 && D != 96 && D != 128) return SWA_ERR_UNSUPPORTED;
-  if (B == 0 || N == 0) return SWA_OK;
-  return launch_fwd_f32(q, k, v, out, lse, B, H, Hkv, N, D, win_left, win_right, dilation,
-                        dilation_block, global_idx, n_global, resolve_scale(scale, D),
-                        static_cast<cudaStream_t>(stream));
+  const swa_params p = make_params(q, k, v, out, lse, B, H, Hkv, N, D, win_left, win_right,
+                                   dilation, dilation_block, global_idx, n_global, scale,
+                                   SWA_DTYPE_F32);
+  return swa_forward_ex(&p, stream);
 }
 
 SWA_API int swa_decode_ex(const void* q, const void* k_ring, const void* v_ring, void* out,

@@ -37,6 +37,7 @@ namespace swa {
 namespace {
 
 constexpr int kRows = 64;           // key rows per stage
+constexpr int kDecodeChunk = 1024;  // ring-decode keys per CTA: amortises set-up and merge
 constexpr int kStagesR = 2;
 constexpr int kComputeWarps = 4;
 constexpr int kThreadsR = (kComputeWarps + 1) * 32;
@@ -752,7 +753,7 @@ int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* o
   p.grp = H / Hkv;
   p.rows_per_cta = 1;
   p.nrowchunks = 1;
-  p.chunk = 1024;  // keys per CTA: amortises the per-CTA set-up and merge
+  p.chunk = kDecodeChunk;
   p.nsplit = (W + p.chunk - 1) / p.chunk;
   p.scale_log2 = scale * 1.4426950408889634f;
   const int nq = pow2_at_least(p.grp);
@@ -993,7 +994,7 @@ int launch_decode_noalloc(const void* q, const void* k_ring, const void* v_ring,
   p.grp = H / Hkv;
   p.rows_per_cta = 1;
   p.nrowchunks = 1;
-  p.chunk = 512;
+  p.chunk = kDecodeChunk;  // the same split as swa_decode
   p.nsplit = (W + p.chunk - 1) / p.chunk;
   p.scale_log2 = scale * 1.4426950408889634f;
   const int nq = pow2_at_least(p.grp);

@@ -65,9 +65,14 @@ A = 0x10000  # fake, 16-byte aligned addresses: validation never dereferences th
 
 
 def fwd(*, q=A, k=A, v=A, out=A, lse=None, B=1, H=4, Hkv=2, N=64, D=128, L_=8, R=8, d=1,
-        bs=0, G=None, ng=0, scale=0.0, f32=False):
-    fn = L.swa_forward_f32 if f32 else L.swa_forward_ex
-    return fn(q, k, v, out, lse, B, H, Hkv, N, D, L_, R, d, bs, G, ng, scale, None)
+        bs=0, G=None, ng=0, scale=0.0, f32=False, dtype=None):
+    """swa_forward_ex over a parameter block (swa_forward_f32 for f32=True)."""
+    if f32:
+        return L.swa_forward_f32(q, k, v, out, lse, B, H, Hkv, N, D, L_, R, d, bs, G, ng, scale,
+                                 None)
+    prm = binding.SwaParams(q, k, v, out, lse, B, H, Hkv, N, D, L_, R, d, bs, G, ng, scale,
+                            binding.SWA_DTYPE_BF16 if dtype is None else dtype)
+    return L.swa_forward_ex(ctypes.c_void_p(ctypes.addressof(prm)), None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -93,6 +98,43 @@ def fwd(*, q=A, k=A, v=A, out=A, lse=None, B=1, H=4, Hkv=2, N=64, D=128, L_=8, R
 ])
 def test_forward_validation(kw, code):
     assert fwd(**kw) == code
+
+
+def test_forward_ex_parameter_block():
+    # the dtype field selects the path; NULL and unknown dtypes are rejected
+    assert L.swa_forward_ex(None, None) == ARG
+    assert fwd(dtype=7) == ARG
+    assert fwd(dtype=binding.SWA_DTYPE_F32, D=96, B=0) == OK   # fp32 path serves D=96
+    assert fwd(dtype=binding.SWA_DTYPE_BF16, D=96) == UNSUP    # the bf16 kernel does not
+    assert fwd(dtype=binding.SWA_DTYPE_F32, D=80) == UNSUP
+    assert fwd(dtype=binding.SWA_DTYPE_F32, bs=32, B=0) == OK  # any block size in fp32
+    # plain swa_forward (flat arguments) validates the same way
+    assert L.swa_forward(A, A, A, A, None, 1, 4, 3, 64, 128, 8, 8, 1, None, 0, 0.0, None) == ARG
+    assert L.swa_forward(A, A, A, A, None, 0, 4, 2, 64, 128, 8, 8, 1, None, 0, 0.0, None) == OK
+
+
+def test_params_struct_layout_matches_the_header():
+    """Field offsets of the ctypes mirror equal the C struct's (compiled
+    with gcc against include/swa.h)."""
+    import shutil
+    import subprocess
+    import tempfile
+    if shutil.which("gcc") is None:
+        pytest.skip("needs gcc")
+    fields = [f[0] for f in binding.SwaParams._fields_]
+    prog = "#include <stdio.h>\n#include <stddef.h>\n#include \"swa.h\"\nint main(void){\n"
+    prog += "".join(f'printf("%zu\\n", offsetof(swa_params, {f}));\n' for f in fields)
+    prog += 'printf("%zu\\n", sizeof(swa_params)); return 0; }\n'
+    with tempfile.TemporaryDirectory() as d:
+        src, exe = os.path.join(d, "o.c"), os.path.join(d, "o")
+        open(src, "w").write(prog)
+        subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), src, "-o", exe],
+                       check=True, capture_output=True)
+        got = [int(x) for x in subprocess.run([exe], check=True, capture_output=True,
+                                              text=True).stdout.split()]
+    want = [getattr(binding.SwaParams, f).offset for f in fields] + [
+        ctypes.sizeof(binding.SwaParams)]
+    assert got == want
 
 
 def test_f32_validation():

@@ -101,3 +101,34 @@ def test_append_buffers():
         b.swa_append(q, kn, vn, kr, vr, pos0, lse=t(B, C, H, dtype=F32))
     with pytest.raises(ValueError, match="expected shape"):
         b.swa_append(q, kn, vn, kr, vr, pos0, out=t(B, C, Hkv, D))
+
+
+def _maps_after(code):
+    """Runs `code` in a fresh interpreter and returns the shared objects it
+    has mapped afterwards (from /proc/self/maps)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    prog = (f"import sys; sys.path.insert(0, {root!r})\n{code}\n"
+            "print('\\n'.join(sorted({l.split()[-1] for l in open('/proc/self/maps') "
+            "if l.strip().endswith('.so')})))")
+    res = subprocess.run([sys.executable, "-c", prog], capture_output=True, text=True,
+                         timeout=300, env={**os.environ, "CUDA_VISIBLE_DEVICES": ""})
+    assert res.returncode == 0, res.stderr
+    return res.stdout.split()
+
+
+def test_package_import_maps_no_library():
+    # the seeded generator and the build module serve processes that never
+    # run the CUDA path (the oracle's timing arm, the build check)
+    maps = _maps_after("import sliding_window_attention_fwd_b200 as s\n"
+                       "from sliding_window_attention_fwd_b200 import inputs, build\n"
+                       "inputs.normal((2, 3), 1, 0)")
+    assert not any(m.endswith("libswa.so") for m in maps)
+
+
+def test_first_binding_use_loads_library():
+    maps = _maps_after("import sliding_window_attention_fwd_b200 as s\n"
+                       "assert s.swa_version() > 0")
+    assert any(m.endswith("sliding_window_attention_fwd_b200/libswa.so") for m in maps)

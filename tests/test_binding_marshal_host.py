@@ -53,10 +53,22 @@ def test_forward_ex(lib):
     q, k, v = z(2, 50, 8, 64), z(2, 50, 2, 64), z(2, 50, 2, 64)
     out, lse = z(2, 50, 8, 64), z(2, 8, 50, dtype=torch.float32)
     G = torch.tensor([0, 7], dtype=torch.int32)
+    seen = {}
+
+    def rec(pp, stream):  # read the parameter block while the call lasts
+        prm = ctypes.cast(pp, ctypes.POINTER(b.SwaParams))[0]
+        seen["p"] = [getattr(prm, f[0]) for f in b.SwaParams._fields_]
+        seen["stream"] = stream
+        return 0
+    lib.swa_forward_ex = rec
     b.swa_forward_ex(q, k, v, out, lse, 11, 3, 2, 64, G, 0.25)
-    got = unpack(lib.calls["swa_forward_ex"])
-    assert got == [q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                   2, 8, 2, 50, 64, 11, 3, 2, 64, G.data_ptr(), 2, 0.25, "STREAM"]
+    assert seen["p"] == [q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                         2, 8, 2, 50, 64, 11, 3, 2, 64, G.data_ptr(), 2, 0.25,
+                         b.SWA_DTYPE_BF16]
+    assert seen["stream"] == "STREAM"
+    qf, kf, vf = (t.float() for t in (q, k, v))
+    outf = b.swa_forward_ex(qf, kf, vf, None, None, 1, 1)
+    assert seen["p"][3] == outf.data_ptr() and seen["p"][-1] == b.SWA_DTYPE_F32
 
 
 def test_forward_plain_and_f32(lib):

@@ -28,6 +28,16 @@ int main(void) {
     printf("%%d %%d %%d %%d %%d %%d\n", tiles[0], tiles[1], tiles[2], tiles[3], tiles[4],
            tiles[5]);
   printf("%%s\n", swa_status_string(SWA_ERR_UNSUPPORTED));
+  /* the parameter-block forward, validated on the host: B = 0 is a no-op */
+  swa_params p = {0};
+  p.q = p.k = p.v = (const void*)tiles;
+  p.out = (void*)tiles;
+  p.H = 4; p.Hkv = 2; p.N = 64; p.D = 128; p.dilation = 1;
+  p.dtype = SWA_DTYPE_BF16;
+  int ok0 = swa_forward_ex(&p, NULL);
+  p.dtype = 9;
+  int bad_dtype = swa_forward_ex(&p, NULL);
+  printf("%%d %%d\n", ok0, bad_dtype);
   return 0;
 }
 """
@@ -59,3 +69,4 @@ def test_header_is_c99_and_links(tmp_path, case):
     assert (first, last) == (lo // case["ps"], case["pos"] // case["ps"])
     assert bad == -1  # SWA_ERR_ARG
     assert lines[2] == binding.swa_status_string(-3)
+    assert lines[3].split() == ["0", "-1"]  # SWA_OK, SWA_ERR_ARG
