@@ -132,9 +132,6 @@ int check_forward_bf16(const void* q, const void* k, const void* v, void* out, f
   if (st != SWA_OK) return st;
   if (D != 64 && D != 128) return SWA_ERR_UNSUPPORTED;
   if (dilation_block > 1 && dilation_block != kBlockRows) return SWA_ERR_UNSUPPORTED;
-  // the global query rows run on the row kernel, which serves up to 8
-  // query heads per kv head
-  if (n_global > 0 && H / Hkv > 8) return SWA_ERR_UNSUPPORTED;
   return SWA_OK;
 }
 }  // namespace
@@ -143,15 +140,10 @@ namespace {
 // The bf16 forward of one parameter block, validated by the caller.
 int forward_bf16(const swa_params& p, cudaStream_t s) {
   if (p.B == 0 || p.N == 0) return SWA_OK;
-  const float sc = resolve_scale(p.scale, p.D);
-  int st = launch_fwd_sm100(p.q, p.k, p.v, p.out, p.lse, p.B, p.H, p.Hkv, p.N, p.D, p.win_left,
-                            p.win_right, p.dilation, p.dilation_block, p.global_idx, p.n_global,
-                            sc, s);
-  if (st != SWA_OK) return st;
-  if (p.n_global > 0)
-    st = launch_global_rows(p.q, p.k, p.v, p.out, p.lse, p.B, p.H, p.Hkv, p.N, p.D,
-                            p.win_right == 0, p.global_idx, p.n_global, sc, s);
-  return st;
+  // one launch: band tiles, global-key tiles and the global query rows
+  return launch_fwd_sm100(p.q, p.k, p.v, p.out, p.lse, p.B, p.H, p.Hkv, p.N, p.D, p.win_left,
+                          p.win_right, p.dilation, p.dilation_block, p.global_idx, p.n_global,
+                          resolve_scale(p.scale, p.D), s);
 }
 
 int forward_f32(const swa_params& p, cudaStream_t s) {

@@ -60,9 +60,12 @@ struct FwdParams {
   CUtensorMap tmQ[kMaxClasses];
   CUtensorMap tmK[kMaxClasses];
   CUtensorMap tmV[kMaxClasses];
+  CUtensorMap tmKf;  // K and V over the whole sequence (rows in position order):
+  CUtensorMap tmVf;  // the keys of the global query rows
   uint16_t* out;
   float* lse;
   const int32_t* G;
+  const uint16_t* q_raw;
   const uint16_t* k_raw;
   const uint16_t* v_raw;
   int* err;
@@ -70,6 +73,11 @@ struct FwdParams {
   int B, H, Hkv, N;
   int L, R, d, bs;
   int class0, nclass;
+  // Global query rows: the first n_gitems CTAs of the grid each take up to
+  // 128 global rows (a "global tile") of one (batch, head pair), n_gq_tiles
+  // tiles per pair, and attend every key of the sequence (causal: up to the
+  // row).  The band CTAs leave those rows to them.
+  int n_gitems, n_gq_tiles;
   int qtile_prefix[kMaxClasses + 1];
   int Mv[kMaxClasses];
   float scale_log2;
@@ -104,9 +112,10 @@ struct Cfg {
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
-// QWIN: the query window of a chunked append (compile-time, so the plain
-// forward carries none of its row mapping).
-template <int D, int NSLOT, int NSTREAM, bool QWIN>
+// KIND (compile-time, so each form carries only its own code): 0 band (and
+// token/block dilation) only; 1 the query window of a chunked append; 2 the
+// band plus global tokens (global-key tiles and global query rows).
+template <int D, int NSLOT, int NSTREAM, int KIND>
 __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     swa_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
   using C = Cfg<D, NSLOT, NSTREAM>;
@@ -132,17 +141,26 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // ---- work item: (class, q tile, batch, head pair); heavy (late) tiles first
+  // ---- work item: the global tiles first (each walks the whole sequence),
+  // then (class, q tile, batch, head pair) with heavy (late) tiles first
   const int npair = (p.H + NSLOT - 1) / NSLOT;
   int x = blockIdx.x;
+  constexpr bool glob = KIND == 2;
+  const bool gitem = glob && x < p.n_gitems;
+  if (glob && !gitem) x -= p.n_gitems;
   const int hp = x % npair;
   x /= npair;
   const int b = x % p.B;
   x /= p.B;
-  const int jt = p.qtile_prefix[p.nclass] - 1 - x;
-  int cl = 0;
-  while (cl + 1 < p.nclass && p.qtile_prefix[cl + 1] <= jt) ++cl;
-  const int qt = jt - p.qtile_prefix[cl];
+  int cl = 0, qt = 0, gq0 = 0, gcnt = 0;
+  if (gitem) {
+    gq0 = x * kTileM;  // first global row of this tile
+    gcnt = min(kTileM, p.n_global - gq0);
+  } else {
+    const int jt = p.qtile_prefix[p.nclass] - 1 - x;
+    while (cl + 1 < p.nclass && p.qtile_prefix[cl + 1] <= jt) ++cl;
+    qt = jt - p.qtile_prefix[cl];
+  }
   const int c = p.class0 + cl;
   const int grp = p.H / p.Hkv;
   int head[NSLOT], kvh[NSLOT];
@@ -155,13 +173,23 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     kvh[s] = head[s] / grp;
   }
   const Geometry g = make_geometry(p.N, p.L, p.R, p.d, p.bs);
-  const int Mv = p.Mv[cl];
-  constexpr bool qwin = QWIN;
+  // a global tile's keys are the physical rows of the sequence
+  const int Mv = gitem ? p.N : p.Mv[cl];
+  constexpr bool qwin = KIND == 1;
   const int Mq = qwin ? p.Mq : Mv;  // query rows (local)
   const int q0 = qwin ? p.q0 : 0;   // virtual row of local query row 0
   const int qm0 = q0 + qt * kTileM;
   const int qm1 = q0 + min(qt * kTileM + kTileM - 1, Mq - 1);
-  const TileRange tr = tile_range_rows(g, Mv, qm0, qm1);
+  TileRange tr;
+  if (gitem) {
+    // every key tile (causal: up to the tile's last, i.e. largest, global row)
+    int last = __ldg(p.G + gq0 + gcnt - 1);
+    last = last < 0 ? 0 : (last >= p.N ? p.N - 1 : last);
+    tr.kv_begin = 0;
+    tr.kv_end = p.R == 0 ? last / kTileN + 1 : (p.N + kTileN - 1) / kTileN;
+  } else {
+    tr = tile_range_rows(g, Mv, qm0, qm1);
+  }
   int lo_b = 0;  // first key row holding a real position (query window only)
   if (qwin) {
     const long long pb = p.pos0[b];
@@ -169,7 +197,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     lo_b = lb <= 0 ? 0 : (lb > Mv ? Mv : (int)lb);
   }
   const int n_band = tr.kv_end - tr.kv_begin;
-  const int n_gtiles = (p.n_global + kTileN - 1) / kTileN;
+  const int n_gtiles = (!glob || gitem) ? 0 : (p.n_global + kTileN - 1) / kTileN;
   const int n_tiles = n_band + n_gtiles;
   const bool block_mode = p.bs > 1;
   const int map_idx = block_mode ? 0 : cl;
@@ -216,10 +244,38 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
   if (warp < 4) {
     if (warp == 0) {
       // =========================== producer ===========================
-      if (lane == 0) {
+      const CUtensorMap* mapK = gitem ? &p.tmKf : &p.tmK[map_idx];
+      const CUtensorMap* mapV = gitem ? &p.tmVf : &p.tmV[map_idx];
+      if (gitem) {
+        // gather the tile's global query rows (zeros past the last) with
+        // plain 16-byte loads into the swizzled layout of a TMA box
+        if (lane == 0) {
+          prefetch_tensormap(mapK);
+          prefetch_tensormap(mapV);
+        }
+        constexpr int kC16 = D / 8;  // 16-byte chunks per row
+        for (int s = 0; s < NSLOT; ++s) {
+          for (int idx = lane; idx < kTileM * kC16; idx += 32) {
+            const int row = idx / kC16, c16 = idx % kC16;
+            uint4 val = make_uint4(0u, 0u, 0u, 0u);
+            if (row < gcnt) {
+              int gv = __ldg(p.G + gq0 + row);
+              gv = gv < 0 ? 0 : (gv >= p.N ? p.N - 1 : gv);
+              val = __ldg(reinterpret_cast<const uint4*>(
+                  p.q_raw + (((size_t)b * p.N + gv) * p.H + head[s]) * D + c16 * 8));
+            }
+            uint8_t* d8 = smem + C::kQ + s * C::kTile + (c16 / 8) * kChunkBytes + row * 128 +
+                          (((c16 % 8) ^ (row % 8)) * 16);
+            *reinterpret_cast<uint4*>(d8) = val;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(full_q);
+      } else if (lane == 0) {
         prefetch_tensormap(&p.tmQ[map_idx]);
-        prefetch_tensormap(&p.tmK[map_idx]);
-        prefetch_tensormap(&p.tmV[map_idx]);
+        prefetch_tensormap(mapK);
+        prefetch_tensormap(mapV);
         mbar_arrive_expect_tx(full_q, C::kQBytes);
         for (int s = 0; s < NSLOT; ++s)
           for (int cc = 0; cc < D / 64; ++cc)
@@ -236,16 +292,18 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
           uint64_t* ful = kv ? &full_v[st] : &full_k[st];
           uint8_t* dst = smem + C::kRing + st * C::kStageBytes + kv * NSTREAM * C::kTile;
           if (it >= kStages && !mbar_wait(emp, ph ^ 1u, p.err, abort_flag)) goto producer_done;
-          if (it < n_band) {
+          if (!glob || it < n_band) {
             if (lane == 0) {
-              const CUtensorMap* m = kv ? &p.tmV[map_idx] : &p.tmK[map_idx];
+              const CUtensorMap* m = kv ? mapV : mapK;
               const int t = tr.kv_begin + it;
               mbar_arrive_expect_tx(ful, NSTREAM * C::kTile);
               for (int s = 0; s < NSTREAM; ++s)
                 for (int cc = 0; cc < D / 64; ++cc)
-                  for (int hh = 0; hh < 2; ++hh)
+                  for (int hh = 0; hh < 2; ++hh) {
+                    const int vrow = t * kTileN + hh * 64;
                     tma_load_4d(dst + s * C::kTile + cc * kChunkBytes + hh * (kChunkBytes / 2), m,
-                                ful, cc * 64, kvh[s], box_row(t * kTileN + hh * 64), b);
+                                ful, cc * 64, kvh[s], gitem ? vrow : box_row(vrow), b);
+                  }
             }
           } else {
             // gather global-key rows with plain 16-byte loads into the
@@ -380,11 +438,40 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     const uint32_t tO = tmem + 256u + 128u * slot + lane_off;
     const int h = head[slot];
     const int m_row = qt * kTileM + r;  // local query row
-    const bool row_valid = m_row < Mq && slot_ok[slot];
     const int m_v = q0 + m_row;         // its virtual row among the keys
-    const int klo = max(key_lo(g, m_v), lo_b);
-    const int khi = key_hi(g, m_v, Mv);
-    const int i_phys = (int)phys_row(g, c, m_v);
+    bool row_valid;
+    int klo, khi, i_phys;
+    if (gitem) {
+      // global row: every key of the sequence (causal: up to the row)
+      row_valid = r < gcnt && slot_ok[slot];
+      int gv = r < gcnt ? __ldg(p.G + gq0 + r) : 0;
+      gv = gv < 0 ? 0 : (gv >= p.N ? p.N - 1 : gv);
+      i_phys = gv;
+      klo = 0;
+      khi = r < gcnt ? (p.R == 0 ? gv : p.N - 1) : -1;
+    } else {
+      row_valid = m_row < Mq && slot_ok[slot];
+      klo = max(key_lo(g, m_v), lo_b);
+      khi = key_hi(g, m_v, Mv);
+      i_phys = (int)phys_row(g, c, m_v);
+      // a global row is written by its global tile, not by the band
+      if (glob && row_valid) {
+        int lo = 0, hi = p.n_global - 1;
+        while (lo <= hi) {
+          const int mid = (lo + hi) >> 1;
+          const int gv = __ldg(p.G + mid);
+          if (gv == i_phys) {
+            row_valid = false;
+            break;
+          }
+          if (gv < i_phys) lo = mid + 1;
+          else hi = mid - 1;
+        }
+      }
+    }
+    // a warp of a global tile whose 32 rows are all past the tile's last
+    // global row only keeps the barriers going
+    const bool warp_idle = gitem && quad * 32 >= gcnt;
     const bool causal = p.R == 0;
     // band of the row in physical positions, for the global-key test
     const int glo = p.L < 0 ? -0x40000000
@@ -401,7 +488,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     float m_pend = -INFINITY;  // max seen but not yet adopted (adopted next tile)
     int int_lo, int_hi;        // key tiles that need no element mask
     interior_tiles_rows(g, Mv, qm0, &int_lo, &int_hi);
-    if (lo_b > 0 || qt * kTileM + kTileM > Mq) int_hi = int_lo - 1;  // mask every tile
+    if (gitem || lo_b > 0 || qt * kTileM + kTileM > Mq) int_hi = int_lo - 1;  // mask every tile
 
     // the 64 score columns of key half hf (TMEM -> registers)
     auto read_half = [&](int hf, float (&sv)[64]) {
@@ -419,7 +506,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     // shared select loop
     auto mask_half = [&](int it, int hf, bool edge, float (&sv)[64]) {
       uint64_t keep = ~0ull;
-      if (it < n_band) {
+      if (!glob || it < n_band) {
         if (edge) {
           const int n0 = (tr.kv_begin + it) * kTileN + hf * 64;
           const int lo = max(klo - n0, 0);
@@ -511,11 +598,23 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     // above the running max only enlarge P, by at most 2^64 (safe in fp32
     // and bf16); a larger jump is adopted at once by rescaling O, l, the
     // partial sums and the P already written.
-    for (int it = 0; ok && it < n_tiles; ++it) {
+    for (int it = 0; ok && warp_idle && it < n_tiles; ++it) {
+      // rows without a query: no scores to read and no P to write (the PV
+      // MMA reads whatever these TMEM lanes hold; those O rows are never
+      // stored), but the arrivals keep the phases of the barriers in step
+      const uint32_t ph = (uint32_t)it & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sl_full[slot], ph, p.err, abort_flag))) {
+        ok = false;
+        break;
+      }
+      mbar_arrive(&l_free[slot]);
+      mbar_arrive(&p_full[slot]);
+    }
+    for (int it = 0; ok && !warp_idle && it < n_tiles; ++it) {
       const int e = it & 1;  // early key half; P of the tile lives in its columns
       const uint32_t ph = (uint32_t)it & 1u;
       const int t_kv = tr.kv_begin + it;
-      const bool edge = it < n_band && !(t_kv >= int_lo && t_kv <= int_hi);
+      const bool edge = (!glob || it < n_band) && !(t_kv >= int_lo && t_kv <= int_hi);
 
       // adopt a larger max seen on the previous tile (rare after the start)
       const bool pend = m_pend > m_used;
@@ -588,7 +687,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
       mbar_arrive(&p_full[slot]);
     }
 
-    bool fin = ok && n_tiles > 0;
+    bool fin = ok && n_tiles > 0 && !warp_idle;
     if (fin) fin = mbar_wait(&o_final[slot], 0, p.err, abort_flag);
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
@@ -640,12 +739,12 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
                 int Hkv, int N, int L, int R, int d, int bs, const int32_t* G, int ng,
                 float scale, cudaStream_t stream, const QueryWindow* qw) {
   using C = Cfg<D, NSLOT, NSTREAM>;
-  static std::atomic<unsigned long long> attr_plain{0}, attr_qwin{0};
-  if (!smem_attr_once(reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, false>),
-                      C::kAlloc, attr_plain) ||
-      !smem_attr_once(reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, true>),
-                      C::kAlloc, attr_qwin))
-    return SWA_ERR_CUDA;
+  static std::atomic<unsigned long long> attr_kind[3] = {{0}, {0}, {0}};
+  const int kind = qw ? 1 : (ng > 0 ? 2 : 0);
+  const void* kfn[3] = {reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 0>),
+                        reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 1>),
+                        reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 2>)};
+  if (!smem_attr_once(kfn[kind], C::kAlloc, attr_kind[kind])) return SWA_ERR_CUDA;
   int* err = device_error_word();
   if (!err) return SWA_ERR_CUDA;
   const Geometry geo = make_geometry(N, L, R, d, bs);
@@ -658,6 +757,7 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
     p.G = G;
+    p.q_raw = static_cast<const uint16_t*>(q);
     p.k_raw = static_cast<const uint16_t*>(k);
     p.v_raw = static_cast<const uint16_t*>(v);
     p.err = err;
@@ -708,15 +808,32 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
                        CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return SWA_ERR_CUDA;
     }
-    const long grid = (long)p.qtile_prefix[p.nclass] * B * ((H + NSLOT - 1) / NSLOT);
+    // the global tiles ride with the first launch
+    if (c0 == 0 && kind == 2) {
+      p.n_gq_tiles = (ng + kTileM - 1) / kTileM;
+      p.n_gitems = p.n_gq_tiles * B * ((H + NSLOT - 1) / NSLOT);
+      const uint64_t df[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)N, (uint64_t)B};
+      const uint64_t sf[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
+                              (uint64_t)N * Hkv * D * 2};
+      if (encode_tiled(&p.tmKf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(k), df, sf,
+                       box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+          encode_tiled(&p.tmVf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(v), df, sf,
+                       box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+        return SWA_ERR_CUDA;
+    }
+    const long grid = (long)p.n_gitems +
+                      (long)p.qtile_prefix[p.nclass] * B * ((H + NSLOT - 1) / NSLOT);
     if (grid <= 0) continue;
     if (grid > 0x7fffffffL) return SWA_ERR_UNSUPPORTED;
-    if (qw)
-      swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, true><<<(unsigned)grid, C::kThreads, C::kAlloc,
-                                                      stream>>>(p);
+    if (kind == 1)
+      swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 1><<<(unsigned)grid, C::kThreads, C::kAlloc,
+                                                   stream>>>(p);
+    else if (kind == 2)
+      swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 2><<<(unsigned)grid, C::kThreads, C::kAlloc,
+                                                   stream>>>(p);
     else
-      swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, false><<<(unsigned)grid, C::kThreads, C::kAlloc,
-                                                       stream>>>(p);
+      swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 0><<<(unsigned)grid, C::kThreads, C::kAlloc,
+                                                   stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
   }
   return SWA_OK;

@@ -52,12 +52,6 @@ int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, flo
                      const int32_t* G, int ng, float scale, cudaStream_t stream,
                      const QueryWindow* qw = nullptr);
 
-// Dense rows for global queries: every global row i attends keys
-// [0, N) (causal: [0, i]); overwrites those rows of out / lse.
-int launch_global_rows(const void* q, const void* k, const void* v, void* out, float* lse,
-                       int B, int H, int Hkv, int N, int D, bool causal, const int32_t* G,
-                       int ng, float scale, cudaStream_t stream);
-
 int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* out,
                   float* lse, const int64_t* pos, int B, int H, int Hkv, int D, int W,
                   float scale, cudaStream_t stream);

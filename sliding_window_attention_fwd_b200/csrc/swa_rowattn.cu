@@ -1,12 +1,10 @@
 // swa_rowattn.cu -- split-KV attention of a few query vectors against a long
-// contiguous run of key rows, on CUDA cores.  Two users:
+// contiguous run of key rows, on CUDA cores.  Three users:
 //
 //  * ring-buffer decode: one new token per sequence attends the valid slots
 //    of its W-slot cache (page "大模型窗口扩展技术" §3.1: token t lives in
 //    slot t % W; aiqz.cc page, "推理优化策略": the cache rolls like a
 //    conveyor belt, old entries are overwritten);
-//  * global query rows: a global token attends every key (aiqz.cc page,
-//    "全局注意力token"); causal problems clip it to keys <= its position;
 //  * paged decode: the cache lives in fixed-size pages found through a block
 //    table, so pages that leave the window can be released ("空洞滑窗机制"
 //    page, §四, KV cache management with PagedAttention);
@@ -16,10 +14,10 @@
 //
 // The work is HBM-bound (each key/value byte is used for a handful of
 // flops), so the kernel is built for bandwidth: one CTA streams a chunk of
-// key rows of one (batch, kv head) through a 3-stage TMA ring (64 rows per
+// key rows of one (batch, kv head) through a 2-stage TMA ring (64 rows per
 // stage, 128-byte swizzle so the reads below are bank-conflict free) and
 // serves all NQ query vectors that read those rows (the GQA group of the kv
-// head, and for global rows several global tokens) from that single read.
+// head, and for an append several tokens) from that single read.
 // Math is fp32 on the FMA pipe.  Chunks of one query set are merged with
 // the log-sum-exp identity by whichever CTA of the set finishes last.
 #include <cuda.h>
@@ -43,7 +41,7 @@ constexpr int kComputeWarps = 4;
 constexpr int kThreadsR = (kComputeWarps + 1) * 32;
 
 struct RowParams {
-  CUtensorMap tmK;   // decode: ring; global rows: sequence; paged: page pool
+  CUtensorMap tmK;   // decode: ring; paged: page pool; append: ring
   CUtensorMap tmV;
   CUtensorMap tmKn;  // chunked append: the chunk's new keys / values
   CUtensorMap tmVn;
@@ -53,13 +51,12 @@ struct RowParams {
   uint16_t* out;
   float* lse;
   const int64_t* pos;
-  const int32_t* G;
   float* ws_o;
   float* ws_ml;
   int* cnt;
   int* err;
-  int mode;  // 0: decode, 1: global rows, 2: paged decode, 3: chunked append
-  int B, H, Hkv, N, W, grp, ng, causal;
+  int mode;  // 0: decode, 2: paged decode, 3: chunked append
+  int B, H, Hkv, N, W, grp;
   int rows_per_cta, nrowchunks;
   int chunk, nsplit;
   float scale_log2;
@@ -123,7 +120,7 @@ __device__ __forceinline__ float reduce8_transposed(float (&v)[NQ], int t, int* 
   return w[0];
 }
 
-// MODE: 0 ring decode, 1 global rows, 2 paged decode, 3 chunked append
+// MODE: 0 ring decode, 2 paged decode, 3 chunked append
 // (compile-time, so each user's kernel carries only its own addressing).
 template <int D, int NQ, int MODE>
 __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
@@ -200,23 +197,13 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
         lo_r[s] = (int)((ps - p.W + 1 < 0 ? 0 : ps - p.W + 1) - tA);
         hi_r[s] = (int)(ps - tA);
         qoff[s] = ((long)b * p.H + h) * D;
-      } else if (MODE == 3) {
+      } else {
         const int c = rowchunk * p.rows_per_cta + rsub;
         if (c < p.N) {
           const long long pc = p.pos[b] + c;
           lo_r[s] = (int)((pc - p.W + 1 < 0 ? 0 : pc - p.W + 1) - tA);
           hi_r[s] = (int)(pc - tA);
           qoff[s] = (((long)b * p.N + c) * p.H + h) * D;
-        }
-      } else {
-        const int j = rowchunk * p.rows_per_cta + rsub;
-        if (j < p.ng) {
-          int i = p.G[j];
-          i = i < 0 ? 0 : (i >= p.N ? p.N - 1 : i);
-          const int limit = p.causal ? i + 1 : p.N;
-          hi_r[s] = limit - 1;
-          qoff[s] = (((long)b * p.N + i) * p.H + h) * D;
-          max_limit = limit > max_limit ? limit : max_limit;
         }
       }
     }
@@ -354,7 +341,7 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
           const int idx = key0 + k * kRows + r;
           const int rel = idx < seg_n ? idx : idx + off_b;
           int lo = lo_r[0], hi = hi_r[0];  // decode, paged: one sequence per set
-          if (MODE == 1 || MODE == 3) {
+          if (MODE == 3) {
 #pragma unroll
             for (int s = 1; s < NQ; ++s)
               if (s == myslot) {
@@ -362,7 +349,7 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
                 hi = hi_r[s];
               }
           }
-          const bool ok = (MODE == 0 || MODE == 1)
+          const bool ok = MODE == 0
                               ? idx <= hi
                               : (rel >= lo && rel <= hi && (idx >= seg_n || rel < a_end_r));
           sc[r * NQ + myslot] = ok ? tot : -INFINITY;
@@ -474,7 +461,7 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
     if (p.lse && threadIdx.x < NQ && qoff[threadIdx.x] >= 0) {
       const int s = threadIdx.x;
       const float lv = (sc[s] + __log2f(sc[NQ + s])) * 0.69314718055994531f;
-      const long row = qoff[s] / D;  // decode: b*H + h; global: (b*N + i)*H + h
+      const long row = qoff[s] / D;  // decode: b*H + h; append: (b*C + c)*H + h
       long li;
       if (MODE == 0 || MODE == 2) li = row;
       else {
@@ -550,7 +537,7 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
 }
 
 // ------------------------------------------------------------ workspaces
-// Per device and per user (0: decode, 1: global rows, 2: paged decode,
+// Per device and per user (0: decode, 1: unused, 2: paged decode,
 // 3: chunked append, 4: the staged key sequence of a tensor-core append):
 // split counters and
 // split partials in separate buffers.  Every merge resets its counter to
@@ -564,7 +551,7 @@ struct Workspace {
   size_t part_bytes = 0;
 };
 constexpr int kMaxDev = 64;
-Workspace g_ws[kMaxDev][5];  // users: decode, global rows, paged, append, append staging
+Workspace g_ws[kMaxDev][5];  // users: decode, (unused), paged, append, append staging
 std::mutex g_ws_mu;
 
 bool get_workspace(int which, size_t cnt_bytes, size_t part_bytes, cudaStream_t stream,
@@ -619,12 +606,9 @@ int launch_rows(RowParams& p, int nsets, cudaStream_t stream) {
 }
 
 // decode and paged decode serve a GQA group (1, 2, 4 or 8 query vectors);
-// global rows and chunked append always fill 8 slots
+// a chunked append fills 4 or 8 slots with whole groups
 template <int D>
 int dispatch_nq(RowParams& p, int nq, int nsets, cudaStream_t stream) {
-  if (p.mode == 1)
-    return nq == 8 ? launch_rows<D, 8, 1>(p, nsets, stream)
-                   : (nq == 4 ? launch_rows<D, 4, 1>(p, nsets, stream) : SWA_ERR_UNSUPPORTED);
   if (p.mode == 3)
     return nq == 8 ? launch_rows<D, 8, 3>(p, nsets, stream)
                    : (nq == 4 ? launch_rows<D, 4, 3>(p, nsets, stream) : SWA_ERR_UNSUPPORTED);
@@ -758,36 +742,6 @@ int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* o
   p.scale_log2 = scale * 1.4426950408889634f;
   const int nq = pow2_at_least(p.grp);
   return run(p, D, nq, B * Hkv, 0, stream);
-}
-
-int launch_global_rows(const void* q, const void* k, const void* v, void* out, float* lse,
-                       int B, int H, int Hkv, int N, int D, bool causal, const int32_t* G,
-                       int ng, float scale, cudaStream_t stream) {
-  RowParams p;
-  std::memset(&p, 0, sizeof(p));
-  if (encode_kv(&p.tmK, k, D, Hkv, N, B) != SWA_OK || encode_kv(&p.tmV, v, D, Hkv, N, B) != SWA_OK)
-    return SWA_ERR_CUDA;
-  p.q = static_cast<const uint16_t*>(q);
-  p.out = static_cast<uint16_t*>(out);
-  p.lse = lse;
-  p.G = G;
-  p.err = device_error_word();
-  if (!p.err) return SWA_ERR_CUDA;
-  p.mode = 1;
-  p.B = B;
-  p.H = H;
-  p.Hkv = Hkv;
-  p.N = N;
-  p.grp = H / Hkv;
-  p.ng = ng;
-  p.causal = causal ? 1 : 0;
-  const int nq = p.grp <= 4 ? 4 : 8;
-  p.rows_per_cta = nq / p.grp;
-  p.nrowchunks = (ng + p.rows_per_cta - 1) / p.rows_per_cta;
-  p.chunk = 512;
-  p.nsplit = (N + p.chunk - 1) / p.chunk;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  return run(p, D, nq, B * Hkv * p.nrowchunks, 1, stream);
 }
 
 int launch_decode_paged(const void* q, const void* k_pages, const void* v_pages, void* out,

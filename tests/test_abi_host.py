@@ -89,9 +89,9 @@ def fwd(*, q=A, k=A, v=A, out=A, lse=None, B=1, H=4, Hkv=2, N=64, D=128, L_=8, R
     (dict(D=96), UNSUP),
     (dict(D=256), UNSUP),
     (dict(bs=32), UNSUP),
-    # global query rows serve GQA groups of up to 8 (a wider group used to
-    # reach a division by zero in the launcher)
-    (dict(H=32, Hkv=2, ng=1, G=A), UNSUP),
+    # global query rows run in the fused kernel, which serves any GQA group
+    # (B = 0 keeps the call on the host)
+    (dict(H=32, Hkv=2, ng=1, G=A, B=0), OK),
     (dict(H=32, Hkv=2, B=0), OK),
     (dict(B=0), OK),
     (dict(N=0), OK),

@@ -108,6 +108,13 @@ SMALL_BF16 = [
     (1, 1000, 2, 2, 64, 128, 0, 2, 64, [3, 500]),  # block, causal, ragged, globals
     (1, 500, 8, 1, 128, 64, 64, 1, 0, [0, 250]),   # globals with a GQA group of 8
     (1, 400, 8, 2, 64, 40, 0, 1, 0, [5, 399]),     # globals, GQA 4, causal, last row global
+    # global query rows run inside the fused launch (global tiles of up to
+    # 128 rows each, every key of the sequence):
+    (1, 300, 32, 2, 128, 30, 30, 1, 0, [0, 100, 299]),        # GQA 16 with globals
+    (1, 700, 4, 4, 64, 20, 0, 1, 0, list(range(0, 700, 4))),  # 175 globals: two global tiles
+    (2, 900, 2, 2, 64, 16, 16, 4, 0, [1, 2, 450, 899]),       # token dilation + globals
+    (1, 96, 2, 1, 128, 3, 3, 1, 0, list(range(96))),          # every row global = full attention
+    (1, 260, 3, 3, 128, 10, 0, 1, 0, [129, 130, 259]),        # odd head count, causal
 ]
 
 
@@ -172,3 +179,26 @@ def test_bf16_score_jumps(swa, D, H, Hkv):
     k = k.to(torch.bfloat16)
     full_check(swa, (q, k, v, 600, 0, 1, 0, None, 0.0))
     full_check(swa, (q, k, v, 200, 200, 1, 0, None, 0.0))
+
+
+def test_globals_allocate_nothing(swa):
+    """The forward with global tokens runs in one launch with no library
+    workspace: after swa_release() the device's free memory is unchanged by
+    the call (torch's own tensors are made before the first reading)."""
+    cfg = inputs.CONFIGS["small_global"]
+    q, k, v, G = inputs.forward_inputs(cfg)
+    qd, kd, vd, Gd = q.cuda(), k.cuda(), v.cuda(), G.cuda()
+    out = torch.empty_like(qd)
+    lse = torch.empty(cfg.B, cfg.H, cfg.N, device="cuda")
+    swa.swa_release()
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    swa.swa_forward(qd, kd, vd, out, lse, cfg.win_left, cfg.win_right, cfg.dilation, Gd,
+                    cfg.scale)
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert swa.swa_device_error() == 0
+    ref_o, ref_l = oracle.forward(q, k, v, cfg.win_left, cfg.win_right, cfg.dilation, 0, G.numpy(),
+                                  cfg.scale)
+    compare(out.float().cpu().numpy(), ref_o, BF16_MAX_ABS, BF16_MEAN_ABS, what="out")
+    compare(lse.cpu().numpy(), ref_l, LSE_ABS, what="lse")
