@@ -25,18 +25,24 @@
 //              Tile j's P is kept in the columns of its early half (j & 1);
 //              the early half of tile j+1 goes to the other columns as soon
 //              as the softmax has read them, so it is ready when the softmax
-//              finishes tile j, and only the late half waits for PV(j).  One
-//              issuer per slot, each on its own SM sub-partition: a single
-//              issuer sharing a sub-partition with two busy softmax warps
-//              gets too few issue slots to keep the tensor core fed;
+//              finishes tile j, and only the late half waits for PV(j).  PV
+//              itself is issued in two key halves: the early half's share as
+//              soon as its P is written, so only a quarter-tile of PV sits
+//              between the end of tile j's softmax and S of tile j+1's late
+//              half.  One issuer per slot, each on its own SM sub-partition:
+//              a single issuer sharing a sub-partition with two busy softmax
+//              warps gets too few issue slots to keep the tensor core fed;
 //   softmax    thread t of warpgroup 1+s owns query row t of slot s: row max
 //              and row sum are thread-local tree reductions, no shuffles.
 //              Element masks only on tiles the scheduler marks as edges.
 //              Scores are read from TMEM 64 columns at a time and turned into
-//              P against the current running max in the same pass (the max
-//              changes rarely); a max that grows by more than 2^8 is adopted
-//              before the next tile by rescaling O and l, and the final
-//              O / l is exact either way.
+//              P against the current running max while the half's max is
+//              found (the max changes rarely); a max that grows by more than
+//              2^8 is adopted before the next tile by rescaling O and l, one
+//              that jumps by more than 2^64 at once (the half is redone), and
+//              the final O / l is exact either way.  With two slots the
+//              producer/issuer warpgroup gives registers to the softmax
+//              warpgroups (setmaxnreg), which then run without spills.
 // Per row: out = O / l (bf16), lse = m + ln l (fp32).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -105,7 +111,7 @@ struct Cfg {
   static constexpr int kBar = kRing + kStages * kStageBytes;
   // full_q, full_k[S], empty_k[S], full_v[S], empty_v[S],
   // se_full[2], sl_full[2], l_free[2], p_full[2], o_done[2], o_final[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 12;
+  static constexpr int kNumBars = 1 + 4 * kStages + 16;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
@@ -135,6 +141,8 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
   uint64_t* p_full = l_free + 2;
   uint64_t* o_done = p_full + 2;
   uint64_t* o_final = o_done + 2;
+  uint64_t* pe_full = o_final + 2;  // [slot]: P of the early half written
+  uint64_t* oe_done = pe_full + 2;  // [slot]: PV of the early half done
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
 
@@ -221,6 +229,8 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
       mbar_init(&p_full[s], 128);
       mbar_init(&o_done[s], 1);
       mbar_init(&o_final[s], 1);
+      mbar_init(&pe_full[s], 128);
+      mbar_init(&oe_done[s], 1);
     }
     fence_mbar_init();
   }
@@ -242,6 +252,9 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
   };
 
   if (warp < 4) {
+    // producer and issuers need few registers: hand the rest to the softmax
+    // warpgroups (128 x 56 + 256 x 208 = 60416 <= 384 x 168 launched)
+    if (NSLOT == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
     if (warp == 0) {
       // =========================== producer ===========================
       const CUtensorMap* mapK = gitem ? &p.tmKf : &p.tmK[map_idx];
@@ -374,21 +387,24 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
           }
           tc_commit(done);
         };
-        // O_s += P_s V of tile it; P (bf16 pairs) sits in the columns of the
-        // early half e: keys of half e at [64 e, 64 e + 32), keys of the
-        // other half at [64 e + 32, 64 e + 64)
-        auto pv = [&](int it) {
+        // O_s += P_s V over the keys of one half of tile it.  P (bf16 pairs)
+        // sits in the columns of the tile's early half e = it & 1: the early
+        // keys' P at [64 e, 64 e + 32), the late keys' at [64 e + 32, 64 e + 64).
+        // The early half's share is issued as soon as its P is written, so
+        // after the softmax finishes a tile only a quarter-tile of PV stands
+        // between it and the late half of the next tile's S.
+        auto pv_half = [&](int it, bool early) {
           const uint64_t dv = dv0 + (uint64_t)(it % kStages) * kStageStep;
           const uint32_t to = tmem + 256u + 128u * s;
-          const uint32_t tp = tslot + 64u * (uint32_t)(it & 1);
-          const int odd = it & 1;
+          const int e = it & 1;
+          const uint32_t tp = tslot + 64u * (uint32_t)e + (early ? 0u : 32u);
+          const int kh = early ? e : (e ^ 1);  // key half
 #pragma unroll
-          for (int k = 0; k < kTileN / 16; ++k) {
-            const uint32_t col = ((k / 4) != odd ? 32u : 0u) + 8u * (k % 4);
-            mma_ts(to, tp + col, dv + (uint64_t)((k * 2048) >> 4), idesc_pv,
-                   (it > 0 || k > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const int k = kh * 4 + kk;
+            mma_ts(to, tp + 8u * kk, dv + (uint64_t)((k * 2048) >> 4), idesc_pv,
+                   (it > 0 || !early || kk > 0) ? 1u : 0u);
           }
-          tc_commit(&o_done[s]);
         };
         bool ok = mbar_wait(full_q, 0, p.err, abort_flag) &&
                   mbar_wait(&full_k[0], 0, p.err, abort_flag);
@@ -402,6 +418,12 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
           const int st = it % kStages;
           const bool more = it + 1 < n_tiles;
           const int e_next = (it + 1) & 1;  // early half of tile it + 1
+          // the early half's P is in TMEM: its share of PV goes first
+          if (!mbar_wait(&pe_full[s], (uint32_t)it & 1u, p.err, abort_flag)) break;
+          if (!mbar_wait(&full_v[st], (uint32_t)(it / kStages) & 1u, p.err, abort_flag)) break;
+          tc_fence_after();
+          pv_half(it, true);
+          tc_commit(&oe_done[s]);
           if (more) {
             // the softmax has read the late half of tile it; K of tile it + 1
             if (!mbar_wait(&l_free[s], (uint32_t)it & 1u, p.err, abort_flag)) break;
@@ -413,9 +435,9 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
           }
           // P of tile it is in TMEM; V of tile it
           if (!mbar_wait(&p_full[s], (uint32_t)it & 1u, p.err, abort_flag)) break;
-          if (!mbar_wait(&full_v[st], (uint32_t)(it / kStages) & 1u, p.err, abort_flag)) break;
           tc_fence_after();
-          pv(it);
+          pv_half(it, false);
+          tc_commit(&o_done[s]);
           tc_commit(&empty_v[st]);
           if (more) {
             qk_half(it + 1, e_next ^ 1, &sl_full[s]);
@@ -429,6 +451,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
       __syncwarp();
     }
   } else {
+    if (NSLOT == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
     // ============================ softmax ============================
     const int slot = warp / 4 - 1;
     const int quad = warp & 3;
@@ -545,9 +568,10 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
       return max3f(max3f(t[0], t[1], t[2]), max3f(t[3], t[4], t[5]), fmaxf(t[6], t[7]));
     };
     // P = 2^(s * scale * log2 e - m_ref) for one key half, stored as 32
-    // columns of bf16 pairs from TMEM column pcol.  Three of every four
+    // columns of bf16 pairs from TMEM column pcol.  Seven of every eight
     // column pairs go to the MUFU ex2 unit and one to the FMA pipe
-    // (polynomial), so the two softmax warpgroups do not saturate MUFU.
+    // (polynomial), which takes some load off MUFU (measured best of 0, 1/8,
+    // 1/4 and 1/2 on the FMA pipe with the split PV and the register split).
     auto exp_half = [&](int pcol, const float (&sv)[64], float m_ref, float2 (&ls)[4]) {
       const float2 sl2_2 = make_float2(sl2, sl2), negm2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
@@ -558,7 +582,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
           const float2 xa =
               fma2(make_float2(sv[jj * 32 + 2 * e], sv[jj * 32 + 2 * e + 1]), sl2_2, negm2);
           float2 pr;
-          if ((e & 3) == 3) {
+          if ((e & 7) == 7) {
             pr = exp2_poly2(xa);
           } else {
             pr.x = ex2_approx(xa.x);
@@ -607,6 +631,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
         ok = false;
         break;
       }
+      mbar_arrive(&pe_full[slot]);
       mbar_arrive(&l_free[slot]);
       mbar_arrive(&p_full[slot]);
     }
@@ -632,16 +657,35 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
       tc_fence_after();
       read_half(e, sv);
       mask_half(it, e, edge, sv);
-      float tmax = half_max(sv);
-      {
+      float tmax;
+      if (!__any_sync(0xffffffffu, m_used == -INFINITY)) {
+        // optimistic: exponentiate against the running max while the half's
+        // max is found (no dependence between the two); a jump (rare)
+        // rescales O and l and redoes the half against the new max
+        exp_half(64 * e, sv, m_used, ls);
+        tmax = half_max(sv);
+        const bool jump = tmax * sl2 > m_used + 64.f;
+        if (__any_sync(0xffffffffu, jump)) {
+          if (!rescale_o(it, jump, fmaxf(m_used, tmax * sl2))) { ok = false; break; }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) ls[j] = make_float2(0.f, 0.f);
+          tmem_wait_st();
+          exp_half(64 * e, sv, m_used, ls);
+        }
+      } else {
+        // some row of the warp meets its first keys: find the max first
+        tmax = half_max(sv);
         const bool adopt = m_used == -INFINITY;
         const bool jump = !adopt && tmax * sl2 > m_used + 64.f;
         if (adopt) m_used = tmax * sl2;
         if (__any_sync(0xffffffffu, jump)) {
           if (!rescale_o(it, jump, fmaxf(m_used, tmax * sl2))) { ok = false; break; }
         }
+        exp_half(64 * e, sv, m_used == -INFINITY ? 0.f : m_used, ls);
       }
-      exp_half(64 * e, sv, m_used == -INFINITY ? 0.f : m_used, ls);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&pe_full[slot]);
 
       // ---- late half
       w_ok = mbar_wait(&sl_full[slot], ph, p.err, abort_flag);
@@ -652,30 +696,48 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
       tc_fence_before();
       mbar_arrive(&l_free[slot]);
       mask_half(it, e ^ 1, edge, sv);
-      const float tmax1 = half_max(sv);
-      tmax = fmaxf(tmax, tmax1);
-      {
+      if (!__any_sync(0xffffffffu, m_used == -INFINITY)) {
+        // optimistic as above; on a jump O must also hold the early half's
+        // PV (issued once its P was written) before it is scaled
+        float2 lh[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
+        exp_half(64 * e + 32, sv, m_used, lh);
+        const float tmax1 = half_max(sv);
+        tmax = fmaxf(tmax, tmax1);
+        const bool jump = tmax1 * sl2 > m_used + 64.f;
+        if (__any_sync(0xffffffffu, jump)) {
+          const float m_old = m_used;
+          const bool oe_ok = mbar_wait(&oe_done[slot], (uint32_t)it & 1u, p.err, abort_flag);
+          if (!__all_sync(0xffffffffu, oe_ok)) { ok = false; break; }
+          if (!rescale_o(it, jump, fmaxf(m_used, tmax1 * sl2))) { ok = false; break; }
+          const float f = jump ? ex2_approx(m_old - m_used) : 1.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            ls[j] = make_float2(ls[j].x * f, ls[j].y * f);
+            lh[j] = make_float2(0.f, 0.f);
+          }
+          tmem_wait_st();
+          exp_half(64 * e + 32, sv, m_used, lh);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ls[j] = add2(ls[j], lh[j]);
+      } else {
+        const float tmax1 = half_max(sv);
+        tmax = fmaxf(tmax, tmax1);
         const bool adopt = m_used == -INFINITY;
         const bool jump = !adopt && tmax1 * sl2 > m_used + 64.f;
         if (adopt) m_used = tmax1 * sl2;
         if (__any_sync(0xffffffffu, jump)) {
           const float m_old = m_used;
+          const bool oe_ok = mbar_wait(&oe_done[slot], (uint32_t)it & 1u, p.err, abort_flag);
+          if (!__all_sync(0xffffffffu, oe_ok)) { ok = false; break; }
           if (!rescale_o(it, jump, fmaxf(m_used, tmax1 * sl2))) { ok = false; break; }
           const float f = jump ? ex2_approx(m_old - m_used) : 1.f;
 #pragma unroll
           for (int j = 0; j < 4; ++j) ls[j] = make_float2(ls[j].x * f, ls[j].y * f);
-          uint32_t v[32];
-          tmem_wait_st();
-          tmem_ld32(tS + 64 * e, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            v[j] = pack_bf16x2(__uint_as_float(v[j] << 16) * f,
-                               __uint_as_float(v[j] & 0xFFFF0000u) * f);
-          tmem_st32(tS + 64 * e, v);
         }
+        exp_half(64 * e + 32, sv, m_used == -INFINITY ? 0.f : m_used, ls);
       }
-      exp_half(64 * e + 32, sv, m_used == -INFINITY ? 0.f : m_used, ls);
       {
         const float2 a2 = add2(add2(ls[0], ls[1]), add2(ls[2], ls[3]));
         l += a2.x + a2.y;
@@ -745,6 +807,19 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
                         reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 1>),
                         reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 2>)};
   if (!smem_attr_once(kfn[kind], C::kAlloc, attr_kind[kind])) return SWA_ERR_CUDA;
+  if (NSLOT == 2) {
+    // The register split (warpgroup 0: 56 per thread, the softmax
+    // warpgroups: 208) must fit in what the block is launched with, or
+    // setmaxnreg.inc would never return: checked once per kernel form.
+    static std::atomic<int> regs_ok[3] = {{0}, {0}, {0}};
+    if (regs_ok[kind].load(std::memory_order_acquire) == 0) {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kfn[kind]) != cudaSuccess) return SWA_ERR_CUDA;
+      regs_ok[kind].store((long)fa.numRegs * C::kThreads >= 128L * 56 + 256L * 208 ? 1 : -1,
+                          std::memory_order_release);
+    }
+    if (regs_ok[kind].load(std::memory_order_acquire) < 0) return SWA_ERR_UNSUPPORTED;
+  }
   int* err = device_error_word();
   if (!err) return SWA_ERR_CUDA;
   const Geometry geo = make_geometry(N, L, R, d, bs);
