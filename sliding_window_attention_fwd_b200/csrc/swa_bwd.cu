@@ -1,4 +1,6 @@
-// swa_bwd.cu -- sliding-window attention backward (dq, dk, dv) on CUDA cores.
+// swa_bwd.cu -- sliding-window attention backward (dq, dk, dv): the entry
+// point, and the CUDA-core kernel that serves problems with global tokens
+// (band problems run on the tensor cores, swa_bwd_sm100.cu).
 //
 // The pages use the method for training but describe no backward pass; this
 // is the derivative of the forward definition, over the same key sets (band
@@ -349,6 +351,16 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
                     const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                     int H, int Hkv, int N, int D, int L, int R, int d, int bs, const int32_t* G,
                     int ng, float scale, cudaStream_t stream) {
+  if (ng == 0) {
+    // band problems: the tensor-core kernels (swa_bwd_sm100.cu), with a
+    // [B, H, N] fp32 workspace for Delta_i = dO_i . out_i
+    float* delta = bwd_workspace((size_t)B * H * N * sizeof(float), stream);
+    if (!delta) return SWA_ERR_NOMEM;
+    return launch_backward_tc(q, k, v, out, dout, lse, dq, dk, dv, delta, B, H, Hkv, N, D, L, R,
+                              d, bs, scale, stream);
+  }
+  // with global tokens (whole-sequence rows and columns of the key sets):
+  // one warp per (batch, row, kv head) on CUDA cores, below
   const size_t n_kv = (size_t)B * N * Hkv * D;
   float* acc = bwd_workspace(2 * n_kv * sizeof(float), stream);
   if (!acc) return SWA_ERR_NOMEM;

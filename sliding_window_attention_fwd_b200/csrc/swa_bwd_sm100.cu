@@ -1,0 +1,744 @@
+// swa_bwd_sm100.cu -- sliding-window attention backward on the tcgen05
+// tensor cores (bf16 operands, fp32 accumulators in TMEM).
+//
+// The pages train with the method but print no backward pass; this is the
+// derivative of the forward definition over the same key sets (band with
+// token- or block-level dilation, causal clip), with keys outside the
+// window never touched.  With P_ij = exp(s_ij - lse_i) recomputed from the
+// forward's lse and Delta_i = dO_i . out_i:
+//   dP_ij = dO_i . v_j,   dS_ij = P_ij (dP_ij - Delta_i),
+//   dQ_i = scale sum_j dS_ij k_j,   dK_j = scale sum_i dS_ij q_i,
+//   dV_j = sum_i P_ij dO_i.
+// Every product above is a dense contraction inside a 128 x 128 tile, so it
+// runs on the tensor cores; the element-wise steps (exp, dS) run on the
+// CUDA cores of four "compute" warps, one thread per TMEM lane.
+//
+// Two kernels, no atomics:
+//  * swa_bwd_dq_kernel, query-stationary: a CTA owns 128 query rows of one
+//    head (Q and dO tiles in shared memory) and walks the key tiles of the
+//    band (the forward's scheduler):
+//        S = Q K^T, dP = dO V^T      tcgen05.mma (smem x smem), TMEM fp32
+//        dS (bf16) over S's columns  compute warps
+//        dQ += dS K                  tcgen05.mma (TMEM x smem)
+//    It also writes Delta_i for the second kernel.
+//  * swa_bwd_dkdv_kernel, key-stationary: a CTA owns 128 key rows of one kv
+//    head (K and V tiles in shared memory) and walks every (query tile,
+//    query head of the GQA group) whose rows see those keys (the transposed
+//    scheduler, query_lo / query_hi):
+//        S^T = K Q^T, dP^T = V dO^T  tcgen05.mma (smem x smem)
+//        P^T, dS^T (bf16) in place   compute warps (one key row per thread)
+//        dV += P^T dO, dK += dS^T Q  tcgen05.mma (TMEM x smem)
+//    dK and dV stay in TMEM for the CTA's whole walk.
+// Warp roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer (and
+// TMEM owner), warps 4-7 compute.  Every wait is bounded (swa_ptx.cuh).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "swa_internal.h"
+#include "swa_ptx.cuh"
+#include "swa_sched.cuh"
+
+namespace swa {
+namespace {
+
+constexpr int kMaxClassesB = 8;                 // residue classes per launch
+constexpr int kChunkB = kTileM * 128;           // 128 rows x 64 bf16 columns
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kThreadsB = 256;
+
+struct BwdTcParams {
+  CUtensorMap tmQ[kMaxClassesB];
+  CUtensorMap tmDO[kMaxClassesB];
+  CUtensorMap tmK[kMaxClassesB];
+  CUtensorMap tmV[kMaxClassesB];
+  const uint16_t* out;
+  const uint16_t* dout;
+  const float* lse;
+  float* delta;  // [B, H, N] fp32: written by the dq kernel, read by the dkdv kernel
+  uint16_t* dq;
+  uint16_t* dk;
+  uint16_t* dv;
+  int* err;
+  int B, H, Hkv, N, grp;
+  int L, R, d, bs;
+  int class0, nclass;
+  int tile_prefix[kMaxClassesB + 1];  // 128-row tiles per class, prefix sums
+  int Mv[kMaxClassesB];
+  float scale, scale_log2;
+};
+
+template <int D>
+struct BCfg {
+  static constexpr int kTile = D / 64 * kChunkB;  // 128 rows x D bf16
+  static constexpr int kStages = D == 128 ? 2 : 3;
+  // two fixed tiles at offset 0 (dq: Q, dO; dkdv: K, V), then the stages of
+  // two streamed tiles (dq: K, V; dkdv: Q, dO)
+  static constexpr int kRing = 2 * kTile;
+  static constexpr int kStageBytes = 2 * kTile;
+  static constexpr int kVec = kRing + kStages * kStageBytes;  // dkdv: [stage][lse2 | delta][128]
+  static constexpr int kBar = kVec + kStages * 2 * kTileM * 4;
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 * kStages + 4;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kAlloc = kMisc + 16 + 1024;  // slack for 1024-byte alignment
+  static_assert(kAlloc <= 232448, "shared memory budget");
+  // TMEM columns: S (or S^T) [0, 128), dP (or dP^T) [128, 256), then the
+  // accumulators: dq kernel dQ [256, 256 + D); dkdv kernel dV, dK.
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+__device__ __forceinline__ int box_row_of(const BwdTcParams& p, int c, int vrow) {
+  return p.bs > 1 ? (c + p.d * (vrow / kBlockRows)) * kBlockRows + vrow % kBlockRows : vrow;
+}
+
+// Loads one 128-row tile (D columns) as 64-row x 64-column boxes into the
+// swizzled layout the MMA descriptors expect.
+template <int D>
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* m, uint64_t* bar,
+                                          const BwdTcParams& p, int c, int head, int vrow0,
+                                          int b) {
+  for (int cc = 0; cc < D / 64; ++cc)
+    for (int hh = 0; hh < 2; ++hh)
+      tma_load_4d(dst + cc * kChunkB + hh * (kChunkB / 2), m, bar, cc * 64, head,
+                  box_row_of(p, c, vrow0 + hh * 64), b);
+}
+
+// K-major operand tile descriptor offset of K-step k (16 columns).
+__device__ __forceinline__ uint64_t kmajor_off(int k) {
+  return (uint64_t)(((k / 4) * kChunkB + (k % 4) * 32) >> 4);
+}
+
+// 2^x for a pair: MUFU for one element, the FMA-pipe polynomial for the
+// other when `poly` (one warp per sub-partition: the FMA pipe is idle).
+__device__ __forceinline__ float2 exp2_pair(float2 x, bool poly) {
+  if (poly) return exp2_poly2(x);
+  return make_float2(ex2_approx(x.x), ex2_approx(x.y));
+}
+
+// ======================================================== dq kernel
+template <int D>
+__global__ void __launch_bounds__(kThreadsB, 1)
+    swa_bwd_dq_kernel(const __grid_constant__ BwdTcParams p) {
+  using C = BCfg<D>;
+  constexpr int S_ = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBar);
+  uint64_t* full_q = bars;              // Q and dO tiles
+  uint64_t* full_k = bars + 1;          // [S_]
+  uint64_t* full_v = full_k + S_;       // [S_]
+  uint64_t* empty_k = full_v + S_;      // [S_]
+  uint64_t* empty_v = empty_k + S_;     // [S_]
+  uint64_t* s_full = empty_v + S_;      // S of the step in TMEM
+  uint64_t* dp_full = s_full + 1;       // dP of the step in TMEM
+  uint64_t* ds_full = dp_full + 1;      // dS of the step written (128 arrivals)
+  uint64_t* done = ds_full + 1;         // every MMA finished
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // ---- work item: (class, query tile, batch, head); heavy (late) tiles first
+  int x = blockIdx.x;
+  const int h = x % p.H;
+  x /= p.H;
+  const int b = x % p.B;
+  x /= p.B;
+  const int jt = p.tile_prefix[p.nclass] - 1 - x;
+  int cl = 0;
+  while (cl + 1 < p.nclass && p.tile_prefix[cl + 1] <= jt) ++cl;
+  const int qt = jt - p.tile_prefix[cl];
+  const int c = p.class0 + cl;
+  const int g_kv = h / p.grp;
+  const Geometry geo = make_geometry(p.N, p.L, p.R, p.d, p.bs);
+  const int Mv = p.Mv[cl];
+  const TileRange tr = tile_range(geo, Mv, qt);
+  const int n_tiles = tr.kv_end - tr.kv_begin;
+  const int map_idx = p.bs > 1 ? 0 : cl;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(full_q, 1);
+    for (int s = 0; s < S_; ++s) {
+      mbar_init(&full_k[s], 1);
+      mbar_init(&full_v[s], 1);
+      mbar_init(&empty_k[s], 1);
+      mbar_init(&empty_v[s], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(ds_full, 128);
+    mbar_init(done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t q_addr = smem_u32(smem);
+  const uint32_t do_addr = q_addr + C::kTile;
+  const uint32_t ring_addr = smem_u32(smem + C::kRing);
+
+  if (warp == 0) {
+    // ============================== producer ==============================
+    if (lane == 0) {
+      prefetch_tensormap(&p.tmQ[map_idx]);
+      prefetch_tensormap(&p.tmDO[map_idx]);
+      prefetch_tensormap(&p.tmK[map_idx]);
+      prefetch_tensormap(&p.tmV[map_idx]);
+      mbar_arrive_expect_tx(full_q, 2 * C::kTile);
+      load_tile<D>(smem, &p.tmQ[map_idx], full_q, p, c, h, qt * kTileM, b);
+      load_tile<D>(smem + C::kTile, &p.tmDO[map_idx], full_q, p, c, h, qt * kTileM, b);
+      for (int it = 0; it < n_tiles; ++it) {
+        const int st = it % S_;
+        const uint32_t ph = (uint32_t)(it / S_) & 1u;
+        const int t = tr.kv_begin + it;
+        uint8_t* kb = smem + C::kRing + st * C::kStageBytes;
+        if (it >= S_ && !mbar_wait(&empty_k[st], ph ^ 1u, p.err, abort_flag)) break;
+        mbar_arrive_expect_tx(&full_k[st], C::kTile);
+        load_tile<D>(kb, &p.tmK[map_idx], &full_k[st], p, c, g_kv, t * kTileN, b);
+        if (it >= S_ && !mbar_wait(&empty_v[st], ph ^ 1u, p.err, abort_flag)) break;
+        mbar_arrive_expect_tx(&full_v[st], C::kTile);
+        load_tile<D>(kb + C::kTile, &p.tmV[map_idx], &full_v[st], p, c, g_kv, t * kTileN, b);
+      }
+    }
+  } else if (warp == 1) {
+    // ============================== MMA issuer ==============================
+    if (lane == 0 && n_tiles > 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(kTileM, kTileN, 0, 0);
+      const uint32_t idesc_dq = idesc_bf16_f32(kTileM, D, 0, 1);
+      const uint64_t dq_ = sdesc_sw128(q_addr, 16, 1024);
+      const uint64_t ddo = sdesc_sw128(do_addr, 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(ring_addr, 16, 1024);                // K, K-major
+      const uint64_t dkmn0 = sdesc_sw128(ring_addr, kChunkB, 1024);         // K, MN-major
+      const uint64_t dv0 = sdesc_sw128(ring_addr + C::kTile, 16, 1024);     // V, K-major
+      constexpr uint64_t kStageStep = C::kStageBytes >> 4;
+      bool ok = mbar_wait(full_q, 0, p.err, abort_flag);
+      for (int it = 0; ok && it < n_tiles; ++it) {
+        const int st = it % S_;
+        const uint32_t ph = (uint32_t)(it / S_) & 1u;
+        // S = Q K^T (the previous step's dQ MMA, issued before, has read dS)
+        if (!mbar_wait(&full_k[st], ph, p.err, abort_flag)) break;
+        tc_fence_after();
+        const uint64_t dk = dk0 + (uint64_t)st * kStageStep;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_ss(tmem, dq_ + kmajor_off(k), dk + kmajor_off(k), idesc_s, k > 0 ? 1u : 0u);
+        tc_commit(s_full);
+        // dP = dO V^T
+        if (!mbar_wait(&full_v[st], ph, p.err, abort_flag)) break;
+        tc_fence_after();
+        const uint64_t dv = dv0 + (uint64_t)st * kStageStep;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_ss(tmem + 128u, ddo + kmajor_off(k), dv + kmajor_off(k), idesc_s,
+                 k > 0 ? 1u : 0u);
+        tc_commit(dp_full);
+        tc_commit(&empty_v[st]);
+        // dQ += dS K, dS (bf16) over S's columns
+        if (!mbar_wait(ds_full, (uint32_t)it & 1u, p.err, abort_flag)) break;
+        tc_fence_after();
+        const uint64_t dkmn = dkmn0 + (uint64_t)st * kStageStep;
+#pragma unroll
+        for (int k = 0; k < kTileN / 16; ++k)
+          mma_ts(tmem + 256u, tmem + 8u * k, dkmn + (uint64_t)((k * 2048) >> 4), idesc_dq,
+                 (it > 0 || k > 0) ? 1u : 0u);
+        tc_commit(&empty_k[st]);
+      }
+      tc_commit(done);  // also on the abort path: TMEM quiescent before it is freed
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ============================== compute ==============================
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off;
+    const uint32_t tP = tmem + 128u + lane_off;
+    const uint32_t tQ = tmem + 256u + lane_off;
+    const int m_v = qt * kTileM + r;
+    const bool row_valid = m_v < Mv;
+    const int i_phys = (int)phys_row(geo, c, m_v);
+    const int klo = key_lo(geo, m_v);
+    const int khi = key_hi(geo, m_v, Mv);
+    int int_lo, int_hi;
+    interior_tiles(geo, Mv, qt, &int_lo, &int_hi);
+    const float sl2 = p.scale_log2;
+    // Delta_i = dO_i . out_i and lse in log2 units; rows past the class
+    // end get P = 0
+    float delta = 0.f, lse2 = INFINITY;
+    if (row_valid) {
+      const size_t row = ((size_t)b * p.N + i_phys) * p.H + h;
+      const uint4* a = reinterpret_cast<const uint4*>(p.dout + row * D);
+      const uint4* o = reinterpret_cast<const uint4*>(p.out + row * D);
+      float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 4
+      for (int u = 0; u < D / 8; ++u) {
+        const uint4 wa = __ldg(a + u), wo = __ldg(o + u);
+        const uint32_t xa[4] = {wa.x, wa.y, wa.z, wa.w}, xo[4] = {wo.x, wo.y, wo.z, wo.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc0 = fmaf(__uint_as_float(xa[e] << 16), __uint_as_float(xo[e] << 16), acc0);
+          acc1 = fmaf(__uint_as_float(xa[e] & 0xFFFF0000u), __uint_as_float(xo[e] & 0xFFFF0000u),
+                      acc1);
+        }
+      }
+      delta = acc0 + acc1;
+      const size_t li = ((size_t)b * p.H + h) * p.N + i_phys;
+      lse2 = __ldg(p.lse + li) * kLog2e;
+      p.delta[li] = delta;
+    }
+    bool ok = true;
+    for (int it = 0; it < n_tiles; ++it) {
+      const uint32_t ph = (uint32_t)it & 1u;
+      const int t = tr.kv_begin + it;
+      const bool edge = !(t >= int_lo && t <= int_hi);
+      bool w = mbar_wait(s_full, ph, p.err, abort_flag) && mbar_wait(dp_full, ph, p.err, abort_flag);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t sv[32], dpv[32];
+        tmem_ld32(tS + 32 * ch, sv);
+        tmem_ld32(tP + 32 * ch, dpv);
+        tmem_wait_ld();
+        const int n0 = t * kTileN + 32 * ch;
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float2 xs = fma2(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
+                           make_float2(sl2, sl2), make_float2(-lse2, -lse2));
+          if (edge) {
+            const int j0 = n0 + 2 * e;
+            if (!(j0 >= klo && j0 <= khi && j0 < Mv)) xs.x = -INFINITY;
+            if (!(j0 + 1 >= klo && j0 + 1 <= khi && j0 + 1 < Mv)) xs.y = -INFINITY;
+          }
+          const float2 pr = exp2_pair(xs, (e & 1) != 0 && !edge);
+          const float2 ds = make_float2(pr.x * (__uint_as_float(dpv[2 * e]) - delta),
+                                        pr.y * (__uint_as_float(dpv[2 * e + 1]) - delta));
+          pk[e] = pack_bf16x2(ds.x, ds.y);
+        }
+        // dS of keys [32 ch, 32 ch + 32) -> S columns [16 ch, 16 ch + 16)
+        // (already read: chunk ch / 2 <= ch)
+        tmem_st16(tS + 16 * ch, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    bool fin = ok && n_tiles > 0 && mbar_wait(done, 0, p.err, abort_flag);
+    if (__all_sync(0xffffffffu, fin)) {
+      tc_fence_after();
+      uint16_t* orow = p.dq + (((size_t)b * p.N + i_phys) * p.H + h) * D;
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        uint32_t v[32];
+        tmem_ld32(tQ + 32 * j, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * p.scale,
+                              __uint_as_float(v[2 * e + 1]) * p.scale);
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + j * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
+      }
+    } else if (row_valid && n_tiles == 0) {
+      // no key at all (cannot happen for a valid row: its own key is always
+      // in the window), kept for completeness
+      uint4* dst = reinterpret_cast<uint4*>(p.dq + (((size_t)b * p.N + i_phys) * p.H + h) * D);
+      for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+
+  // ---- teardown: no MMA in flight, then free TMEM
+  if (warp == 1 && lane == 0 && n_tiles > 0 && *abort_flag) {
+    volatile int no_abort = 0;
+    mbar_wait(done, 0, nullptr, &no_abort, 100000000ull);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ======================================================== dk / dv kernel
+template <int D>
+__global__ void __launch_bounds__(kThreadsB, 1)
+    swa_bwd_dkdv_kernel(const __grid_constant__ BwdTcParams p) {
+  using C = BCfg<D>;
+  constexpr int S_ = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBar);
+  uint64_t* full_kv = bars;           // K and V tiles
+  uint64_t* full = bars + 1;          // [S_]: Q, dO tiles + lse / Delta vectors
+  uint64_t* empty = full + S_;        // [S_]
+  uint64_t* st_full = empty + S_;     // S^T and dP^T of the step in TMEM
+  uint64_t* pt_full = st_full + 1;    // P^T, dS^T written (128 arrivals)
+  uint64_t* done = pt_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
+  float* vec = reinterpret_cast<float*>(smem + C::kVec);  // [S_][2][128]
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // ---- work item: (class, key tile, batch, kv head); early (heavy) tiles first
+  int x = blockIdx.x;
+  const int g_kv = x % p.Hkv;
+  x /= p.Hkv;
+  const int b = x % p.B;
+  x /= p.B;
+  const int jt = x;
+  int cl = 0;
+  while (cl + 1 < p.nclass && p.tile_prefix[cl + 1] <= jt) ++cl;
+  const int kt = jt - p.tile_prefix[cl];
+  const int c = p.class0 + cl;
+  const Geometry geo = make_geometry(p.N, p.L, p.R, p.d, p.bs);
+  const int Mv = p.Mv[cl];
+  const TileRange qr = qtile_range_keys(geo, Mv, kt * kTileN);
+  const int grp = p.grp;
+  const int n_steps = (qr.kv_end - qr.kv_begin) * grp;  // (query tile, head of the group)
+  const int map_idx = p.bs > 1 ? 0 : cl;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(full_kv, 1);
+    for (int s = 0; s < S_; ++s) {
+      mbar_init(&full[s], 1 + 32);  // the TMA bytes + every producer lane's vectors
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(st_full, 1);
+    mbar_init(pt_full, 128);
+    mbar_init(done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t k_addr = smem_u32(smem);
+  const uint32_t v_addr = k_addr + C::kTile;
+  const uint32_t ring_addr = smem_u32(smem + C::kRing);
+
+  if (warp == 0) {
+    // ============================== producer ==============================
+    if (lane == 0) {
+      prefetch_tensormap(&p.tmQ[map_idx]);
+      prefetch_tensormap(&p.tmDO[map_idx]);
+      prefetch_tensormap(&p.tmK[map_idx]);
+      prefetch_tensormap(&p.tmV[map_idx]);
+      mbar_arrive_expect_tx(full_kv, 2 * C::kTile);
+      load_tile<D>(smem, &p.tmK[map_idx], full_kv, p, c, g_kv, kt * kTileN, b);
+      load_tile<D>(smem + C::kTile, &p.tmV[map_idx], full_kv, p, c, g_kv, kt * kTileN, b);
+    }
+    for (int s = 0; s < n_steps; ++s) {
+      const int st = s % S_;
+      const uint32_t ph = (uint32_t)(s / S_) & 1u;
+      const int qt = qr.kv_begin + s / grp;
+      const int h = g_kv * grp + s % grp;
+      if (s >= S_ && !mbar_wait(&empty[st], ph ^ 1u, p.err, abort_flag)) break;
+      if (lane == 0) {
+        uint8_t* qb = smem + C::kRing + st * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[st], 2 * C::kTile);
+        load_tile<D>(qb, &p.tmQ[map_idx], &full[st], p, c, h, qt * kTileM, b);
+        load_tile<D>(qb + C::kTile, &p.tmDO[map_idx], &full[st], p, c, h, qt * kTileM, b);
+      }
+      // lse (log2 units) and Delta of the tile's 128 query rows; rows past the
+      // class end get lse = +inf (P = 0)
+      float* vl = vec + st * 2 * kTileM;
+      for (int e = lane; e < kTileM; e += 32) {
+        const int m = qt * kTileM + e;
+        float l2 = INFINITY, dl = 0.f;
+        if (m < Mv) {
+          const size_t li = ((size_t)b * p.H + h) * p.N + phys_row(geo, c, m);
+          l2 = __ldg(p.lse + li) * kLog2e;
+          dl = p.delta[li];
+        }
+        vl[e] = l2;
+        vl[kTileM + e] = dl;
+      }
+      mbar_arrive(&full[st]);
+    }
+  } else if (warp == 1) {
+    // ============================== MMA issuer ==============================
+    if (lane == 0 && n_steps > 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(kTileN, kTileM, 0, 0);
+      const uint32_t idesc_o = idesc_bf16_f32(kTileN, D, 0, 1);
+      const uint64_t dk_ = sdesc_sw128(k_addr, 16, 1024);                 // K, K-major (A)
+      const uint64_t dv_ = sdesc_sw128(v_addr, 16, 1024);                 // V, K-major (A)
+      const uint64_t dq0 = sdesc_sw128(ring_addr, 16, 1024);              // Q, K-major (B)
+      const uint64_t ddo0 = sdesc_sw128(ring_addr + C::kTile, 16, 1024);  // dO, K-major (B)
+      const uint64_t dqmn0 = sdesc_sw128(ring_addr, kChunkB, 1024);       // Q, MN-major (B)
+      const uint64_t ddomn0 = sdesc_sw128(ring_addr + C::kTile, kChunkB, 1024);
+      constexpr uint64_t kStageStep = C::kStageBytes >> 4;
+      const uint32_t t_dv = tmem + 256u, t_dk = tmem + 256u + (uint32_t)D;
+      bool ok = mbar_wait(full_kv, 0, p.err, abort_flag);
+      for (int s = 0; ok && s < n_steps; ++s) {
+        const int st = s % S_;
+        const uint32_t ph = (uint32_t)(s / S_) & 1u;
+        if (!mbar_wait(&full[st], ph, p.err, abort_flag)) break;
+        tc_fence_after();
+        const uint64_t sq = (uint64_t)st * kStageStep;
+        // S^T = K Q^T and dP^T = V dO^T (the previous step's dV / dK MMAs,
+        // issued before, have read P^T and dS^T)
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_ss(tmem, dk_ + kmajor_off(k), dq0 + sq + kmajor_off(k), idesc_s, k > 0 ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          mma_ss(tmem + 128u, dv_ + kmajor_off(k), ddo0 + sq + kmajor_off(k), idesc_s,
+                 k > 0 ? 1u : 0u);
+        tc_commit(st_full);
+        // dV += P^T dO, dK += dS^T Q
+        if (!mbar_wait(pt_full, (uint32_t)s & 1u, p.err, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < kTileM / 16; ++k)
+          mma_ts(t_dv, tmem + 8u * k, ddomn0 + sq + (uint64_t)((k * 2048) >> 4), idesc_o,
+                 (s > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < kTileM / 16; ++k)
+          mma_ts(t_dk, tmem + 128u + 8u * k, dqmn0 + sq + (uint64_t)((k * 2048) >> 4), idesc_o,
+                 (s > 0 || k > 0) ? 1u : 0u);
+        tc_commit(&empty[st]);
+      }
+      tc_commit(done);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ============================== compute ==============================
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off;
+    const uint32_t tP = tmem + 128u + lane_off;
+    const int j_v = kt * kTileN + r;  // this thread's key row (virtual)
+    const bool key_valid = j_v < Mv;
+    // query rows that see this key
+    int qlo = query_lo(geo, j_v), qhi = query_hi(geo, j_v, Mv);
+    qhi = qhi > Mv - 1 ? Mv - 1 : qhi;
+    int int_lo, int_hi;
+    interior_qtiles_keys(geo, Mv, kt * kTileN, &int_lo, &int_hi);
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int s = 0; s < n_steps; ++s) {
+      const int st = s % S_;
+      const int qt = qr.kv_begin + s / grp;
+      const bool edge = !(qt >= int_lo && qt <= int_hi);
+      const bool w = mbar_wait(st_full, (uint32_t)s & 1u, p.err, abort_flag);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* vl = vec + st * 2 * kTileM;
+#pragma unroll 1
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t sv[32], dpv[32];
+        tmem_ld32(tS + 32 * ch, sv);
+        tmem_ld32(tP + 32 * ch, dpv);
+        tmem_wait_ld();
+        const int i0 = qt * kTileM + 32 * ch;
+        uint32_t pp[16], pd[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = 32 * ch + 2 * e;
+          const float2 l2 = *reinterpret_cast<const float2*>(vl + c0);
+          const float2 dl = *reinterpret_cast<const float2*>(vl + kTileM + c0);
+          float2 xs = fma2(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
+                           make_float2(sl2, sl2), make_float2(-l2.x, -l2.y));
+          if (edge) {
+            if (!(i0 + 2 * e >= qlo && i0 + 2 * e <= qhi)) xs.x = -INFINITY;
+            if (!(i0 + 2 * e + 1 >= qlo && i0 + 2 * e + 1 <= qhi)) xs.y = -INFINITY;
+          }
+          const float2 pr = exp2_pair(xs, (e & 1) != 0 && !edge);
+          const float2 ds = make_float2(pr.x * (__uint_as_float(dpv[2 * e]) - dl.x),
+                                        pr.y * (__uint_as_float(dpv[2 * e + 1]) - dl.y));
+          pp[e] = pack_bf16x2(pr.x, pr.y);
+          pd[e] = pack_bf16x2(ds.x, ds.y);
+        }
+        // P^T / dS^T of query columns [32 ch, 32 ch + 32) over the first
+        // half of S^T's / dP^T's columns (already read)
+        tmem_st16(tS + 16 * ch, pp);
+        tmem_st16(tP + 16 * ch, pd);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(pt_full);
+    }
+    bool fin = ok && n_steps > 0 && mbar_wait(done, 0, p.err, abort_flag);
+    if (__all_sync(0xffffffffu, fin)) {
+      tc_fence_after();
+      const size_t row = ((size_t)b * p.N + phys_row(geo, c, j_v)) * p.Hkv + g_kv;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK (scaled)
+        uint16_t* orow = (which ? p.dk : p.dv) + row * D;
+        const float f = which ? p.scale : 1.f;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) {
+          uint32_t v[32];
+          tmem_ld32(tmem + 256u + (uint32_t)(which * D) + lane_off + 32 * j, v);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * f, __uint_as_float(v[2 * e + 1]) * f);
+          if (key_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + j * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+      }
+    } else if (key_valid && n_steps == 0) {
+      const size_t row = ((size_t)b * p.N + phys_row(geo, c, j_v)) * p.Hkv + g_kv;
+      uint4* a = reinterpret_cast<uint4*>(p.dk + row * D);
+      uint4* v = reinterpret_cast<uint4*>(p.dv + row * D);
+      for (int e = 0; e < D / 8; ++e) a[e] = v[e] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+
+  if (warp == 1 && lane == 0 && n_steps > 0 && *abort_flag) {
+    volatile int no_abort = 0;
+    mbar_wait(done, 0, nullptr, &no_abort, 100000000ull);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D>
+int launch_bwd_tc_impl(const void* q, const void* k, const void* v, const void* out,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                       float* delta, int B, int H, int Hkv, int N, int L, int R, int d, int bs,
+                       float scale, cudaStream_t stream) {
+  using C = BCfg<D>;
+  static std::atomic<unsigned long long> attr_dq{0}, attr_dkdv{0};
+  if (!smem_attr_once(reinterpret_cast<const void*>(swa_bwd_dq_kernel<D>), C::kAlloc, attr_dq) ||
+      !smem_attr_once(reinterpret_cast<const void*>(swa_bwd_dkdv_kernel<D>), C::kAlloc,
+                      attr_dkdv))
+    return SWA_ERR_CUDA;
+  int* err = device_error_word();
+  if (!err) return SWA_ERR_CUDA;
+  const Geometry geo = make_geometry(N, L, R, d, bs);
+  const bool block_mode = geo.bs > 1;
+  // two passes over the class chunks: every Delta is written (dq kernel)
+  // before any is read (dkdv kernel)
+  for (int pass = 0; pass < 2; ++pass) {
+    for (int c0 = 0; c0 < geo.nclass; c0 += kMaxClassesB) {
+      BwdTcParams p;
+      std::memset(&p, 0, sizeof(p));
+      p.nclass = geo.nclass - c0 < kMaxClassesB ? geo.nclass - c0 : kMaxClassesB;
+      p.class0 = c0;
+      p.out = static_cast<const uint16_t*>(out);
+      p.dout = static_cast<const uint16_t*>(dout);
+      p.lse = lse;
+      p.delta = delta;
+      p.dq = static_cast<uint16_t*>(dq);
+      p.dk = static_cast<uint16_t*>(dk);
+      p.dv = static_cast<uint16_t*>(dv);
+      p.err = err;
+      p.B = B;
+      p.H = H;
+      p.Hkv = Hkv;
+      p.N = N;
+      p.grp = H / Hkv;
+      p.L = L;
+      p.R = R;
+      p.d = d;
+      p.bs = geo.bs;
+      p.scale = scale;
+      p.scale_log2 = scale * kLog2e;
+      p.tile_prefix[0] = 0;
+      for (int cl = 0; cl < p.nclass; ++cl) {
+        p.Mv[cl] = class_valid_rows(geo, c0 + cl);
+        p.tile_prefix[cl + 1] = p.tile_prefix[cl] + (p.Mv[cl] + kTileM - 1) / kTileM;
+      }
+      const uint32_t box[4] = {64, 1, (uint32_t)kBlockRows, 1};
+      const int nmaps = block_mode ? 1 : p.nclass;
+      for (int cl = 0; cl < nmaps; ++cl) {
+        const int cc = c0 + cl;
+        const uint64_t rows = block_mode ? (uint64_t)N : (uint64_t)class_rows(geo, cc);
+        const uint64_t rstep = block_mode ? 1 : (uint64_t)d;
+        const size_t qoff = block_mode ? 0 : (size_t)cc * H * D;
+        const size_t kvoff = block_mode ? 0 : (size_t)cc * Hkv * D;
+        const uint64_t dq_[4] = {(uint64_t)D, (uint64_t)H, rows, (uint64_t)B};
+        const uint64_t sq[3] = {(uint64_t)D * 2, rstep * H * D * 2, (uint64_t)N * H * D * 2};
+        const uint64_t dk_[4] = {(uint64_t)D, (uint64_t)Hkv, rows, (uint64_t)B};
+        const uint64_t sk[3] = {(uint64_t)D * 2, rstep * Hkv * D * 2,
+                                (uint64_t)N * Hkv * D * 2};
+        void* qb = (void*)(static_cast<const uint16_t*>(q) + qoff);
+        void* db = (void*)(static_cast<const uint16_t*>(dout) + qoff);
+        void* kb = (void*)(static_cast<const uint16_t*>(k) + kvoff);
+        void* vb = (void*)(static_cast<const uint16_t*>(v) + kvoff);
+        if (encode_tiled(&p.tmQ[cl], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, qb, dq_, sq, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+            encode_tiled(&p.tmDO[cl], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, db, dq_, sq, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+            encode_tiled(&p.tmK[cl], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, kb, dk_, sk, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+            encode_tiled(&p.tmV[cl], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, vb, dk_, sk, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+          return SWA_ERR_CUDA;
+      }
+      const long ntiles = (long)p.tile_prefix[p.nclass];
+      if (pass == 0) {
+        const long grid = ntiles * B * H;
+        if (grid <= 0) continue;
+        if (grid > 0x7fffffffL) return SWA_ERR_UNSUPPORTED;
+        swa_bwd_dq_kernel<D><<<(unsigned)grid, kThreadsB, C::kAlloc, stream>>>(p);
+      } else {
+        const long grid = ntiles * B * Hkv;
+        if (grid <= 0) continue;
+        if (grid > 0x7fffffffL) return SWA_ERR_UNSUPPORTED;
+        swa_bwd_dkdv_kernel<D><<<(unsigned)grid, kThreadsB, C::kAlloc, stream>>>(p);
+      }
+      if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
+    }
+  }
+  return SWA_OK;
+}
+
+}  // namespace
+
+int launch_backward_tc(const void* q, const void* k, const void* v, const void* out,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                       float* delta, int B, int H, int Hkv, int N, int D, int L, int R, int d,
+                       int bs, float scale, cudaStream_t stream) {
+  if (D == 128)
+    return launch_bwd_tc_impl<128>(q, k, v, out, dout, lse, dq, dk, dv, delta, B, H, Hkv, N, L,
+                                   R, d, bs, scale, stream);
+  if (D == 64)
+    return launch_bwd_tc_impl<64>(q, k, v, out, dout, lse, dq, dk, dv, delta, B, H, Hkv, N, L, R,
+                                  d, bs, scale, stream);
+  return SWA_ERR_UNSUPPORTED;
+}
+
+}  // namespace swa

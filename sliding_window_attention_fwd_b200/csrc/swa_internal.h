@@ -78,5 +78,11 @@ int launch_backward(const void* q, const void* k, const void* v, const void* out
                     int H, int Hkv, int N, int D, int L, int R, int d, int bs, const int32_t* G,
                     int ng, float scale, cudaStream_t stream);
 void release_backward_workspace();
+// Tensor-core backward of band problems (no global tokens): dq kernel then
+// dk / dv kernel; delta is a [B, H, N] fp32 workspace.
+int launch_backward_tc(const void* q, const void* k, const void* v, const void* out,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                       float* delta, int B, int H, int Hkv, int N, int D, int L, int R, int d,
+                       int bs, float scale, cudaStream_t stream);
 
 }  // namespace swa

@@ -103,6 +103,22 @@ SWA_HD int key_hi(const Geometry& g, int m, int Mv) {
   return m + g.R;
 }
 
+// First and last query row (virtual rows of the class, before clipping to
+// [0, Mv-1]) whose key interval [key_lo, key_hi] contains key row j: the
+// transpose of key_lo / key_hi (both are monotone in the row, so the rows
+// that see a key form one interval).  The backward walks it key-stationary.
+SWA_HD int query_lo(const Geometry& g, int j) {
+  if (g.R < 0) return 0;
+  if (g.R == 0) return j;
+  if (g.bs) return (j / g.bs - g.R / g.bs) * g.bs;
+  return j - g.R;
+}
+SWA_HD int query_hi(const Geometry& g, int j, int Mv) {
+  if (g.L < 0) return Mv - 1;
+  if (g.bs) return (j / g.bs + g.L / g.bs + 1) * g.bs - 1;
+  return j + g.L;
+}
+
 struct TileRange {
   int kv_begin, kv_end;  // kv tiles [begin, end) of the class
 };
@@ -150,6 +166,37 @@ SWA_HD void interior_tiles_rows(const Geometry& g, int Mv, int m0, int* lo, int*
 // The same for query tile qt of a class with Mv valid rows.
 SWA_HD void interior_tiles(const Geometry& g, int Mv, int qt, int* lo, int* hi) {
   interior_tiles_rows(g, Mv, qt * kTileM, lo, hi);
+}
+
+// Query tiles that see any key of the 128 key rows [j0, j0 + 127] of a
+// class with Mv valid rows (the key-stationary walk of the backward).
+SWA_HD TileRange qtile_range_keys(const Geometry& g, int Mv, int j0) {
+  int j1 = j0 + kTileN - 1;
+  if (j1 > Mv - 1) j1 = Mv - 1;
+  int lo = query_lo(g, j0);
+  if (lo < 0) lo = 0;
+  int hi = query_hi(g, j1, Mv);
+  if (hi > Mv - 1) hi = Mv - 1;
+  TileRange r;
+  r.kv_begin = lo / kTileM;
+  r.kv_end = hi / kTileM + 1;
+  if (r.kv_end < r.kv_begin) r.kv_end = r.kv_begin;
+  return r;
+}
+
+// Query tiles [*lo, *hi] in which every (query, key) pair with a key of
+// [j0, j0 + 127] is inside the window and in range (no element mask).
+SWA_HD void interior_qtiles_keys(const Geometry& g, int Mv, int j0, int* lo, int* hi) {
+  const int j1 = j0 + kTileN - 1;
+  *lo = 1;
+  *hi = 0;
+  if (j1 > Mv - 1) return;
+  int a = query_lo(g, j1);
+  if (a < 0) a = 0;
+  int b = query_hi(g, j0, Mv);
+  if (b > Mv - 1) b = Mv - 1;
+  *lo = (a + kTileM - 1) / kTileM;
+  *hi = (b + 1) / kTileM - 1;
 }
 
 }  // namespace swa

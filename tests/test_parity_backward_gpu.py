@@ -40,6 +40,14 @@ def rel_check(got, ref, what):
     (1, 320, 2, 1, 64, 128, 128, 2, 64, None),
     (1, 300, 4, 4, 128, 50, 50, 1, 0, [0, 150]),
     (1, 200, 8, 1, 128, -1, 0, 1, 0, None),
+    # band problems run on the tensor-core kernels: several query and key
+    # tiles, ragged tails, every window kind
+    (1, 1000, 8, 2, 128, 300, 0, 1, 0, None),    # causal, GQA 4, ragged
+    (2, 700, 4, 4, 64, 100, 100, 1, 0, None),    # bidirectional, D = 64
+    (1, 1100, 4, 1, 64, 90, 90, 3, 0, None),     # token dilation 3, GQA 4
+    (1, 900, 2, 2, 128, 200, 0, 2, 64, None),    # block dilation, causal
+    (1, 129, 2, 1, 128, -1, -1, 1, 0, None),     # full bidirectional, tile + 1
+    (1, 2048, 8, 2, 128, 600, 0, 1, 0, None),    # many interior tiles
 ])
 def test_backward_matches_oracle(swa, B, N, H, Hkv, D, L, R, d, bs, G):
     seed = N + H + D
@@ -75,3 +83,30 @@ def test_backward_twice_gives_identical_results(swa):
     b = swa.swa_backward(q, k, v, out, do, lse, 100, 0)
     for x, y in zip(a, b):
         assert (x.float() - y.float()).abs().max().item() <= 1e-2 * x.float().abs().max().item()
+
+
+def test_backward_full_size_properties(swa):
+    """Mistral-shaped prefill (B1 N8192 H32/8 D128, causal W=4096): closed
+    forms that hold at any size.  Softmax is shift invariant, so every row's
+    dS sums to zero and sum_j dK_j = 0 per (batch, kv head); every row's P
+    sums to one, so sum_j dV_j = sum over the group's heads of sum_i dO_i.
+    Both are compared against the scale of the summed terms (bf16 rounding
+    of each row of dK / dV)."""
+    cfg = inputs.CONFIGS["mistral_causal_prefill"]
+    q, k, v, _ = inputs.forward_inputs(cfg, device="cuda")
+    do = inputs.normal((cfg.B, cfg.N, cfg.H, cfg.D), cfg.seed, 9, torch.bfloat16, "cuda")
+    lse = torch.empty(cfg.B, cfg.H, cfg.N, device="cuda")
+    out = swa.swa_forward(q, k, v, None, lse, cfg.win_left, cfg.win_right)
+    dq, dk, dv = swa.swa_backward(q, k, v, out, do, lse, cfg.win_left, cfg.win_right)
+    torch.cuda.synchronize()
+    assert swa.swa_device_error() == 0
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t.float()).all()
+    grp = cfg.H // cfg.Hkv
+    sum_do = do.float().view(cfg.B, cfg.N, cfg.Hkv, grp, cfg.D).sum(dim=(1, 3))
+    sum_dv = dv.float().sum(1)
+    tol_v = 2e-2 * dv.float().abs().amax() * cfg.N ** 0.5 + 1e-3 * sum_do.abs().amax()
+    assert (sum_dv - sum_do).abs().max().item() <= tol_v.item()
+    sum_dk = dk.float().sum(1)
+    tol_k = 2e-2 * dk.float().abs().amax() * cfg.N ** 0.5
+    assert sum_dk.abs().max().item() <= tol_k.item()
