@@ -381,6 +381,31 @@ SWA_API int swa_schedule(int N, int win_left, int win_right, int dilation,
    has one, after synchronising that device; later calls allocate again. */
 SWA_API int swa_release(void);
 
+/*
+ * Caller-provided allocator for the library-owned workspaces (no
+ * counterpart on the method's pages: a deployment hook).  alloc(bytes, user)
+ * must return `bytes` of device memory on the calling thread's current
+ * device (16-byte aligned) or NULL; free_fn(ptr, user) gives back a block
+ * alloc returned.  Both are called with the device current, from inside
+ * library calls, on the calling thread, under a library lock (they must not
+ * call back into the library).  A serving engine routes the workspaces
+ * through its own memory pool this way.
+ */
+typedef void* (*swa_alloc_fn)(size_t bytes, void* user);
+typedef void (*swa_free_fn)(void* ptr, void* user);
+
+/*
+ * swa_set_workspace_allocator -- every later workspace allocation and free
+ * goes through alloc / free_fn (both NULL: back to cudaMalloc / cudaFree).
+ * The workspaces that exist are released first, through the allocator that
+ * made them (as swa_release does).  A NULL alloc with a non-NULL free_fn, or
+ * the other way round, is SWA_ERR_ARG.  When alloc returns NULL the call
+ * that needed the memory returns SWA_ERR_NOMEM and launches nothing.  Call
+ * it while no other library call is in progress; alloc, free_fn and user
+ * must stay valid until the allocator is replaced.
+ */
+SWA_API int swa_set_workspace_allocator(swa_alloc_fn alloc, swa_free_fn free_fn, void* user);
+
 /* swa_status_string -- static text for a status code. */
 SWA_API const char* swa_status_string(int status);
 

@@ -33,6 +33,7 @@ _EXPORTS = (
     "swa_release",
     "swa_schedule",
     "swa_selftest_timeout",
+    "swa_set_workspace_allocator",
     "swa_status_string",
     "swa_version",
 )

@@ -61,6 +61,10 @@ _lib.swa_backward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I
 _lib.swa_device_error.argtypes = [_P]
 _lib.swa_selftest_timeout.argtypes = [_I, _P]
 _lib.swa_schedule.argtypes = [_I, _I, _I, _I, _I, _P, _I]
+_ALLOC_FN = ctypes.CFUNCTYPE(ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p)
+_FREE_FN = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_void_p)
+_lib.swa_set_workspace_allocator.argtypes = [_ALLOC_FN, _FREE_FN, _P]
+_lib.swa_set_workspace_allocator.restype = _I
 _lib.swa_release.argtypes = []
 _lib.swa_status_string.argtypes = [_I]
 _lib.swa_status_string.restype = ctypes.c_char_p
@@ -411,3 +415,38 @@ def swa_schedule(N, win_left, win_right, dilation=1, dilation_block=0):
 
 def swa_release() -> None:
     _check(_lib.swa_release(), "swa_release")
+
+
+_allocator_keep = None  # the installed callbacks must outlive every library call
+
+
+def swa_set_workspace_allocator(alloc=None, free=None) -> None:
+    """Routes the library-owned workspaces through the caller's allocator
+    (C: swa_set_workspace_allocator): alloc(nbytes) -> device pointer as an
+    int (0 when out of memory), free(ptr).  No arguments: back to cudaMalloc
+    / cudaFree.  Existing workspaces are released first."""
+    global _allocator_keep
+    if (alloc is None) != (free is None):
+        raise ValueError("give both alloc and free, or neither")
+    if alloc is None:
+        _check(_lib.swa_set_workspace_allocator(_ALLOC_FN(), _FREE_FN(), None),
+               "swa_set_workspace_allocator")
+        _allocator_keep = None
+        return
+
+    def _a(nbytes, _user):
+        try:
+            return int(alloc(int(nbytes)) or 0) or None
+        except Exception:  # an allocator error is an allocation failure
+            return None
+
+    def _f(ptr, _user):
+        try:
+            free(int(ptr))
+        except Exception:
+            pass
+
+    keep = (_ALLOC_FN(_a), _FREE_FN(_f))
+    _check(_lib.swa_set_workspace_allocator(keep[0], keep[1], None),
+           "swa_set_workspace_allocator")
+    _allocator_keep = keep

@@ -321,12 +321,12 @@ float* bwd_workspace(size_t bytes, cudaStream_t stream) {
   if (g_bwd_bytes[dev] < bytes) {
     if (g_bwd_ws[dev]) {
       cudaStreamSynchronize(stream);
-      cudaFree(g_bwd_ws[dev]);
+      ws_free(g_bwd_ws[dev]);
       g_bwd_ws[dev] = nullptr;
       g_bwd_bytes[dev] = 0;
     }
-    void* ptr = nullptr;
-    if (cudaMalloc(&ptr, bytes) != cudaSuccess) return nullptr;
+    void* ptr = ws_alloc(bytes);
+    if (!ptr) return nullptr;
     g_bwd_ws[dev] = ptr;
     g_bwd_bytes[dev] = bytes;
   }
@@ -415,7 +415,7 @@ void release_backward_workspace() {
     cudaGetDevice(&cur);
     cudaSetDevice(dv);
     cudaDeviceSynchronize();
-    cudaFree(g_bwd_ws[dv]);
+    ws_free(g_bwd_ws[dv]);
     cudaSetDevice(cur);
     g_bwd_ws[dv] = nullptr;
     g_bwd_bytes[dv] = 0;

@@ -196,6 +196,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       mbar_arrive_expect_tx(full_q, 2 * C::kTile);
       load_tile<D>(smem, &p.tmQ[map_idx], full_q, p, c, h, qt * kTileM, b);
       load_tile<D>(smem + C::kTile, &p.tmDO[map_idx], full_q, p, c, h, qt * kTileM, b);
+      int last_k = -1, last_v = -1;
       for (int it = 0; it < n_tiles; ++it) {
         const int st = it % S_;
         const uint32_t ph = (uint32_t)(it / S_) & 1u;
@@ -204,9 +205,16 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         if (it >= S_ && !mbar_wait(&empty_k[st], ph ^ 1u, p.err, abort_flag)) break;
         mbar_arrive_expect_tx(&full_k[st], C::kTile);
         load_tile<D>(kb, &p.tmK[map_idx], &full_k[st], p, c, g_kv, t * kTileN, b);
+        last_k = it;
         if (it >= S_ && !mbar_wait(&empty_v[st], ph ^ 1u, p.err, abort_flag)) break;
         mbar_arrive_expect_tx(&full_v[st], C::kTile);
         load_tile<D>(kb + C::kTile, &p.tmV[map_idx], &full_v[st], p, c, g_kv, t * kTileN, b);
+        last_v = it;
+      }
+      if (*abort_flag) {  // leave no copy writing shared memory behind
+        drain_copies(full_q, 1, 0, 0);
+        drain_copies(full_k, S_, 0, last_k);
+        drain_copies(full_v, S_, 0, last_v);
       }
     }
   } else if (warp == 1) {
@@ -453,6 +461,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       load_tile<D>(smem, &p.tmK[map_idx], full_kv, p, c, g_kv, kt * kTileN, b);
       load_tile<D>(smem + C::kTile, &p.tmV[map_idx], full_kv, p, c, g_kv, kt * kTileN, b);
     }
+    int last = -1;
     for (int s = 0; s < n_steps; ++s) {
       const int st = s % S_;
       const uint32_t ph = (uint32_t)(s / S_) & 1u;
@@ -480,6 +489,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         vl[kTileM + e] = dl;
       }
       mbar_arrive(&full[st]);
+      last = s;
+    }
+    if (lane == 0 && *abort_flag) {  // leave no copy writing shared memory behind
+      drain_copies(full_kv, 1, 0, 0);
+      drain_copies(full, S_, 0, last);
     }
   } else if (warp == 1) {
     // ============================== MMA issuer ==============================

@@ -88,6 +88,39 @@ CUresult encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, int rank, voi
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+namespace {
+std::mutex g_alloc_mu;
+swa_alloc_fn g_alloc = nullptr;
+swa_free_fn g_free = nullptr;
+void* g_alloc_user = nullptr;
+}  // namespace
+
+void* ws_alloc(size_t bytes) {
+  std::lock_guard<std::mutex> lk(g_alloc_mu);
+  if (g_alloc) return g_alloc(bytes, g_alloc_user);
+  void* p = nullptr;
+  return cudaMalloc(&p, bytes) == cudaSuccess ? p : nullptr;
+}
+
+void ws_free(void* ptr) {
+  if (!ptr) return;
+  std::lock_guard<std::mutex> lk(g_alloc_mu);
+  if (g_free) g_free(ptr, g_alloc_user);
+  else cudaFree(ptr);
+}
+
+int set_workspace_allocator(swa_alloc_fn alloc, swa_free_fn free_fn, void* user) {
+  if ((alloc == nullptr) != (free_fn == nullptr)) return SWA_ERR_ARG;
+  // blocks of the old allocator go back to it before the switch
+  release_workspaces();
+  release_backward_workspace();
+  std::lock_guard<std::mutex> lk(g_alloc_mu);
+  g_alloc = alloc;
+  g_free = free_fn;
+  g_alloc_user = user;
+  return SWA_OK;
+}
+
 int launch_timeout_selftest(int limit_us, cudaStream_t stream) {
   int* err = device_error_word();
   if (!err) return SWA_ERR_CUDA;
@@ -404,6 +437,10 @@ SWA_API int swa_schedule(int N, int win_left, int win_right, int dilation, int d
     }
   }
   return n;
+}
+
+SWA_API int swa_set_workspace_allocator(swa_alloc_fn alloc, swa_free_fn free_fn, void* user) {
+  return set_workspace_allocator(alloc, free_fn, user);
 }
 
 SWA_API int swa_release(void) {

@@ -297,6 +297,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
                           &p.tmQ[map_idx], full_q, cc * 64, head[s],
                           box_row(qt * kTileM + hh * 64), b);
       }
+      int last_k = -1, last_v = -1;  // last tiles whose loads were issued
       for (int it = 0; it < n_tiles; ++it) {
         const int st = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
@@ -305,6 +306,12 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
           uint64_t* ful = kv ? &full_v[st] : &full_k[st];
           uint8_t* dst = smem + C::kRing + st * C::kStageBytes + kv * NSTREAM * C::kTile;
           if (it >= kStages && !mbar_wait(emp, ph ^ 1u, p.err, abort_flag)) goto producer_done;
+          (kv ? last_v : last_k) = it;
+#ifdef SWA_TEST_WITHHOLD_TILE
+          // failure-detection test build only: this K tile is never loaded,
+          // so the MMA issuer's bounded wait for it runs out
+          if (kv == 0 && it == SWA_TEST_WITHHOLD_TILE) continue;
+#endif
           if (!glob || it < n_band) {
             if (lane == 0) {
               const CUtensorMap* m = kv ? mapV : mapK;
@@ -347,7 +354,18 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
           }
         }
       }
-    producer_done:;
+    producer_done:
+      if (lane == 0 && *abort_flag) {
+        // leave no copy writing shared memory behind
+#ifdef SWA_TEST_WITHHOLD_TILE
+        const int skip = SWA_TEST_WITHHOLD_TILE;
+#else
+        const int skip = -1;
+#endif
+        drain_copies(full_q, 1, 0, 0);
+        drain_copies(full_k, kStages, 0, last_k, skip);
+        drain_copies(full_v, kStages, 0, last_v);
+      }
     } else if (warp <= NSLOT) {
       // =========================== MMA issuers ===========================
       // Warp 1 + s issues the MMAs of slot s (lane 0; the rest of the warp

@@ -30,6 +30,12 @@ inline bool smem_attr_once(const void* kernel, int bytes, std::atomic<unsigned l
 // Device error word of the current device (bounded waits write into it).
 int* device_error_word();
 
+// Device memory of the library-owned workspaces, on the current device:
+// through the caller's allocator when one is set (swa_set_workspace_allocator),
+// else cudaMalloc / cudaFree.  ws_alloc returns nullptr on failure.
+void* ws_alloc(size_t bytes);
+void ws_free(void* ptr);
+
 // Encodes a tiled tensor map through the driver entry point (no -lcuda).
 CUresult encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, int rank, void* base,
                       const uint64_t* dims, const uint64_t* strides_bytes,

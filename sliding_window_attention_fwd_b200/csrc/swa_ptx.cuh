@@ -16,8 +16,14 @@ enum DeviceError : int {
 };
 
 // Default bound on any single device-side wait: 2 seconds.  Legitimate
-// waits in these kernels last microseconds.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// waits in these kernels last microseconds.  (A failure-detection test
+// build lowers it to a few milliseconds.)
+#ifndef SWA_WAIT_LIMIT_NS
+#define SWA_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = SWA_WAIT_LIMIT_NS;
+// Bound on the waits of an abort path (in-flight copies, MMAs).
+constexpr uint64_t kDrainLimitNs = 100000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -79,6 +85,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
       }
     }
   }
+}
+
+// Abort path of a producer: waits, with its own limit and whatever the abort
+// flag says, until the bulk copies it issued into tiles first..last of a ring
+// of `stages` barriers (tile t -> bars[t % stages], phase parity
+// (t / stages) & 1) have landed, so that none still writes shared memory
+// when the CTA exits.  Only the last `stages` tiles can be outstanding;
+// `skip` names a tile whose copy was never issued (or -1).
+__device__ __forceinline__ void drain_copies(uint64_t* bars, int stages, int first, int last,
+                                             int skip = -1) {
+  volatile int no_abort = 0;
+  for (int t = (last - stages + 1 > first ? last - stages + 1 : first); t <= last; ++t)
+    if (t != skip)
+      mbar_wait(&bars[t % stages], (uint32_t)(t / stages) & 1u, nullptr, &no_abort,
+                kDrainLimitNs);
 }
 
 // ------------------------------------------------------------------ TMA
@@ -285,8 +306,9 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
 // degree-3 polynomial fitted by iterated weighted least squares to minimise
 // the relative error on [-1/2, 1/2] (max relative error 7.6e-5); 2^n is
 // applied by adding n to the exponent field.  Inputs below -125 are clamped
-// to -125, so the result is >= 2^-125 (never denormal, never 0): callers use
-// it only where such a value is negligible against a sum >= 1.
+// to -125, so the result is 2^-125 within that error (never denormal, never
+// 0): callers use it only where such a value is negligible against a sum
+// >= 1.
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   constexpr float kC0 = 0.99992823600769043f, kC1 = 0.69326096773147583f,
                   kC2 = 0.24260851740837097f, kC3 = 0.05517049878835678f;

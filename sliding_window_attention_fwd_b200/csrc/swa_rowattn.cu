@@ -242,11 +242,21 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
         prefetch_tensormap(&p.tmKn);
         prefetch_tensormap(&p.tmVn);
       }
+      int last = -1;  // last stage whose loads were issued
+#ifdef SWA_TEST_WITHHOLD_TILE
+      const int skip = SWA_TEST_WITHHOLD_TILE;
+#else
+      const int skip = -1;
+#endif
       for (int k = 0; k < n_stages; ++k) {
         const int st = k % kStagesR;
         if (k >= kStagesR &&
             !mbar_wait(&empty[st], ((uint32_t)(k / kStagesR) & 1u) ^ 1u, p.err, abort_flag))
           break;
+        last = k;
+        // failure-detection test build only: these 64 rows are never loaded,
+        // so the compute warps' bounded wait for them runs out
+        if (k == skip) continue;
         uint8_t* kb = smem + st * S::kStage;
         uint8_t* vb = kb + S::kTile;
         // source of the 64 key rows [idx0, idx0 + 64): a row of the ring /
@@ -278,6 +288,8 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
           tma_load_4d(vb + cc * (kRows * 128), mv, &full[st], cc * 64, g, row, bc);
         }
       }
+      // leave no copy writing shared memory behind
+      if (*abort_flag) drain_copies(full, kStagesR, 0, last, skip);
     }
   } else {
     // ============================ compute ============================
@@ -563,14 +575,14 @@ bool get_workspace(int which, size_t cnt_bytes, size_t part_bytes, cudaStream_t 
   if (w.cnt_bytes < cnt_bytes) {
     if (w.cnt) {
       cudaStreamSynchronize(stream);
-      cudaFree(w.cnt);
+      ws_free(w.cnt);
       w.cnt = nullptr;
       w.cnt_bytes = 0;
     }
-    void* p = nullptr;
-    if (cudaMalloc(&p, cnt_bytes) != cudaSuccess) return false;
+    void* p = ws_alloc(cnt_bytes);
+    if (!p) return false;
     if (cudaMemsetAsync(p, 0, cnt_bytes, stream) != cudaSuccess) {
-      cudaFree(p);
+      ws_free(p);
       return false;
     }
     w.cnt = p;
@@ -579,12 +591,12 @@ bool get_workspace(int which, size_t cnt_bytes, size_t part_bytes, cudaStream_t 
   if (w.part_bytes < part_bytes) {
     if (w.part) {
       cudaStreamSynchronize(stream);
-      cudaFree(w.part);
+      ws_free(w.part);
       w.part = nullptr;
       w.part_bytes = 0;
     }
-    void* p = nullptr;
-    if (cudaMalloc(&p, part_bytes) != cudaSuccess) return false;
+    void* p = ws_alloc(part_bytes);
+    if (!p) return false;
     w.part = p;
     w.part_bytes = part_bytes;
   }
@@ -882,8 +894,8 @@ void release_workspaces() {
       cudaGetDevice(&cur);
       cudaSetDevice(d);
       cudaDeviceSynchronize();
-      if (ws.cnt) cudaFree(ws.cnt);
-      if (ws.part) cudaFree(ws.part);
+      if (ws.cnt) ws_free(ws.cnt);
+      if (ws.part) ws_free(ws.part);
       cudaSetDevice(cur);
       ws = Workspace();
     }

@@ -43,3 +43,32 @@ def sample_rows(B, H, N, n, seed, extra_i=()):
     if extra:
         rows = np.concatenate([rows, np.array(extra)], 0)
     return rows.astype(np.int64)
+
+
+def build_test_library(out_dir, defines):
+    """Compiles libswa's sources with extra preprocessor definitions (a
+    test-only build, e.g. a failure-injection switch) into out_dir and
+    returns the path of the shared library.  Each source compiles in its own
+    nvcc process, in parallel."""
+    import glob
+    import os
+    import subprocess
+
+    from sliding_window_attention_fwd_b200 import build as b
+
+    flags = [f for f in b.NVCC_FLAGS if f != "-shared"]
+    objs, procs = [], []
+    for src in b.sources():
+        obj = os.path.join(out_dir, os.path.basename(src) + ".o")
+        objs.append(obj)
+        procs.append(subprocess.Popen(
+            ["nvcc", *flags, *(f"-D{d}" for d in defines), "-I", b.INCLUDE, "-I", b.CSRC, "-c",
+             src, "-o", obj], stdout=subprocess.PIPE, stderr=subprocess.STDOUT))
+    for pr in procs:
+        out, _ = pr.communicate()
+        assert pr.returncode == 0, out.decode()[-2000:]
+    lib = os.path.join(out_dir, "libswa_test.so")
+    subprocess.run(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", lib,
+                    *objs], check=True, capture_output=True)
+    assert glob.glob(lib)
+    return lib

@@ -231,3 +231,17 @@ def test_layers_validation_names_the_bad_layer():
     bad = ctypes.c_int(-7)
     assert L.swa_forward_layers(None, 0, 1, 4, 2, 64, 128, ctypes.byref(bad), None) == OK
     assert L.swa_forward_layers(None, 2, 1, 4, 2, 64, 128, ctypes.byref(bad), None) == ARG
+
+
+def test_workspace_allocator_arguments():
+    """Both callbacks or neither; restoring the default touches no GPU (no
+    workspace exists in this process)."""
+    from sliding_window_attention_fwd_b200 import binding as b
+    alloc = b._ALLOC_FN(lambda n, u: None)
+    free = b._FREE_FN(lambda p, u: None)
+    assert L.swa_set_workspace_allocator(alloc, b._FREE_FN(), None) == ARG
+    assert L.swa_set_workspace_allocator(b._ALLOC_FN(), free, None) == ARG
+    assert L.swa_set_workspace_allocator(b._ALLOC_FN(), b._FREE_FN(), None) == OK
+    with pytest.raises(ValueError):
+        swa.swa_set_workspace_allocator(lambda n: 0)
+    swa.swa_set_workspace_allocator()
