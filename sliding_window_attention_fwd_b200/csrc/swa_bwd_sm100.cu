@@ -29,8 +29,9 @@
 //        P^T, dS^T (bf16) in place   compute warps (one key row per thread)
 //        dV += P^T dO, dK += dS^T Q  tcgen05.mma (TMEM x smem)
 //    dK and dV stay in TMEM for the CTA's whole walk.
-// Warp roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer (and
-// TMEM owner), warps 4-7 compute.  Every wait is bounded (swa_ptx.cuh).
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM owner),
+// warps 4.. compute (kGroupsB warpgroups).  Every wait is bounded
+// (swa_ptx.cuh).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -48,7 +49,26 @@ namespace {
 constexpr int kMaxClassesB = 8;                 // residue classes per launch
 constexpr int kChunkB = kTileM * 128;           // 128 rows x 64 bf16 columns
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kThreadsB = 256;
+// Compute warpgroups: each takes 128 / kGroupsB of a step's 128 columns
+// (a TMEM lane quadrant belongs to one warp of every group), so several
+// warps per SM sub-partition hide each other's latencies.  Measured on the
+// Mistral-shaped backward: 1 group 3.12 ms, 2 groups 2.26, 4 groups 2.05.
+#ifndef SWA_BWD_GROUPS
+#define SWA_BWD_GROUPS 4
+#endif
+constexpr int kGroupsB = SWA_BWD_GROUPS;
+constexpr int kCpg = 4 / kGroupsB;  // 32-column chunks per group
+constexpr int kThreadsB = 128 * (1 + kGroupsB);
+static_assert(kGroupsB == 1 || kGroupsB == 2 || kGroupsB == 4, "1, 2 or 4 compute groups");
+
+// TMEM column (relative to the operand block) of the bf16 pairs of K-step k
+// (16 elements) of a P / dS operand written in place over fp32 scores: chunk
+// ch of 32 scores (group g = ch / kCpg, its i-th chunk) is packed into the 16
+// columns 32 kCpg g + 16 i, inside the group's own (already read) columns.
+__device__ __forceinline__ uint32_t pcol(int k) {
+  const int ch = k / 2, g = ch / kCpg, i = ch % kCpg;
+  return (uint32_t)(32 * kCpg * g + 16 * i + 8 * (k % 2));
+}
 
 struct BwdTcParams {
   CUtensorMap tmQ[kMaxClassesB];
@@ -170,7 +190,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(ds_full, 128);
+    mbar_init(ds_full, 128 * kGroupsB);
     mbar_init(done, 1);
     fence_mbar_init();
   }
@@ -256,7 +276,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         const uint64_t dkmn = dkmn0 + (uint64_t)st * kStageStep;
 #pragma unroll
         for (int k = 0; k < kTileN / 16; ++k)
-          mma_ts(tmem + 256u, tmem + 8u * k, dkmn + (uint64_t)((k * 2048) >> 4), idesc_dq,
+          mma_ts(tmem + 256u, tmem + pcol(k), dkmn + (uint64_t)((k * 2048) >> 4), idesc_dq,
                  (it > 0 || k > 0) ? 1u : 0u);
         tc_commit(&empty_k[st]);
       }
@@ -265,6 +285,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ============================== compute ==============================
+    // group cg takes the keys [32 kCpg cg, 32 kCpg (cg + 1)) of every step
+    const int cg = (warp - 4) / 4;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -301,7 +323,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       delta = acc0 + acc1;
       const size_t li = ((size_t)b * p.H + h) * p.N + i_phys;
       lse2 = __ldg(p.lse + li) * kLog2e;
-      p.delta[li] = delta;
+      if (cg == 0) p.delta[li] = delta;
     }
     bool ok = true;
     for (int it = 0; it < n_tiles; ++it) {
@@ -315,12 +337,14 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       }
       tc_fence_after();
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int i = 0; i < kCpg; ++i) {
+        const int ch = cg * kCpg + i;
         uint32_t sv[32], dpv[32];
         tmem_ld32(tS + 32 * ch, sv);
         tmem_ld32(tP + 32 * ch, dpv);
         tmem_wait_ld();
         const int n0 = t * kTileN + 32 * ch;
+        const float2 ndl = make_float2(-delta, -delta);
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -332,13 +356,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             if (!(j0 + 1 >= klo && j0 + 1 <= khi && j0 + 1 < Mv)) xs.y = -INFINITY;
           }
           const float2 pr = exp2_pair(xs, (e & 1) != 0 && !edge);
-          const float2 ds = make_float2(pr.x * (__uint_as_float(dpv[2 * e]) - delta),
-                                        pr.y * (__uint_as_float(dpv[2 * e + 1]) - delta));
+          const float2 ds = mul2(pr, add2(make_float2(__uint_as_float(dpv[2 * e]),
+                                                      __uint_as_float(dpv[2 * e + 1])), ndl));
           pk[e] = pack_bf16x2(ds.x, ds.y);
         }
-        // dS of keys [32 ch, 32 ch + 32) -> S columns [16 ch, 16 ch + 16)
-        // (already read: chunk ch / 2 <= ch)
-        tmem_st16(tS + 16 * ch, pk);
+        // dS of these 32 keys over the group's own (already read) S columns
+        tmem_st16(tS + 32 * kCpg * cg + 16 * i, pk);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -348,8 +371,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
       uint16_t* orow = p.dq + (((size_t)b * p.N + i_phys) * p.H + h) * D;
-#pragma unroll
-      for (int j = 0; j < D / 32; ++j) {
+      // the groups share the row's D / 32 column chunks
+#pragma unroll 1
+      for (int j = cg; j < D / 32; j += kGroupsB) {
         uint32_t v[32];
         tmem_ld32(tQ + 32 * j, v);
         tmem_wait_ld();
@@ -365,7 +389,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
         }
       }
-    } else if (row_valid && n_tiles == 0) {
+    } else if (row_valid && n_tiles == 0 && cg == 0) {
       // no key at all (cannot happen for a valid row: its own key is always
       // in the window), kept for completeness
       uint4* dst = reinterpret_cast<uint4*>(p.dq + (((size_t)b * p.N + i_phys) * p.H + h) * D);
@@ -434,7 +458,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(st_full, 1);
-    mbar_init(pt_full, 128);
+    mbar_init(pt_full, 128 * kGroupsB);
     mbar_init(done, 1);
     fence_mbar_init();
   }
@@ -530,11 +554,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kTileM / 16; ++k)
-          mma_ts(t_dv, tmem + 8u * k, ddomn0 + sq + (uint64_t)((k * 2048) >> 4), idesc_o,
+          mma_ts(t_dv, tmem + pcol(k), ddomn0 + sq + (uint64_t)((k * 2048) >> 4), idesc_o,
                  (s > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
         for (int k = 0; k < kTileM / 16; ++k)
-          mma_ts(t_dk, tmem + 128u + 8u * k, dqmn0 + sq + (uint64_t)((k * 2048) >> 4), idesc_o,
+          mma_ts(t_dk, tmem + 128u + pcol(k), dqmn0 + sq + (uint64_t)((k * 2048) >> 4), idesc_o,
                  (s > 0 || k > 0) ? 1u : 0u);
         tc_commit(&empty[st]);
       }
@@ -543,6 +567,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ============================== compute ==============================
+    // group cg takes the query columns [32 kCpg cg, 32 kCpg (cg + 1))
+    const int cg = (warp - 4) / 4;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
@@ -569,34 +595,41 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       tc_fence_after();
       const float* vl = vec + st * 2 * kTileM;
 #pragma unroll 1
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int i = 0; i < kCpg; ++i) {
+        const int ch = cg * kCpg + i;
         uint32_t sv[32], dpv[32];
         tmem_ld32(tS + 32 * ch, sv);
         tmem_ld32(tP + 32 * ch, dpv);
         tmem_wait_ld();
         const int i0 = qt * kTileM + 32 * ch;
+        const float4* l4 = reinterpret_cast<const float4*>(vl + 32 * ch);
+        const float4* d4 = reinterpret_cast<const float4*>(vl + kTileM + 32 * ch);
         uint32_t pp[16], pd[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = 32 * ch + 2 * e;
-          const float2 l2 = *reinterpret_cast<const float2*>(vl + c0);
-          const float2 dl = *reinterpret_cast<const float2*>(vl + kTileM + c0);
-          float2 xs = fma2(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
-                           make_float2(sl2, sl2), make_float2(-l2.x, -l2.y));
-          if (edge) {
-            if (!(i0 + 2 * e >= qlo && i0 + 2 * e <= qhi)) xs.x = -INFINITY;
-            if (!(i0 + 2 * e + 1 >= qlo && i0 + 2 * e + 1 <= qhi)) xs.y = -INFINITY;
+        for (int e2 = 0; e2 < 8; ++e2) {
+          const float4 l = l4[e2], dl = d4[e2];  // this pair of pairs' lse2 and Delta
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = 2 * e2 + h2;
+            const float2 lp = h2 ? make_float2(l.z, l.w) : make_float2(l.x, l.y);
+            const float2 dp = h2 ? make_float2(-dl.z, -dl.w) : make_float2(-dl.x, -dl.y);
+            float2 xs = fma2(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
+                             make_float2(sl2, sl2), make_float2(-lp.x, -lp.y));
+            if (edge) {
+              if (!(i0 + 2 * e >= qlo && i0 + 2 * e <= qhi)) xs.x = -INFINITY;
+              if (!(i0 + 2 * e + 1 >= qlo && i0 + 2 * e + 1 <= qhi)) xs.y = -INFINITY;
+            }
+            const float2 pr = exp2_pair(xs, h2 != 0 && !edge);
+            const float2 ds = mul2(pr, add2(make_float2(__uint_as_float(dpv[2 * e]),
+                                                        __uint_as_float(dpv[2 * e + 1])), dp));
+            pp[e] = pack_bf16x2(pr.x, pr.y);
+            pd[e] = pack_bf16x2(ds.x, ds.y);
           }
-          const float2 pr = exp2_pair(xs, (e & 1) != 0 && !edge);
-          const float2 ds = make_float2(pr.x * (__uint_as_float(dpv[2 * e]) - dl.x),
-                                        pr.y * (__uint_as_float(dpv[2 * e + 1]) - dl.y));
-          pp[e] = pack_bf16x2(pr.x, pr.y);
-          pd[e] = pack_bf16x2(ds.x, ds.y);
         }
-        // P^T / dS^T of query columns [32 ch, 32 ch + 32) over the first
-        // half of S^T's / dP^T's columns (already read)
-        tmem_st16(tS + 16 * ch, pp);
-        tmem_st16(tP + 16 * ch, pd);
+        // P^T / dS^T of these 32 query columns over the group's own (already
+        // read) columns of S^T / dP^T
+        tmem_st16(tS + 32 * kCpg * cg + 16 * i, pp);
+        tmem_st16(tP + 32 * kCpg * cg + 16 * i, pd);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -606,12 +639,13 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
       const size_t row = ((size_t)b * p.N + phys_row(geo, c, j_v)) * p.Hkv + g_kv;
+      // the groups share the 2 x D / 32 column chunks of dV and dK
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK (scaled)
+      for (int u = cg; u < 2 * (D / 32); u += kGroupsB) {
+        const int which = u / (D / 32), j = u % (D / 32);  // which 0: dV, 1: dK (scaled)
         uint16_t* orow = (which ? p.dk : p.dv) + row * D;
         const float f = which ? p.scale : 1.f;
-#pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
+        {
           uint32_t v[32];
           tmem_ld32(tmem + 256u + (uint32_t)(which * D) + lane_off + 32 * j, v);
           tmem_wait_ld();
@@ -627,7 +661,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
           }
         }
       }
-    } else if (key_valid && n_steps == 0) {
+    } else if (key_valid && n_steps == 0 && cg == 0) {
       const size_t row = ((size_t)b * p.N + phys_row(geo, c, j_v)) * p.Hkv + g_kv;
       uint4* a = reinterpret_cast<uint4*>(p.dk + row * D);
       uint4* v = reinterpret_cast<uint4*>(p.dv + row * D);
