@@ -159,6 +159,34 @@ typedef struct swa_params {
 SWA_API int swa_forward_ex(const swa_params* p, void* stream);
 
 /*
+ * swa_forward_host -- swa_forward_ex (bf16) for inputs and outputs in host
+ * memory: copies q, k, v from the host into the caller's device buffers,
+ * runs the forward and copies out (and lse) back, overlapping the three.
+ *   q_host, k_host, v_host, out_host [layouts as above] and lse_host
+ *   [B, H, N] (or NULL): host memory, page-locked (cudaHostAlloc /
+ *   cudaHostRegister) for the copies to overlap; q_dev ... lse_dev: device
+ *   buffers of the same shapes (lse_dev NULL iff lse_host is NULL).
+ * The query rows are copied, computed and copied back in chunks of 1024
+ * rows (whole query tiles), each chunk's k / v rows just before its
+ * kernel, on two library-owned copy streams and `stream` (the kernels),
+ * ordered by events: the copy in of chunk c + 1, the kernel of chunk c and
+ * the copy out of chunk c - 1 overlap.  Windows unbounded on the right,
+ * dilation > 1, block dilation and global tokens are one chunk.  The call
+ * is asynchronous on `stream` like the others: work queued on `stream`
+ * before it comes first, work queued after it sees out_host / lse_host
+ * complete; the host buffers must stay valid until then.  Other arguments,
+ * validation and errors as for swa_forward_ex.  The first call on a device
+ * creates the copy streams and their events (kept until swa_release); calls
+ * on one device share them.
+ */
+SWA_API int swa_forward_host(const void* q_host, const void* k_host, const void* v_host,
+                             void* out_host, float* lse_host, void* q_dev, void* k_dev,
+                             void* v_dev, void* out_dev, float* lse_dev, int B, int H, int Hkv,
+                             int N, int D, int win_left, int win_right, int dilation,
+                             int dilation_block, const int32_t* global_idx, int n_global,
+                             float scale, void* stream);
+
+/*
  * One layer of a per-layer window schedule (see swa_forward_layers).  Every
  * field means what the field of the same name means in swa_params (bf16).
  */
@@ -377,8 +405,9 @@ SWA_API int swa_schedule(int N, int win_left, int win_right, int dilation,
                          int dilation_block, int32_t* tile_out, int cap);
 
 /* swa_release -- frees every library-owned workspace (the row kernel's
-   split workspaces and the backward's accumulators) on every device that
-   has one, after synchronising that device; later calls allocate again. */
+   split workspaces and the backward's accumulators) and the copy streams of
+   swa_forward_host on every device that has them, after synchronising that
+   device; later calls make them again. */
 SWA_API int swa_release(void);
 
 /*

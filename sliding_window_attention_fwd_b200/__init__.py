@@ -28,6 +28,7 @@ _EXPORTS = (
     "swa_forward",
     "swa_forward_ex",
     "swa_forward_f32",
+    "swa_forward_host",
     "swa_forward_layers",
     "swa_paged_window",
     "swa_release",

@@ -22,6 +22,8 @@ _F = ctypes.c_float
 
 _lib.swa_forward.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I, _F, _P]
 _lib.swa_forward_ex.argtypes = [_P, _P]
+_lib.swa_forward_host.argtypes = [_P] * 10 + [_I] * 9 + [_P, _I, _F, _P]
+_lib.swa_forward_host.restype = _I
 _lib.swa_forward_f32.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _I,
                                  _F, _P]
 _lib.swa_decode.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
@@ -184,6 +186,40 @@ def swa_forward_ex(q, k, v, out=None, lse=None, win_left=-1, win_right=-1, dilat
         _check(_lib.swa_forward_ex(ctypes.c_void_p(ctypes.addressof(prm)), _stream(stream)),
                "swa_forward_ex")
     return out
+
+
+def swa_forward_host(q_host, k_host, v_host, q_dev, k_dev, v_dev, out_host=None, out_dev=None,
+                     lse_host=None, lse_dev=None, win_left=-1, win_right=-1, dilation=1,
+                     dilation_block=0, global_idx=None, scale=0.0, stream=None):
+    """The bf16 forward for host-resident inputs and outputs (C:
+    swa_forward_host): q/k/v are copied from the (pinned) host tensors into
+    the given device tensors, the forward runs, out (and lse) come back into
+    out_host / lse_host, the copies overlapping the kernels chunk by chunk.
+    Asynchronous on `stream`; returns out_host."""
+    for name, h, dv in (("q", q_host, q_dev), ("k", k_host, k_dev), ("v", v_host, v_dev)):
+        if h.is_cuda or not h.is_contiguous() or h.shape != dv.shape or h.dtype != dv.dtype:
+            raise ValueError(f"{name}_host: a contiguous host tensor shaped like {name}_dev")
+    if out_dev is None:
+        out_dev = torch.empty_like(q_dev)
+    if out_host is None:
+        out_host = torch.empty(q_host.shape, dtype=q_host.dtype, pin_memory=True)
+    if (lse_host is None) != (lse_dev is None):
+        raise ValueError("give both lse_host and lse_dev, or neither")
+    B, N, H, Hkv, D, out_dev, gi, ng = _fwd_common(q_dev, k_dev, v_dev, out_dev, lse_dev,
+                                                    global_idx, torch.bfloat16)
+    if out_host.is_cuda or not out_host.is_contiguous() or out_host.shape != out_dev.shape:
+        raise ValueError("out_host: a contiguous host tensor shaped like out")
+    if lse_host is not None and (lse_host.is_cuda or not lse_host.is_contiguous()
+                                 or lse_host.shape != lse_dev.shape):
+        raise ValueError("lse_host: a contiguous host tensor shaped like lse")
+    with torch.cuda.device(q_dev.device):
+        _check(_lib.swa_forward_host(_ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(out_host),
+                                     _ptr(lse_host), _ptr(q_dev), _ptr(k_dev), _ptr(v_dev),
+                                     _ptr(out_dev), _ptr(lse_dev), B, H, Hkv, N, D,
+                                     int(win_left), int(win_right), int(dilation),
+                                     int(dilation_block), _ptr(gi), ng, float(scale),
+                                     _stream(stream)), "swa_forward_host")
+    return out_host
 
 
 def swa_forward_layers(layers, stream=None):

@@ -240,6 +240,24 @@ SWA_API int swa_forward(const void* q, const void* k, const void* v, void* out, 
   return swa_forward_ex(&p, stream);
 }
 
+SWA_API int swa_forward_host(const void* q_host, const void* k_host, const void* v_host,
+                             void* out_host, float* lse_host, void* q_dev, void* k_dev,
+                             void* v_dev, void* out_dev, float* lse_dev, int B, int H, int Hkv,
+                             int N, int D, int win_left, int win_right, int dilation,
+                             int dilation_block, const int32_t* global_idx, int n_global,
+                             float scale, void* stream) {
+  int st = check_forward_bf16(q_dev, k_dev, v_dev, out_dev, lse_dev, B, H, Hkv, N, D, dilation,
+                              dilation_block, global_idx, n_global);
+  if (st != SWA_OK) return st;
+  if (!q_host || !k_host || !v_host || !out_host) return SWA_ERR_ARG;
+  if ((lse_host == nullptr) != (lse_dev == nullptr)) return SWA_ERR_ARG;
+  if (B == 0 || N == 0) return SWA_OK;
+  return forward_host(q_host, k_host, v_host, out_host, lse_host, const_cast<void*>(q_dev),
+                      const_cast<void*>(k_dev), const_cast<void*>(v_dev), out_dev, lse_dev, B, H,
+                      Hkv, N, D, win_left, win_right, dilation, dilation_block, global_idx,
+                      n_global, resolve_scale(scale, D), static_cast<cudaStream_t>(stream));
+}
+
 SWA_API int swa_forward_layers(const swa_layer* layers, int n_layers, int B, int H, int Hkv,
                                int N, int D, int* bad_layer, void* stream) {
   if (bad_layer) *bad_layer = -1;
@@ -446,6 +464,7 @@ SWA_API int swa_set_workspace_allocator(swa_alloc_fn alloc, swa_free_fn free_fn,
 SWA_API int swa_release(void) {
   release_workspaces();
   release_backward_workspace();
+  release_host_pipes();
   return SWA_OK;
 }
 

@@ -9,9 +9,10 @@
 //
 // Two query heads per CTA let the tensor core alternate between them:
 // while one softmax warpgroup turns S into P for head 0, the MMAs of head 1
-// run, and the other way round.  The two heads either share a kv head (GQA:
-// one K/V stream) or read two kv heads (two K/V streams, D = 64 only, to fit
-// shared memory).
+// run, and the other way round.  The two heads share a kv head (GQA: one
+// K/V stream; the kernel can also stream two kv heads, NSTREAM = 2).
+// Without such a pair a CTA takes one head; at D = 64 two of those CTAs
+// share an SM and alternate the same way.
 //
 // Warp roles (warpgroup 0 = warps 0-3; warpgroup 1 + s = softmax of slot s):
 //   warp 0     producer: TMA loads of the Q tiles once and of the K/V tiles
@@ -61,7 +62,6 @@ namespace {
 constexpr int kMaxClasses = 8;   // residue classes per launch (tensor maps in params)
 constexpr int kChunkBytes = kTileM * 128;  // one 64-column slice of a 128-row tile
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-constexpr uint32_t kTmemCols = 512;
 struct FwdParams {
   CUtensorMap tmQ[kMaxClasses];
   CUtensorMap tmK[kMaxClasses];
@@ -85,6 +85,7 @@ struct FwdParams {
   // row).  The band CTAs leave those rows to them.
   int n_gitems, n_gq_tiles;
   int qtile_prefix[kMaxClasses + 1];
+  int qt_base;  // first query tile of the launch (a row-range launch of one class)
   int Mv[kMaxClasses];
   float scale_log2;
   // Query window (chunked append; pos0 == NULL otherwise): the Mq query
@@ -101,7 +102,14 @@ struct Cfg {
   static constexpr int kTile = D / 64 * kChunkBytes;        // 128 rows x D bf16
   static constexpr int kStageBytes = 2 * NSTREAM * kTile;   // K and V of every stream
   static constexpr int kQBytes = NSLOT * kTile;
-  static constexpr int kBudget = 224 * 1024;
+  // one head at D = 64 is small enough for two CTAs per SM (shared memory,
+  // TMEM and, with the register split below, registers), so one CTA's fill
+  // and drain overlap the other's tiles
+  static constexpr int kMinBlocks = (NSLOT == 1 && D == 64) ? 2 : 1;
+  static constexpr int kBudget = kMinBlocks == 2 ? 96 * 1024 : 224 * 1024;
+  // TMEM: S/P of slot s at [128 s, 128 s + 128), O of slot s at kOcol + D s
+  static constexpr uint32_t kOcol = 128u * NSLOT;
+  static constexpr uint32_t kTmemCols = kOcol + NSLOT * D <= 256 ? 256u : 512u;
   static constexpr int kFit = (kBudget - kQBytes) / kStageBytes;
   static constexpr int kStages = kFit > 4 ? 4 : kFit;
   static_assert(kStages >= 2, "K/V ring needs two stages");
@@ -122,7 +130,8 @@ struct Cfg {
 // token/block dilation) only; 1 the query window of a chunked append; 2 the
 // band plus global tokens (global-key tiles and global query rows).
 template <int D, int NSLOT, int NSTREAM, int KIND>
-__global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
+__global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
+                                  Cfg<D, NSLOT, NSTREAM>::kMinBlocks)
     swa_fwd_sm100_kernel(const __grid_constant__ FwdParams p) {
   using C = Cfg<D, NSLOT, NSTREAM>;
   constexpr int kStages = C::kStages;
@@ -167,7 +176,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
   } else {
     const int jt = p.qtile_prefix[p.nclass] - 1 - x;
     while (cl + 1 < p.nclass && p.qtile_prefix[cl + 1] <= jt) ++cl;
-    qt = jt - p.qtile_prefix[cl];
+    qt = jt - p.qtile_prefix[cl] + p.qt_base;
   }
   const int c = p.class0 + cl;
   const int grp = p.H / p.Hkv;
@@ -235,7 +244,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_alloc(tmem_holder, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -253,8 +262,10 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
 
   if (warp < 4) {
     // producer and issuers need few registers: hand the rest to the softmax
-    // warpgroups (128 x 56 + 256 x 208 = 60416 <= 384 x 168 launched)
-    if (NSLOT == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+    // warpgroups (two slots: 128 x 56 + 256 x 208 = 60416 <= 384 x 168
+    // launched; one slot, two CTAs per SM: 128 x 56 + 128 x 200 = 256 x 128)
+    if (NSLOT == 2 || C::kMinBlocks == 2)
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
     if (warp == 0) {
       // =========================== producer ===========================
       const CUtensorMap* mapK = gitem ? &p.tmKf : &p.tmK[map_idx];
@@ -413,7 +424,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
         // between it and the late half of the next tile's S.
         auto pv_half = [&](int it, bool early) {
           const uint64_t dv = dv0 + (uint64_t)(it % kStages) * kStageStep;
-          const uint32_t to = tmem + 256u + 128u * s;
+          const uint32_t to = tmem + C::kOcol + (uint32_t)D * s;
           const int e = it & 1;
           const uint32_t tp = tslot + 64u * (uint32_t)e + (early ? 0u : 32u);
           const int kh = early ? e : (e ^ 1);  // key half
@@ -470,13 +481,15 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
     }
   } else {
     if (NSLOT == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+    if (NSLOT == 1 && C::kMinBlocks == 2)
+      asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
     // ============================ softmax ============================
     const int slot = warp / 4 - 1;
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + 128u * slot + lane_off;
-    const uint32_t tO = tmem + 256u + 128u * slot + lane_off;
+    const uint32_t tO = tmem + C::kOcol + (uint32_t)D * slot + lane_off;
     const int h = head[slot];
     const int m_row = qt * kTileM + r;  // local query row
     const int m_v = q0 + m_row;         // its virtual row among the keys
@@ -810,14 +823,14 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
 template <int D, int NSLOT, int NSTREAM>
 int launch_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
                 int Hkv, int N, int L, int R, int d, int bs, const int32_t* G, int ng,
-                float scale, cudaStream_t stream, const QueryWindow* qw) {
+                float scale, cudaStream_t stream, const QueryWindow* qw, int qt_lo, int qt_hi) {
   using C = Cfg<D, NSLOT, NSTREAM>;
   static std::atomic<unsigned long long> attr_kind[3] = {{0}, {0}, {0}};
   const int kind = qw ? 1 : (ng > 0 ? 2 : 0);
@@ -825,15 +838,17 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
                         reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 1>),
                         reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 2>)};
   if (!smem_attr_once(kfn[kind], C::kAlloc, attr_kind[kind])) return SWA_ERR_CUDA;
-  if (NSLOT == 2) {
-    // The register split (warpgroup 0: 56 per thread, the softmax
-    // warpgroups: 208) must fit in what the block is launched with, or
-    // setmaxnreg.inc would never return: checked once per kernel form.
+  if (NSLOT == 2 || C::kMinBlocks == 2) {
+    // The register split (warpgroup 0: 56 per thread, each softmax
+    // warpgroup: 208 with two slots, 200 with one) must fit in what the
+    // block is launched with, or setmaxnreg.inc would never return: checked
+    // once per kernel form.
+    const long need = NSLOT == 2 ? 128L * 56 + 256L * 208 : 128L * 56 + 128L * 200;
     static std::atomic<int> regs_ok[3] = {{0}, {0}, {0}};
     if (regs_ok[kind].load(std::memory_order_acquire) == 0) {
       cudaFuncAttributes fa;
       if (cudaFuncGetAttributes(&fa, kfn[kind]) != cudaSuccess) return SWA_ERR_CUDA;
-      regs_ok[kind].store((long)fa.numRegs * C::kThreads >= 128L * 56 + 256L * 208 ? 1 : -1,
+      regs_ok[kind].store((long)fa.numRegs * C::kThreads >= need ? 1 : -1,
                           std::memory_order_release);
     }
     if (regs_ok[kind].load(std::memory_order_acquire) < 0) return SWA_ERR_UNSUPPORTED;
@@ -869,6 +884,15 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
       p.Mv[cl] = class_valid_rows(geo, c0 + cl);
       const int rows_q = qw ? qw->Mq : p.Mv[cl];
       p.qtile_prefix[cl + 1] = p.qtile_prefix[cl] + (rows_q + kTileM - 1) / kTileM;
+    }
+    if (qt_hi >= 0) {
+      // a row-range launch (one class): only query tiles [qt_lo, qt_hi)
+      if (geo.nclass != 1 || qw) return SWA_ERR_UNSUPPORTED;
+      const int all = p.qtile_prefix[1];
+      const int lo = qt_lo < 0 ? 0 : (qt_lo > all ? all : qt_lo);
+      const int hi = qt_hi > all ? all : (qt_hi < lo ? lo : qt_hi);
+      p.qt_base = lo;
+      p.qtile_prefix[1] = hi - lo;
     }
     if (qw) {
       p.pos0 = qw->pos0;
@@ -935,25 +959,27 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
 }  // namespace
 
 // Two query heads per CTA when they share a kv head (GQA group of even
-// size), or, at D = 64, when two K/V streams fit in shared memory; one head
-// per CTA otherwise.
+// size); otherwise one head per CTA, two CTAs per SM at D = 64 (measured on
+// the D = 64 MHA workloads against two heads with two K/V streams per CTA:
+// Longformer 133 -> 125 us, token dilation 172 -> 155, block 169 -> 156).
 int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, float* lse, int B,
                      int H, int Hkv, int N, int D, int L, int R, int d, int bs, const int32_t* G,
-                     int ng, float scale, cudaStream_t stream, const QueryWindow* qw) {
+                     int ng, float scale, cudaStream_t stream, const QueryWindow* qw, int qt_lo,
+                     int qt_hi) {
   const bool gqa_pair = (H / Hkv) % 2 == 0;
   if (D == 128) {
     if (gqa_pair)
       return launch_impl<128, 2, 1>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
-                                    stream, qw);
+                                    stream, qw, qt_lo, qt_hi);
     return launch_impl<128, 1, 1>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
-                                  stream, qw);
+                                  stream, qw, qt_lo, qt_hi);
   }
   if (D == 64) {
     if (gqa_pair)
       return launch_impl<64, 2, 1>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
-                                   stream, qw);
-    return launch_impl<64, 2, 2>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
-                                 stream, qw);
+                                   stream, qw, qt_lo, qt_hi);
+    return launch_impl<64, 1, 1>(q, k, v, out, lse, B, H, Hkv, N, L, R, d, bs, G, ng, scale,
+                                 stream, qw, qt_lo, qt_hi);
   }
   return SWA_ERR_UNSUPPORTED;
 }

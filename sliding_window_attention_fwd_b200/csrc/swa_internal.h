@@ -53,10 +53,12 @@ struct QueryWindow {
   const int64_t* pos0;
   int q0, Mq, win;
 };
+// qt_lo / qt_hi (token-level, d == 1, no query window): launch only the
+// query tiles [qt_lo, qt_hi) of the sequence (qt_hi < 0: all).
 int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, float* lse,
                      int B, int H, int Hkv, int N, int D, int L, int R, int d, int bs,
                      const int32_t* G, int ng, float scale, cudaStream_t stream,
-                     const QueryWindow* qw = nullptr);
+                     const QueryWindow* qw = nullptr, int qt_lo = 0, int qt_hi = -1);
 
 int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* out,
                   float* lse, const int64_t* pos, int B, int H, int Hkv, int D, int W,
@@ -79,6 +81,12 @@ int launch_append(const void* q, const void* k_new, const void* v_new, void* k_r
                   void* out, float* lse, const int64_t* pos0, int B, int C, int H, int Hkv, int D,
                   int W, float scale, cudaStream_t stream);
 void release_workspaces();
+// The forward over host-resident inputs and outputs (swa_host.cu).
+int forward_host(const void* qh, const void* kh, const void* vh, void* oh, float* lh, void* qd,
+                 void* kd, void* vd, void* od, float* ld, int B, int H, int Hkv, int N, int D,
+                 int L, int R, int d, int bs, const int32_t* G, int ng, float scale,
+                 cudaStream_t stream);
+void release_host_pipes();
 int launch_backward(const void* q, const void* k, const void* v, const void* out,
                     const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
                     int H, int Hkv, int N, int D, int L, int R, int d, int bs, const int32_t* G,

@@ -245,3 +245,20 @@ def test_workspace_allocator_arguments():
     with pytest.raises(ValueError):
         swa.swa_set_workspace_allocator(lambda n: 0)
     swa.swa_set_workspace_allocator()
+
+
+def test_forward_host_validation():
+    """Host and device buffers both required; lse both or neither; B = 0 is a
+    no-op before any CUDA call."""
+    def fh(**kw):
+        a = [kw.get(n, A) for n in ("qh", "kh", "vh", "oh")] + [kw.get("lh", None)]
+        a += [kw.get(n, A) for n in ("qd", "kd", "vd", "od")] + [kw.get("ld", None)]
+        return L.swa_forward_host(*a, kw.get("B", 1), 4, 2, 64, 128, 8, 0, 1, 0, None, 0, 0.0,
+                                  None)
+    assert fh(qh=None) == ARG
+    assert fh(oh=None) == ARG
+    assert fh(qd=None) == ARG
+    assert fh(lh=A) == ARG          # lse on the host but not on the device
+    assert fh(qd=A + 8) == ALIGN
+    assert fh(B=0) == OK
+    assert fh(B=0, lh=A, ld=A) == OK
