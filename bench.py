@@ -322,6 +322,9 @@ def run_ours(args, rank, world, local_rank):
     if args.only == "decode":
         run_decode_only(args, swa, inputs, dev, stream, flush)
         return
+    if args.only in SMALL_CASES:
+        run_small_case(args, swa, inputs, dev)
+        return
     if args.only in ("paged", "append", "backward"):
         run_next_only(args, swa, inputs, dev, stream, flush)
         return
@@ -562,6 +565,49 @@ def run_next_only(args, swa, inputs, dev, stream, flush):
     print(json.dumps({"only": args.only, "ms_per_step": sum(ms) / len(ms)}), flush=True)
 
 
+# Smaller cases of the timed kernels for ncu captures that take many passes
+# (the full-size workloads are captured with one-pass metrics only).
+SMALL_CASES = ("fwd_small", "bwd_small", "dec_small")
+
+
+def run_small_case(args, swa, inputs, dev):
+    """fwd_small: causal forward B1 N4096 H32/8 D128 W2048; bwd_small: its
+    backward (B1 N4096 H8/2 D128 W2048); dec_small: ring decode B16 H32/8
+    D128 W4096.  Seeded N(0,1) bf16 inputs, args.warmup + args.steps calls."""
+    import torch
+    bf = torch.bfloat16
+    n = args.warmup + args.steps
+    if args.only == "dec_small":
+        B, H, Hkv, D, W = 16, 32, 8, 128, 4096
+        q = inputs.normal((B, H, D), 7, 0, bf, dev)
+        k = inputs.normal((B, W, Hkv, D), 7, 1, bf, dev)
+        v = inputs.normal((B, W, Hkv, D), 7, 2, bf, dev)
+        pos = torch.full((B,), 100000, dtype=torch.int64, device=dev)
+        out = torch.empty_like(q)
+        for _ in range(n):
+            swa.swa_decode(q, k, v, pos, out)
+    else:
+        B, N, D, L = 1, 4096, 128, 2047
+        H, Hkv = (32, 8) if args.only == "fwd_small" else (8, 2)
+        q = inputs.normal((B, N, H, D), 9, 0, bf, dev)
+        k = inputs.normal((B, N, Hkv, D), 9, 1, bf, dev)
+        v = inputs.normal((B, N, Hkv, D), 9, 2, bf, dev)
+        lse = torch.empty(B, H, N, device=dev)
+        out = torch.empty_like(q)
+        swa.swa_forward(q, k, v, out, lse, L, 0)
+        if args.only == "fwd_small":
+            for _ in range(n):
+                swa.swa_forward(q, k, v, out, lse, L, 0)
+        else:
+            do = inputs.normal((B, N, H, D), 9, 3, bf, dev)
+            g = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+            for _ in range(n):
+                swa.swa_backward(q, k, v, out, do, lse, L, 0, dq=g[0], dk=g[1], dv=g[2])
+    torch.cuda.synchronize()
+    assert swa.swa_device_error() == 0
+    print(json.dumps({"only": args.only, "calls": n}), flush=True)
+
+
 def torch_empty_like(t):
     import torch
     return torch.empty_like(t)
@@ -622,7 +668,7 @@ def main():
                     help="also write the clock samples of the timed region to this CSV file")
     ap.add_argument("--only", default="all",
                     choices=["all", "forward", "decode", "paged", "append", "backward",
-                             "others"],
+                             "others", *SMALL_CASES],
                     help="run one workload alone (profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -105,6 +105,7 @@ struct BCfg {
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16 + 1024;  // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory budget");
+  static_assert(2 * kStages >= kGroupsB, "dq kernel: the Delta parts fit in the vector area");
   // TMEM columns: S (or S^T) [0, 128), dP (or dP^T) [128, 256), then the
   // accumulators: dq kernel dQ [256, 256 + D); dkdv kernel dV, dK.
   static constexpr uint32_t kTmemCols = 512;
@@ -301,51 +302,60 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     int int_lo, int_hi;
     interior_tiles(geo, Mv, qt, &int_lo, &int_hi);
     const float sl2 = p.scale_log2;
-    // Delta_i = dO_i . out_i and lse in log2 units; rows past the class
-    // end get P = 0
+    // Delta_i = dO_i . out_i (each group sums a quarter of the row, the
+    // parts meet in shared memory) and lse in log2 units; rows past the
+    // class end get P = 0
     float delta = 0.f, lse2 = INFINITY;
-    if (row_valid) {
-      const size_t row = ((size_t)b * p.N + i_phys) * p.H + h;
-      const uint4* a = reinterpret_cast<const uint4*>(p.dout + row * D);
-      const uint4* o = reinterpret_cast<const uint4*>(p.out + row * D);
+    {
+      float* part = reinterpret_cast<float*>(smem + C::kVec);  // [group][128]
       float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 4
-      for (int u = 0; u < D / 8; ++u) {
-        const uint4 wa = __ldg(a + u), wo = __ldg(o + u);
-        const uint32_t xa[4] = {wa.x, wa.y, wa.z, wa.w}, xo[4] = {wo.x, wo.y, wo.z, wo.w};
+      if (row_valid) {
+        const size_t row = ((size_t)b * p.N + i_phys) * p.H + h;
+        const uint4* a = reinterpret_cast<const uint4*>(p.dout + row * D);
+        const uint4* o = reinterpret_cast<const uint4*>(p.out + row * D);
+        constexpr int kU = D / 8 / kGroupsB;  // 16-byte chunks per group
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          acc0 = fmaf(__uint_as_float(xa[e] << 16), __uint_as_float(xo[e] << 16), acc0);
-          acc1 = fmaf(__uint_as_float(xa[e] & 0xFFFF0000u), __uint_as_float(xo[e] & 0xFFFF0000u),
-                      acc1);
+        for (int u = cg * kU; u < (cg + 1) * kU; ++u) {
+          const uint4 wa = __ldg(a + u), wo = __ldg(o + u);
+          const uint32_t xa[4] = {wa.x, wa.y, wa.z, wa.w}, xo[4] = {wo.x, wo.y, wo.z, wo.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            acc0 = fmaf(__uint_as_float(xa[e] << 16), __uint_as_float(xo[e] << 16), acc0);
+            acc1 = fmaf(__uint_as_float(xa[e] & 0xFFFF0000u),
+                        __uint_as_float(xo[e] & 0xFFFF0000u), acc1);
+          }
         }
       }
-      delta = acc0 + acc1;
-      const size_t li = ((size_t)b * p.H + h) * p.N + i_phys;
-      lse2 = __ldg(p.lse + li) * kLog2e;
-      if (cg == 0) p.delta[li] = delta;
+      part[cg * kTileM + r] = acc0 + acc1;
+      asm volatile("bar.sync 1, %0;" ::"r"(kGroupsB * 128) : "memory");
+#pragma unroll
+      for (int g2 = 0; g2 < kGroupsB; ++g2) delta += part[g2 * kTileM + r];
+      if (row_valid) {
+        const size_t li = ((size_t)b * p.H + h) * p.N + i_phys;
+        lse2 = __ldg(p.lse + li) * kLog2e;
+        if (cg == 0) p.delta[li] = delta;
+      }
     }
     bool ok = true;
     for (int it = 0; it < n_tiles; ++it) {
       const uint32_t ph = (uint32_t)it & 1u;
       const int t = tr.kv_begin + it;
       const bool edge = !(t >= int_lo && t <= int_hi);
-      bool w = mbar_wait(s_full, ph, p.err, abort_flag) && mbar_wait(dp_full, ph, p.err, abort_flag);
+      // P as soon as S is in TMEM (dP is still being computed)
+      bool w = mbar_wait(s_full, ph, p.err, abort_flag);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
       }
       tc_fence_after();
-#pragma unroll 1
+      float2 pr[kCpg][16];
+#pragma unroll
       for (int i = 0; i < kCpg; ++i) {
         const int ch = cg * kCpg + i;
-        uint32_t sv[32], dpv[32];
+        uint32_t sv[32];
         tmem_ld32(tS + 32 * ch, sv);
-        tmem_ld32(tP + 32 * ch, dpv);
         tmem_wait_ld();
         const int n0 = t * kTileN + 32 * ch;
-        const float2 ndl = make_float2(-delta, -delta);
-        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           float2 xs = fma2(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
@@ -355,9 +365,28 @@ __global__ void __launch_bounds__(kThreadsB, 1)
             if (!(j0 >= klo && j0 <= khi && j0 < Mv)) xs.x = -INFINITY;
             if (!(j0 + 1 >= klo && j0 + 1 <= khi && j0 + 1 < Mv)) xs.y = -INFINITY;
           }
-          const float2 pr = exp2_pair(xs, (e & 1) != 0 && !edge);
-          const float2 ds = mul2(pr, add2(make_float2(__uint_as_float(dpv[2 * e]),
-                                                      __uint_as_float(dpv[2 * e + 1])), ndl));
+          pr[i][e] = exp2_pair(xs, (e & 1) != 0 && !edge);
+        }
+      }
+      // then dS = P (dP - Delta)
+      w = mbar_wait(dp_full, ph, p.err, abort_flag);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int i = 0; i < kCpg; ++i) {
+        const int ch = cg * kCpg + i;
+        uint32_t dpv[32];
+        tmem_ld32(tP + 32 * ch, dpv);
+        tmem_wait_ld();
+        const float2 ndl = make_float2(-delta, -delta);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float2 ds = mul2(pr[i][e], add2(make_float2(__uint_as_float(dpv[2 * e]),
+                                                            __uint_as_float(dpv[2 * e + 1])), ndl));
           pk[e] = pack_bf16x2(ds.x, ds.y);
         }
         // dS of these 32 keys over the group's own (already read) S columns
@@ -424,8 +453,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   uint64_t* full_kv = bars;           // K and V tiles
   uint64_t* full = bars + 1;          // [S_]: Q, dO tiles + lse / Delta vectors
   uint64_t* empty = full + S_;        // [S_]
-  uint64_t* st_full = empty + S_;     // S^T and dP^T of the step in TMEM
-  uint64_t* pt_full = st_full + 1;    // P^T, dS^T written (128 arrivals)
+  uint64_t* st_full = empty + S_;     // S^T of the step in TMEM
+  uint64_t* dpt_full = st_full + 1;   // dP^T of the step in TMEM
+  uint64_t* pt_full = dpt_full + 1;   // P^T, dS^T written (128 arrivals per group)
   uint64_t* done = pt_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
@@ -458,6 +488,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       mbar_init(&empty[s], 1);
     }
     mbar_init(st_full, 1);
+    mbar_init(dpt_full, 1);
     mbar_init(pt_full, 128 * kGroupsB);
     mbar_init(done, 1);
     fence_mbar_init();
@@ -544,11 +575,12 @@ __global__ void __launch_bounds__(kThreadsB, 1)
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
           mma_ss(tmem, dk_ + kmajor_off(k), dq0 + sq + kmajor_off(k), idesc_s, k > 0 ? 1u : 0u);
+        tc_commit(st_full);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
           mma_ss(tmem + 128u, dv_ + kmajor_off(k), ddo0 + sq + kmajor_off(k), idesc_s,
                  k > 0 ? 1u : 0u);
-        tc_commit(st_full);
+        tc_commit(dpt_full);
         // dV += P^T dO, dK += dS^T Q
         if (!mbar_wait(pt_full, (uint32_t)s & 1u, p.err, abort_flag)) break;
         tc_fence_after();
@@ -587,48 +619,72 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       const int st = s % S_;
       const int qt = qr.kv_begin + s / grp;
       const bool edge = !(qt >= int_lo && qt <= int_hi);
-      const bool w = mbar_wait(st_full, (uint32_t)s & 1u, p.err, abort_flag);
+      // P^T as soon as S^T is in TMEM (dP^T is still being computed)
+      bool w = mbar_wait(st_full, (uint32_t)s & 1u, p.err, abort_flag);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const float* vl = vec + st * 2 * kTileM;
-#pragma unroll 1
+      float2 pr[kCpg][16];
+#pragma unroll
       for (int i = 0; i < kCpg; ++i) {
         const int ch = cg * kCpg + i;
-        uint32_t sv[32], dpv[32];
+        uint32_t sv[32];
         tmem_ld32(tS + 32 * ch, sv);
-        tmem_ld32(tP + 32 * ch, dpv);
         tmem_wait_ld();
         const int i0 = qt * kTileM + 32 * ch;
         const float4* l4 = reinterpret_cast<const float4*>(vl + 32 * ch);
-        const float4* d4 = reinterpret_cast<const float4*>(vl + kTileM + 32 * ch);
-        uint32_t pp[16], pd[16];
+        uint32_t pp[16];
 #pragma unroll
         for (int e2 = 0; e2 < 8; ++e2) {
-          const float4 l = l4[e2], dl = d4[e2];  // this pair of pairs' lse2 and Delta
+          const float4 l = l4[e2];  // lse2 of this pair of pairs
 #pragma unroll
           for (int h2 = 0; h2 < 2; ++h2) {
             const int e = 2 * e2 + h2;
             const float2 lp = h2 ? make_float2(l.z, l.w) : make_float2(l.x, l.y);
-            const float2 dp = h2 ? make_float2(-dl.z, -dl.w) : make_float2(-dl.x, -dl.y);
             float2 xs = fma2(make_float2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1])),
                              make_float2(sl2, sl2), make_float2(-lp.x, -lp.y));
             if (edge) {
               if (!(i0 + 2 * e >= qlo && i0 + 2 * e <= qhi)) xs.x = -INFINITY;
               if (!(i0 + 2 * e + 1 >= qlo && i0 + 2 * e + 1 <= qhi)) xs.y = -INFINITY;
             }
-            const float2 pr = exp2_pair(xs, h2 != 0 && !edge);
-            const float2 ds = mul2(pr, add2(make_float2(__uint_as_float(dpv[2 * e]),
-                                                        __uint_as_float(dpv[2 * e + 1])), dp));
-            pp[e] = pack_bf16x2(pr.x, pr.y);
+            pr[i][e] = exp2_pair(xs, h2 != 0 && !edge);
+            pp[e] = pack_bf16x2(pr[i][e].x, pr[i][e].y);
+          }
+        }
+        // P^T of these 32 query columns over the group's own (already read)
+        // columns of S^T
+        tmem_st16(tS + 32 * kCpg * cg + 16 * i, pp);
+      }
+      // then dS^T = P^T (dP^T - Delta)
+      w = mbar_wait(dpt_full, (uint32_t)s & 1u, p.err, abort_flag);
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int i = 0; i < kCpg; ++i) {
+        const int ch = cg * kCpg + i;
+        uint32_t dpv[32];
+        tmem_ld32(tP + 32 * ch, dpv);
+        tmem_wait_ld();
+        const float4* d4 = reinterpret_cast<const float4*>(vl + kTileM + 32 * ch);
+        uint32_t pd[16];
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) {
+          const float4 dl = d4[e2];  // Delta of this pair of pairs
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = 2 * e2 + h2;
+            const float2 dn = h2 ? make_float2(-dl.z, -dl.w) : make_float2(-dl.x, -dl.y);
+            const float2 ds = mul2(pr[i][e], add2(make_float2(__uint_as_float(dpv[2 * e]),
+                                                              __uint_as_float(dpv[2 * e + 1])), dn));
             pd[e] = pack_bf16x2(ds.x, ds.y);
           }
         }
-        // P^T / dS^T of these 32 query columns over the group's own (already
-        // read) columns of S^T / dP^T
-        tmem_st16(tS + 32 * kCpg * cg + 16 * i, pp);
         tmem_st16(tP + 32 * kCpg * cg + 16 * i, pd);
       }
       tmem_wait_st();
