@@ -202,3 +202,26 @@ def test_globals_allocate_nothing(swa):
                                   cfg.scale)
     compare(out.float().cpu().numpy(), ref_o, BF16_MAX_ABS, BF16_MEAN_ABS, what="out")
     compare(lse.cpu().numpy(), ref_l, LSE_ABS, what="lse")
+
+
+@pytest.mark.parametrize("case", [
+    # (B, N, H, D, L, R, d, bs): D = 64, no GQA pair, short key walks
+    (8, 4296, 16, 64, 100, 100, 1, 0),   # 34 query tiles per head, a ragged last one
+    (8, 4296, 16, 64, 200, 0, 1, 0),     # causal
+    (4, 8192, 16, 64, 64, 64, 2, 0),     # token dilation (two classes)
+    (4, 8192, 16, 64, 128, 128, 2, 64),  # block dilation
+])
+def test_bf16_d64_mha_short_walks(swa, case):
+    """D = 64 heads without a GQA pair (one head per CTA, two CTAs per SM)
+    and walks of two to four key tiles, at batch sizes that fill many waves:
+    sampled rows (tile, class and ragged-tail edges) against the oracle, and
+    every output finite."""
+    B, N, H, D, L, R, d, bs = case
+    q, k, v = rand_case(B, N, H, H, D, 17)
+    out, lse = run_forward(swa, q, k, v, L, R, d, bs, None, 0.0)
+    edges = list(range(0, 4 * 128, 64)) + [N - 1, N - 129, N - 200, 4095, 4096, 4097]
+    rows = sample_rows(B, H, N, 2500, seed=9, extra_i=edges)
+    ref_o, ref_l = oracle.forward(q, k, v, L, R, d, bs, [], 0.0, rows=rows)
+    compare(out[rows[:, 0], rows[:, 2], rows[:, 1]], ref_o, BF16_MAX_ABS, BF16_MEAN_ABS)
+    compare(lse[rows[:, 0], rows[:, 1], rows[:, 2]], ref_l, LSE_ABS, what="lse")
+    assert np.isfinite(out).all() and np.isfinite(lse).all()
