@@ -219,6 +219,49 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
   const bool block_mode = p.bs > 1;
   const int map_idx = block_mode ? 0 : cl;
 
+  // virtual row -> TMA row coordinate of a 64-row box
+  auto box_row = [&](int vrow) -> int {
+    return block_mode ? (c + p.d * (vrow / kBlockRows)) * kBlockRows : vrow;
+  };
+  const CUtensorMap* mapK = gitem ? &p.tmKf : &p.tmK[map_idx];
+  const CUtensorMap* mapV = gitem ? &p.tmVf : &p.tmV[map_idx];
+  // TMA loads (one thread): the Q tiles, and K or V of band tile it
+  auto load_q = [&]() {
+    prefetch_tensormap(&p.tmQ[map_idx]);
+    mbar_arrive_expect_tx(full_q, C::kQBytes);
+    for (int s = 0; s < NSLOT; ++s)
+      for (int cc = 0; cc < D / 64; ++cc)
+        for (int hh = 0; hh < 2; ++hh)
+          tma_load_4d(smem + C::kQ + s * C::kTile + cc * kChunkBytes + hh * (kChunkBytes / 2),
+                      &p.tmQ[map_idx], full_q, cc * 64, head[s], box_row(qt * kTileM + hh * 64),
+                      b);
+  };
+  auto load_kv = [&](int it, int kv) {
+    const int st = it % kStages;
+    uint64_t* ful = kv ? &full_v[st] : &full_k[st];
+    uint8_t* dst = smem + C::kRing + st * C::kStageBytes + kv * NSTREAM * C::kTile;
+    const CUtensorMap* m = kv ? mapV : mapK;
+    const int t = tr.kv_begin + it;
+    mbar_arrive_expect_tx(ful, NSTREAM * C::kTile);
+    for (int s = 0; s < NSTREAM; ++s)
+      for (int cc = 0; cc < D / 64; ++cc)
+        for (int hh = 0; hh < 2; ++hh) {
+          const int vrow = t * kTileN + hh * 64;
+          tma_load_4d(dst + s * C::kTile + cc * kChunkBytes + hh * (kChunkBytes / 2), m, ful,
+                      cc * 64, kvh[s], gitem ? vrow : box_row(vrow), b);
+        }
+  };
+#ifdef SWA_TEST_WITHHOLD_TILE
+  // failure-detection test build only: this K tile is never loaded, so the
+  // MMA issuer's bounded wait for it runs out
+  auto withheld = [](int it, int kv) { return kv == 0 && it == SWA_TEST_WITHHOLD_TILE; };
+#else
+  auto withheld = [](int, int) { return false; };
+#endif
+  // band tiles of the first ring pass, loaded by thread 0 as soon as the
+  // barriers exist (before TMEM allocation and the block barrier)
+  const int n_early = gitem ? 0 : min(kStages, n_band);
+
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(full_q, 1);
@@ -242,6 +285,14 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       mbar_init(&oe_done[s], 1);
     }
     fence_mbar_init();
+    if (!gitem) {
+      prefetch_tensormap(mapK);
+      prefetch_tensormap(mapV);
+      load_q();
+      for (int it = 0; it < n_early; ++it)
+        for (int kv = 0; kv < 2; ++kv)
+          if (!withheld(it, kv)) load_kv(it, kv);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::kTmemCols);
@@ -255,11 +306,6 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
   const uint32_t q_addr = smem_u32(smem + C::kQ);
   const uint32_t ring_addr = smem_u32(smem + C::kRing);
 
-  // virtual row -> TMA row coordinate of a 64-row box
-  auto box_row = [&](int vrow) -> int {
-    return block_mode ? (c + p.d * (vrow / kBlockRows)) * kBlockRows : vrow;
-  };
-
   if (warp < 4) {
     // producer and issuers need few registers: hand the rest to the softmax
     // warpgroups (two slots: 128 x 56 + 256 x 208 = 60416 <= 384 x 168
@@ -268,8 +314,6 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
     if (warp == 0) {
       // =========================== producer ===========================
-      const CUtensorMap* mapK = gitem ? &p.tmKf : &p.tmK[map_idx];
-      const CUtensorMap* mapV = gitem ? &p.tmVf : &p.tmV[map_idx];
       if (gitem) {
         // gather the tile's global query rows (zeros past the last) with
         // plain 16-byte loads into the swizzled layout of a TMA box
@@ -296,20 +340,10 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(full_q);
-      } else if (lane == 0) {
-        prefetch_tensormap(&p.tmQ[map_idx]);
-        prefetch_tensormap(mapK);
-        prefetch_tensormap(mapV);
-        mbar_arrive_expect_tx(full_q, C::kQBytes);
-        for (int s = 0; s < NSLOT; ++s)
-          for (int cc = 0; cc < D / 64; ++cc)
-            for (int hh = 0; hh < 2; ++hh)
-              tma_load_4d(smem + C::kQ + s * C::kTile + cc * kChunkBytes + hh * (kChunkBytes / 2),
-                          &p.tmQ[map_idx], full_q, cc * 64, head[s],
-                          box_row(qt * kTileM + hh * 64), b);
       }
-      int last_k = -1, last_v = -1;  // last tiles whose loads were issued
-      for (int it = 0; it < n_tiles; ++it) {
+      // last tiles whose loads were issued (the first n_early already are)
+      int last_k = n_early - 1, last_v = n_early - 1;
+      for (int it = n_early; it < n_tiles; ++it) {
         const int st = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         for (int kv = 0; kv < 2; ++kv) {  // 0: K, 1: V
@@ -318,24 +352,9 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
           uint8_t* dst = smem + C::kRing + st * C::kStageBytes + kv * NSTREAM * C::kTile;
           if (it >= kStages && !mbar_wait(emp, ph ^ 1u, p.err, abort_flag)) goto producer_done;
           (kv ? last_v : last_k) = it;
-#ifdef SWA_TEST_WITHHOLD_TILE
-          // failure-detection test build only: this K tile is never loaded,
-          // so the MMA issuer's bounded wait for it runs out
-          if (kv == 0 && it == SWA_TEST_WITHHOLD_TILE) continue;
-#endif
+          if (withheld(it, kv)) continue;
           if (!glob || it < n_band) {
-            if (lane == 0) {
-              const CUtensorMap* m = kv ? mapV : mapK;
-              const int t = tr.kv_begin + it;
-              mbar_arrive_expect_tx(ful, NSTREAM * C::kTile);
-              for (int s = 0; s < NSTREAM; ++s)
-                for (int cc = 0; cc < D / 64; ++cc)
-                  for (int hh = 0; hh < 2; ++hh) {
-                    const int vrow = t * kTileN + hh * 64;
-                    tma_load_4d(dst + s * C::kTile + cc * kChunkBytes + hh * (kChunkBytes / 2), m,
-                                ful, cc * 64, kvh[s], gitem ? vrow : box_row(vrow), b);
-                  }
-            }
+            if (lane == 0) load_kv(it, kv);
           } else {
             // gather global-key rows with plain 16-byte loads into the
             // swizzled layout the MMA expects
@@ -787,21 +806,27 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       const float inv = 1.f / l;
       const size_t orow_i = qwin ? (size_t)b * Mq + m_row : (size_t)b * p.N + i_phys;
       uint16_t* orow = p.out + (orow_i * p.H + h) * D;
+      // 64 columns of O per TMEM round trip (two loads, one wait)
 #pragma unroll
-      for (int j = 0; j < D / 32; ++j) {
-        uint32_t v[32];
+      for (int j2 = 0; j2 < D / 64; ++j2) {
+        uint32_t v[2][32];
         __syncwarp();
-        tmem_ld32(tO + j * 32, v);
+        tmem_ld32(tO + j2 * 64, v[0]);
+        tmem_ld32(tO + j2 * 64 + 32, v[1]);
         tmem_wait_ld();
-        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
-        if (row_valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + j * 32);
+        for (int jj = 0; jj < 2; ++jj) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(v[jj][2 * e]) * inv,
+                                __uint_as_float(v[jj][2 * e + 1]) * inv);
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + j2 * 64 + jj * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
         }
       }
       if (row_valid && p.lse)
