@@ -618,10 +618,12 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       return max3f(max3f(t[0], t[1], t[2]), max3f(t[3], t[4], t[5]), fmaxf(t[6], t[7]));
     };
     // P = 2^(s * scale * log2 e - m_ref) for one key half, stored as 32
-    // columns of bf16 pairs from TMEM column pcol.  Seven of every eight
-    // column pairs go to the MUFU ex2 unit and one to the FMA pipe
-    // (polynomial), which takes some load off MUFU (measured best of 0, 1/8,
-    // 1/4 and 1/2 on the FMA pipe with the split PV and the register split).
+    // columns of bf16 pairs from TMEM column pcol.  At D = 128 seven of
+    // every eight column pairs go to the MUFU ex2 unit and one to the FMA
+    // pipe (polynomial), which takes some load off MUFU (measured best of 0,
+    // 1/8, 1/4 and 1/2 on the FMA pipe with the split PV and the register
+    // split); at D = 64 all go to MUFU (1/8 and 1/4 measured 1-4 % slower
+    // on the one-head form).
     auto exp_half = [&](int pcol, const float (&sv)[64], float m_ref, float2 (&ls)[4]) {
       const float2 sl2_2 = make_float2(sl2, sl2), negm2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
@@ -632,7 +634,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
           const float2 xa =
               fma2(make_float2(sv[jj * 32 + 2 * e], sv[jj * 32 + 2 * e + 1]), sl2_2, negm2);
           float2 pr;
-          if ((e & 7) == 7) {
+          if (D != 64 && (e & 7) == 7) {
             pr = exp2_poly2(xa);
           } else {
             pr.x = ex2_approx(xa.x);
