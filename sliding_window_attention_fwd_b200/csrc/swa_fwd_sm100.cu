@@ -95,6 +95,17 @@ struct FwdParams {
   // positions (v < win - 1 - pos0[b]) are masked.
   const int64_t* pos0;
   int q0, Mq, win;
+  // In place (win % 64 == 0): the keys are read from the ring (tmK[0],
+  // tmV[0]: [B, win, Hkv, D]) and the chunk (tmKf, tmVf: [B, Mq, Hkv, D])
+  // without a staged copy.  Per batch, with s_first = (pos0 - win + 1) mod
+  // win the slot of the window's oldest position and hs = s_first mod 64,
+  // virtual key row v < cs reads ring slot (s_first - hs + v) mod win and
+  // row v >= cs chunk row v - cs, where cs = the multiple of 64 at or above
+  // hs + win - 1: every 64-row box then lies inside one source without
+  // wrapping.  The history sits at rows [hs, hs + win - 1), the rows
+  // [hs + win - 1, cs) between it and the chunk are masked, and chunk row c
+  // (virtual row cs + c) sees rows [hs + c, cs + c].
+  int inplace;
 };
 
 template <int D, int NSLOT, int NSTREAM>
@@ -189,12 +200,24 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
     if (!slot_ok[s]) head[s] = p.H - 1;
     kvh[s] = head[s] / grp;
   }
-  const Geometry g = make_geometry(p.N, p.L, p.R, p.d, p.bs);
-  // a global tile's keys are the physical rows of the sequence
-  const int Mv = gitem ? p.N : p.Mv[cl];
   constexpr bool qwin = KIND == 1;
-  const int Mq = qwin ? p.Mq : Mv;  // query rows (local)
-  const int q0 = qwin ? p.q0 : 0;   // virtual row of local query row 0
+  // in-place query window: per-batch key layout (see FwdParams::inplace)
+  const bool inplace = qwin && p.inplace;
+  int ip_hs = 0, ip_cs = 0, ip_base = 0;
+  if (inplace) {
+    const int W = p.win;
+    long long sf = (p.pos0[b] - W + 1) % W;
+    if (sf < 0) sf += W;
+    ip_hs = (int)sf & 63;
+    ip_cs = ip_hs <= 1 ? W : W + 64;
+    ip_base = (int)sf - ip_hs;  // ring slot of virtual row 0, a multiple of 64
+  }
+  const Geometry g = inplace ? make_geometry(ip_cs + p.Mq, ip_cs - ip_hs, 0, 1, 0)
+                             : make_geometry(p.N, p.L, p.R, p.d, p.bs);
+  // a global tile's keys are the physical rows of the sequence
+  const int Mv = gitem ? p.N : (inplace ? ip_cs + p.Mq : p.Mv[cl]);
+  const int Mq = qwin ? p.Mq : Mv;           // query rows (local)
+  const int q0 = qwin ? (inplace ? ip_cs : p.q0) : 0;  // virtual row of local query row 0
   const int qm0 = q0 + qt * kTileM;
   const int qm1 = q0 + min(qt * kTileM + kTileM - 1, Mq - 1);
   TileRange tr;
@@ -210,9 +233,11 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
   int lo_b = 0;  // first key row holding a real position (query window only)
   if (qwin) {
     const long long pb = p.pos0[b];
-    const long long lb = (long long)(p.win - 1) - pb;
-    lo_b = lb <= 0 ? 0 : (lb > Mv ? Mv : (int)lb);
+    const long long lb = (long long)(p.win - 1) - pb + ip_hs;
+    lo_b = lb <= ip_hs ? ip_hs : (lb > Mv ? Mv : (int)lb);
   }
+  // in place: the masked rows between the history and the chunk
+  const int gap_lo = inplace ? ip_hs + p.win - 1 : 0, gap_hi = inplace ? ip_cs : 0;
   const int n_band = tr.kv_end - tr.kv_begin;
   const int n_gtiles = (!glob || gitem) ? 0 : (p.n_global + kTileN - 1) / kTileN;
   const int n_tiles = n_band + n_gtiles;
@@ -225,6 +250,20 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
   };
   const CUtensorMap* mapK = gitem ? &p.tmKf : &p.tmK[map_idx];
   const CUtensorMap* mapV = gitem ? &p.tmVf : &p.tmV[map_idx];
+  // the source of a 64-row key box at virtual row vrow (a multiple of 64):
+  // its tensor map and row coordinate
+  auto kv_box = [&](int kv, int vrow, int* row) -> const CUtensorMap* {
+    if (inplace) {
+      if (vrow < ip_cs) {
+        *row = (ip_base + vrow) % p.win;
+        return kv ? &p.tmV[0] : &p.tmK[0];
+      }
+      *row = vrow - ip_cs;
+      return kv ? &p.tmVf : &p.tmKf;
+    }
+    *row = gitem ? vrow : box_row(vrow);
+    return kv ? mapV : mapK;
+  };
   // TMA loads (one thread): the Q tiles, and K or V of band tile it
   auto load_q = [&]() {
     prefetch_tensormap(&p.tmQ[map_idx]);
@@ -240,16 +279,16 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
     const int st = it % kStages;
     uint64_t* ful = kv ? &full_v[st] : &full_k[st];
     uint8_t* dst = smem + C::kRing + st * C::kStageBytes + kv * NSTREAM * C::kTile;
-    const CUtensorMap* m = kv ? mapV : mapK;
     const int t = tr.kv_begin + it;
     mbar_arrive_expect_tx(ful, NSTREAM * C::kTile);
-    for (int s = 0; s < NSTREAM; ++s)
-      for (int cc = 0; cc < D / 64; ++cc)
-        for (int hh = 0; hh < 2; ++hh) {
-          const int vrow = t * kTileN + hh * 64;
+    for (int hh = 0; hh < 2; ++hh) {
+      int row;
+      const CUtensorMap* m = kv_box(kv, t * kTileN + hh * 64, &row);
+      for (int s = 0; s < NSTREAM; ++s)
+        for (int cc = 0; cc < D / 64; ++cc)
           tma_load_4d(dst + s * C::kTile + cc * kChunkBytes + hh * (kChunkBytes / 2), m, ful,
-                      cc * 64, kvh[s], gitem ? vrow : box_row(vrow), b);
-        }
+                      cc * 64, kvh[s], row, b);
+    }
   };
 #ifdef SWA_TEST_WITHHOLD_TILE
   // failure-detection test build only: this K tile is never loaded, so the
@@ -288,6 +327,10 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
     if (!gitem) {
       prefetch_tensormap(mapK);
       prefetch_tensormap(mapV);
+      if (inplace) {
+        prefetch_tensormap(&p.tmKf);
+        prefetch_tensormap(&p.tmVf);
+      }
       load_q();
       for (int it = 0; it < n_early; ++it)
         for (int kv = 0; kv < 2; ++kv)
@@ -525,6 +568,9 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
     } else {
       row_valid = m_row < Mq && slot_ok[slot];
       klo = max(key_lo(g, m_v), lo_b);
+      // in place: a window that starts past the history starts in the
+      // chunk, beyond the masked rows between the two
+      if (inplace && klo >= gap_lo) klo += gap_hi - gap_lo;
       khi = key_hi(g, m_v, Mv);
       i_phys = (int)phys_row(g, c, m_v);
       // a global row is written by its global tile, not by the band
@@ -561,7 +607,11 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
     float m_pend = -INFINITY;  // max seen but not yet adopted (adopted next tile)
     int int_lo, int_hi;        // key tiles that need no element mask
     interior_tiles_rows(g, Mv, qm0, &int_lo, &int_hi);
-    if (gitem || lo_b > 0 || qt * kTileM + kTileM > Mq) int_hi = int_lo - 1;  // mask every tile
+    // mask every tile: global tiles, rows of negative positions, partial
+    // query tiles, and in-place windows that start in the chunk
+    if (gitem || lo_b > ip_hs || qt * kTileM + kTileM > Mq ||
+        (inplace && qt * kTileM + kTileM - 1 >= p.win - 1))
+      int_hi = int_lo - 1;
 
     // the 64 score columns of key half hf (TMEM -> registers)
     auto read_half = [&](int hf, float (&sv)[64]) {
@@ -585,6 +635,10 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
           const int lo = max(klo - n0, 0);
           const int hi = min(min(khi, Mv - 1) - n0, 63);  // inclusive
           keep = hi < lo ? 0ull : ((~0ull >> (63 - hi)) & (~0ull << lo));
+          if (inplace) {
+            const int a = max(gap_lo - n0, 0), z = min(gap_hi - n0, 64);  // [a, z)
+            if (a < z) keep &= ~((z >= 64 ? ~0ull : ((1ull << z) - 1ull)) & (~0ull << a));
+          }
         }
       } else {
         // a global key joins the row unless it is already in the row's band
@@ -691,7 +745,8 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       const int e = it & 1;  // early key half; P of the tile lives in its columns
       const uint32_t ph = (uint32_t)it & 1u;
       const int t_kv = tr.kv_begin + it;
-      const bool edge = (!glob || it < n_band) && !(t_kv >= int_lo && t_kv <= int_hi);
+      const bool edge = ((!glob || it < n_band) && !(t_kv >= int_lo && t_kv <= int_hi)) ||
+                        (inplace && t_kv * kTileN < gap_hi && t_kv * kTileN + kTileN > gap_lo);
 
       // adopt a larger max seen on the previous tile (rare after the start)
       const bool pend = m_pend > m_used;
@@ -921,11 +976,13 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
       p.qt_base = lo;
       p.qtile_prefix[1] = hi - lo;
     }
+    const bool inplace = qw && qw->kn;
     if (qw) {
       p.pos0 = qw->pos0;
       p.q0 = qw->q0;
       p.Mq = qw->Mq;
       p.win = qw->win;
+      p.inplace = inplace ? 1 : 0;
     }
     const uint32_t box[4] = {64, 1, (uint32_t)kBlockRows, 1};
     const int nmaps = block_mode ? 1 : p.nclass;
@@ -939,8 +996,11 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
       const uint64_t qN = qw ? (uint64_t)qw->Mq : (uint64_t)N;
       const uint64_t dq[4] = {(uint64_t)D, (uint64_t)H, qrows, (uint64_t)B};
       const uint64_t sq[3] = {(uint64_t)D * 2, rstep * H * D * 2, qN * H * D * 2};
-      const uint64_t dk[4] = {(uint64_t)D, (uint64_t)Hkv, rows, (uint64_t)B};
-      const uint64_t sk[3] = {(uint64_t)D * 2, rstep * Hkv * D * 2, (uint64_t)N * Hkv * D * 2};
+      // in place: K / V are the rings, win rows per batch
+      const uint64_t krows = inplace ? (uint64_t)qw->win : rows;
+      const uint64_t kN = inplace ? (uint64_t)qw->win : (uint64_t)N;
+      const uint64_t dk[4] = {(uint64_t)D, (uint64_t)Hkv, krows, (uint64_t)B};
+      const uint64_t sk[3] = {(uint64_t)D * 2, rstep * Hkv * D * 2, kN * Hkv * D * 2};
       void* qb = (void*)(static_cast<const uint16_t*>(q) + qoff);
       void* kb = (void*)(static_cast<const uint16_t*>(k) + kvoff);
       void* vb = (void*)(static_cast<const uint16_t*>(v) + kvoff);
@@ -950,6 +1010,17 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
                        CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
           encode_tiled(&p.tmV[cl], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, vb, dk, sk, box,
                        CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+        return SWA_ERR_CUDA;
+    }
+    if (inplace) {
+      // the chunk's keys and values, [B, Mq, Hkv, D]
+      const uint64_t dn[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)qw->Mq, (uint64_t)B};
+      const uint64_t sn[3] = {(uint64_t)D * 2, (uint64_t)Hkv * D * 2,
+                              (uint64_t)qw->Mq * Hkv * D * 2};
+      if (encode_tiled(&p.tmKf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(qw->kn),
+                       dn, sn, box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS ||
+          encode_tiled(&p.tmVf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(qw->vn),
+                       dn, sn, box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return SWA_ERR_CUDA;
     }
     // the global tiles ride with the first launch

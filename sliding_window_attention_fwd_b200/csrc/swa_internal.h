@@ -52,6 +52,12 @@ int launch_fwd_f32(const float* q, const float* k, const float* v, float* out, f
 struct QueryWindow {
   const int64_t* pos0;
   int q0, Mq, win;
+  // In place (chunked append with win % 64 == 0): k / v passed to the
+  // launch are the rings [B, win, Hkv, D] and kn / vn the chunk [B, Mq, Hkv,
+  // D]; the kernel lays the keys out per batch (see swa_fwd_sm100.cu) and
+  // q0 is not used.  Otherwise k / v hold the staged key sequence.
+  const void* kn = nullptr;
+  const void* vn = nullptr;
 };
 // qt_lo / qt_hi (token-level, d == 1, no query window): launch only the
 // query tiles [qt_lo, qt_hi) of the sequence (qt_hi < 0: all).

@@ -810,14 +810,24 @@ int ring_store(const void* k_new, const void* v_new, void* k_ring, void* v_ring,
 }  // namespace
 
 namespace {
-// Chunks of 32 tokens and more: stage the chunk's key sequence contiguously
-// (ring history below pos0, then the chunk) and run the tcgen05 forward
-// over it with a causal window of W keys, its queries being the last C
-// rows.  Shorter chunks would leave most of a 128-row query tile idle and
-// take the row kernel below.
+// Chunks of 32 tokens and more: the tcgen05 forward with a causal window of
+// W keys over the ring history below pos0 followed by the chunk, its
+// queries being the chunk's C rows.  With W a multiple of 64 it reads the
+// ring and the chunk in place; otherwise it first stages the key sequence
+// contiguously.  Shorter chunks would leave most of a 128-row query tile
+// idle and take the row kernel below.
 int append_attention_tc(const void* q, const void* k_new, const void* v_new, const void* k_ring,
                         const void* v_ring, void* out, float* lse, const int64_t* pos0, int B,
                         int C, int H, int Hkv, int D, int W, float scale, cudaStream_t stream) {
+  if (W % 64 == 0 && (long long)W + 64 + C <= 0x7fffffffLL) {
+    // read the ring and the chunk in place: every 64-row key box then lies
+    // inside one of them (the kernel's per-batch layout), no staged copy
+    QueryWindow qw{pos0, 0, C, W};
+    qw.kn = k_new;
+    qw.vn = v_new;
+    return launch_fwd_sm100(q, k_ring, v_ring, out, lse, B, H, Hkv, W + 64 + C, D, W - 1, 0, 1,
+                            0, nullptr, 0, scale, stream, &qw);
+  }
   const long long Nv = (long long)W - 1 + C;
   if (Nv > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
   const size_t half = (size_t)B * Nv * Hkv * D * 2;

@@ -138,6 +138,11 @@ def test_append_configs(swa, name):
     (2, 40, 4, 4, 64, 128, [100, 3]),              # MHA, D = 64, tensor-core path
     (1, 33, 2, 2, 128, 64, [70]),                  # MHA, D = 128, tensor-core path
     (2, 130, 6, 2, 128, 192, [5, 1000]),           # GQA 3, two query tiles
+    # ring read in place (W % 64 == 0): the window's oldest slot at every
+    # offset class within a 64-row box (0, 1, 2, 63), windows that start
+    # inside the chunk (C > W), positions below W
+    (3, 100, 4, 2, 128, 64, [62, 63, 65]),
+    (2, 150, 4, 4, 64, 128, [129, 64]),
 ])
 def test_append_shapes(swa, B, C, H, Hkv, D, W, pos0):
     q = inputs.normal((B, C, H, D), C + W, 0)
