@@ -11,8 +11,7 @@
  * launched: on failure the call returns a negative swa_status and launches
  * nothing.  No call synchronises the stream; swa_device_error() does.
  * Library-owned device workspaces (split partials of the decode / global
- * row / paged / append kernels, the staged keys of a long append, the
- * backward's accumulators) are one per device and per use: two calls that
+ * row / paged / append kernels, the backward's accumulators) are one per device and per use: two calls that
  * use the same one must not run on the device at the same time, whichever
  * streams they are on.  Workspaces grow on demand (the growing call
  * synchronises its stream first) and are freed by swa_release().
@@ -360,10 +359,11 @@ SWA_API int swa_paged_window(int64_t pos, int W, int page_size, int64_t* first_p
  * taking positions >= pos0 from the chunk and the others from the ring as
  * it was before the call.  W must be a positive multiple of 64; 1 <= C <=
  * 65535; D in {64, 128}; H % Hkv == 0, H / Hkv <= 8; scale <= 0 means
- * 1/sqrt(D).  Launches on `stream`: for C >= 32 a staging copy (the
- * window's history, de-rotated, followed by the chunk, into a library
- * workspace), the tensor-core attention over it and the ring update; for
- * shorter chunks the row-kernel attention and the ring update.
+ * 1/sqrt(D).  Launches on `stream`: for C >= 32 the tensor-core attention
+ * reading ring and chunk in place (when its work items do not fill the
+ * SMs, each key walk is split over several CTAs whose partial results go
+ * to a library workspace and are merged by a second kernel), then the ring
+ * update; for shorter chunks the row-kernel attention and the ring update.
  * Workspace, streams and graphs as for swa_decode.
  */
 SWA_API int swa_append(const void* q, const void* k_new, const void* v_new, void* k_ring,

@@ -106,6 +106,19 @@ struct FwdParams {
   // [hs + win - 1, cs) between it and the chunk are masked, and chunk row c
   // (virtual row cs + c) sees rows [hs + c, cs + c].
   int inplace;
+  // Stacked heads (query window, two slots, Mq <= 64, GQA group a multiple
+  // of 4): a slot's 128-row tile holds two heads of the group, rows 0-63
+  // the first one's tokens and rows 64-127 the second one's, so the four
+  // heads of a CTA share one key walk with no empty query rows.
+  int stack;
+  // Split key walks (query window): each item's key tiles are cut into
+  // nsplit contiguous parts, one CTA each, which write O / l (fp32) and
+  // lse to part_o [nsplit, B, H, Mq, D] and part_lse [nsplit, B, H, Mq];
+  // a merge kernel combines them.  nsplit == 1: the output is written
+  // directly.
+  int nsplit;
+  float* part_o;
+  float* part_lse;
 };
 
 template <int D, int NSLOT, int NSTREAM>
@@ -171,11 +184,18 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
 
   // ---- work item: the global tiles first (each walks the whole sequence),
   // then (class, q tile, batch, head pair) with heavy (late) tiles first
-  const int npair = (p.H + NSLOT - 1) / NSLOT;
+  constexpr bool qwin = KIND == 1;
+  const bool stack = qwin && NSLOT == 2 && p.stack;
+  const int npair = stack ? p.H / (2 * NSLOT) : (p.H + NSLOT - 1) / NSLOT;
   int x = blockIdx.x;
   constexpr bool glob = KIND == 2;
   const bool gitem = glob && x < p.n_gitems;
   if (glob && !gitem) x -= p.n_gitems;
+  int sp = 0;  // part of a split key walk
+  if (qwin) {
+    sp = x % p.nsplit;
+    x /= p.nsplit;
+  }
   const int hp = x % npair;
   x /= npair;
   const int b = x % p.B;
@@ -195,12 +215,12 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
   bool slot_ok[NSLOT];
 #pragma unroll
   for (int s = 0; s < NSLOT; ++s) {
-    head[s] = hp * NSLOT + s;
+    // stacked: slot s holds heads head[s] (rows 0-63) and head[s] + 1
+    head[s] = stack ? hp * 2 * NSLOT + 2 * s : hp * NSLOT + s;
     slot_ok[s] = head[s] < p.H;
     if (!slot_ok[s]) head[s] = p.H - 1;
     kvh[s] = head[s] / grp;
   }
-  constexpr bool qwin = KIND == 1;
   // in-place query window: per-batch key layout (see FwdParams::inplace)
   const bool inplace = qwin && p.inplace;
   int ip_hs = 0, ip_cs = 0, ip_base = 0;
@@ -216,7 +236,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
                              : make_geometry(p.N, p.L, p.R, p.d, p.bs);
   // a global tile's keys are the physical rows of the sequence
   const int Mv = gitem ? p.N : (inplace ? ip_cs + p.Mq : p.Mv[cl]);
-  const int Mq = qwin ? p.Mq : Mv;           // query rows (local)
+  const int Mq = qwin ? p.Mq : Mv;           // query rows (local; stacked: tokens)
   const int q0 = qwin ? (inplace ? ip_cs : p.q0) : 0;  // virtual row of local query row 0
   const int qm0 = q0 + qt * kTileM;
   const int qm1 = q0 + min(qt * kTileM + kTileM - 1, Mq - 1);
@@ -229,6 +249,14 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
     tr.kv_end = p.R == 0 ? last / kTileN + 1 : (p.N + kTileN - 1) / kTileN;
   } else {
     tr = tile_range_rows(g, Mv, qm0, qm1);
+    if (qwin && p.nsplit > 1) {
+      // this CTA's part of the key walk
+      const int n = tr.kv_end - tr.kv_begin;
+      const int part = (n + p.nsplit - 1) / p.nsplit;
+      const int a = tr.kv_begin + sp * part;
+      tr.kv_begin = min(a, tr.kv_end);
+      tr.kv_end = min(a + part, tr.kv_end);
+    }
   }
   int lo_b = 0;  // first key row holding a real position (query window only)
   if (qwin) {
@@ -272,8 +300,8 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       for (int cc = 0; cc < D / 64; ++cc)
         for (int hh = 0; hh < 2; ++hh)
           tma_load_4d(smem + C::kQ + s * C::kTile + cc * kChunkBytes + hh * (kChunkBytes / 2),
-                      &p.tmQ[map_idx], full_q, cc * 64, head[s], box_row(qt * kTileM + hh * 64),
-                      b);
+                      &p.tmQ[map_idx], full_q, cc * 64, head[s] + (stack ? hh : 0),
+                      stack ? 0 : box_row(qt * kTileM + hh * 64), b);
   };
   auto load_kv = [&](int it, int kv) {
     const int st = it % kStages;
@@ -324,7 +352,9 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       mbar_init(&oe_done[s], 1);
     }
     fence_mbar_init();
-    if (!gitem) {
+    // (an empty part of a split key walk loads nothing: no copy may still
+    // be landing in shared memory when the CTA exits)
+    if (!gitem && n_tiles > 0) {
       prefetch_tensormap(mapK);
       prefetch_tensormap(mapV);
       if (inplace) {
@@ -552,8 +582,9 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + 128u * slot + lane_off;
     const uint32_t tO = tmem + C::kOcol + (uint32_t)D * slot + lane_off;
-    const int h = head[slot];
-    const int m_row = qt * kTileM + r;  // local query row
+    // stacked: lanes 64-127 are the slot's second head, same tokens
+    const int h = head[slot] + (stack ? (r >> 6) : 0);
+    const int m_row = stack ? (r & 63) : qt * kTileM + r;  // local query row
     const int m_v = q0 + m_row;         // its virtual row among the keys
     bool row_valid;
     int klo, khi, i_phys;
@@ -606,11 +637,14 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
 
     float m_pend = -INFINITY;  // max seen but not yet adopted (adopted next tile)
     int int_lo, int_hi;        // key tiles that need no element mask
-    interior_tiles_rows(g, Mv, qm0, &int_lo, &int_hi);
+    // (stacked: from the tokens' rows, conservatively as if they were the
+    // last 128 rows below the last token)
+    interior_tiles_rows(g, Mv, stack ? q0 + Mq - kTileM : qm0, &int_lo, &int_hi);
+    const int last_row = stack ? Mq - 1 : qt * kTileM + kTileM - 1;  // local
     // mask every tile: global tiles, rows of negative positions, partial
     // query tiles, and in-place windows that start in the chunk
-    if (gitem || lo_b > ip_hs || qt * kTileM + kTileM > Mq ||
-        (inplace && qt * kTileM + kTileM - 1 >= p.win - 1))
+    if (gitem || lo_b > ip_hs || (stack ? Mq < 64 : qt * kTileM + kTileM > Mq) ||
+        (inplace && last_row >= p.win - 1))
       int_hi = int_lo - 1;
 
     // the 64 score columns of key half hf (TMEM -> registers)
@@ -856,11 +890,22 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       mbar_arrive(&p_full[slot]);
     }
 
+    // split key walk: this CTA's part goes to the partials (fp32 O / l and
+    // lse); an empty part contributes nothing (lse = -inf)
+    const bool split = qwin && p.nsplit > 1;
+    const size_t prow = (((size_t)sp * p.B + b) * p.H + h) * (size_t)Mq + m_row;
+    if (split && ok && n_tiles == 0 && row_valid && !warp_idle) {
+      float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D);
+      for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      p.part_lse[prow] = -INFINITY;
+    }
     bool fin = ok && n_tiles > 0 && !warp_idle;
     if (fin) fin = mbar_wait(&o_final[slot], 0, p.err, abort_flag);
     if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
-      const float inv = 1.f / l;
+      // (l == 0: a part of a split walk with none of the row's keys; its
+      // lse is -inf and the merge skips it)
+      const float inv = l > 0.f ? 1.f / l : 0.f;
       const size_t orow_i = qwin ? (size_t)b * Mq + m_row : (size_t)b * p.N + i_phys;
       uint16_t* orow = p.out + (orow_i * p.H + h) * D;
       // 64 columns of O per TMEM round trip (two loads, one wait)
@@ -871,6 +916,18 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
         tmem_ld32(tO + j2 * 64, v[0]);
         tmem_ld32(tO + j2 * 64 + 32, v[1]);
         tmem_wait_ld();
+        if (split) {
+          if (row_valid) {
+            float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D + j2 * 64);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              dst[e] = make_float4(__uint_as_float(v[e >> 3][(e & 7) * 4]) * inv,
+                                   __uint_as_float(v[e >> 3][(e & 7) * 4 + 1]) * inv,
+                                   __uint_as_float(v[e >> 3][(e & 7) * 4 + 2]) * inv,
+                                   __uint_as_float(v[e >> 3][(e & 7) * 4 + 3]) * inv);
+          }
+          continue;
+        }
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
           uint32_t pk[16];
@@ -886,9 +943,11 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
           }
         }
       }
-      if (row_valid && p.lse)
-        p.lse[((size_t)b * p.H + h) * (qwin ? Mq : p.N) + (qwin ? m_row : i_phys)] =
-            (m_used + __log2f(l)) * 0.69314718055994531f;
+      const float lse_v = (m_used + __log2f(l)) * 0.69314718055994531f;
+      if (row_valid && split)
+        p.part_lse[prow] = lse_v;
+      else if (row_valid && p.lse)
+        p.lse[((size_t)b * p.H + h) * (qwin ? Mq : p.N) + (qwin ? m_row : i_phys)] = lse_v;
     }
   }
 
@@ -983,6 +1042,13 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
       p.Mq = qw->Mq;
       p.win = qw->win;
       p.inplace = inplace ? 1 : 0;
+      p.stack = (NSLOT == 2 && qw->stack) ? 1 : 0;
+      p.nsplit = qw->nsplit > 1 ? qw->nsplit : 1;
+      if (p.nsplit > 1) {
+        if (!qw->part) return SWA_ERR_ARG;
+        p.part_o = qw->part;
+        p.part_lse = qw->part + (size_t)p.nsplit * B * H * qw->Mq * D;
+      }
     }
     const uint32_t box[4] = {64, 1, (uint32_t)kBlockRows, 1};
     const int nmaps = block_mode ? 1 : p.nclass;
@@ -1036,8 +1102,10 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
                        box, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
         return SWA_ERR_CUDA;
     }
-    const long grid = (long)p.n_gitems +
-                      (long)p.qtile_prefix[p.nclass] * B * ((H + NSLOT - 1) / NSLOT);
+    const long heads_per_item = p.stack ? 2 * NSLOT : NSLOT;
+    const long grid = (long)p.n_gitems + (long)p.qtile_prefix[p.nclass] * B *
+                                             ((H + heads_per_item - 1) / heads_per_item) *
+                                             (qw ? p.nsplit : 1);
     if (grid <= 0) continue;
     if (grid > 0x7fffffffL) return SWA_ERR_UNSUPPORTED;
     if (kind == 1)
@@ -1055,6 +1123,11 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
 }
 
 }  // namespace
+
+bool fwd_qwin_stacks(int H, int Hkv, int Mq) {
+  const int grp = H / Hkv;
+  return grp % 4 == 0 && Mq <= 64;  // two slots (even group), four heads per CTA
+}
 
 // Two query heads per CTA when they share a kv head (GQA group of even
 // size); otherwise one head per CTA, two CTAs per SM at D = 64 (measured on

@@ -55,10 +55,21 @@ struct QueryWindow {
   // In place (chunked append with win % 64 == 0): k / v passed to the
   // launch are the rings [B, win, Hkv, D] and kn / vn the chunk [B, Mq, Hkv,
   // D]; the kernel lays the keys out per batch (see swa_fwd_sm100.cu) and
-  // q0 is not used.  Otherwise k / v hold the staged key sequence.
+  // q0 is not used.  Otherwise k / v hold the key sequence contiguously
+  // (row v: position pos0 - (win - 1) + v) and the queries sit at rows q0..
   const void* kn = nullptr;
   const void* vn = nullptr;
+  // stack: two heads per 128-row tile (Mq <= 64, two slots, GQA group a
+  // multiple of 4); nsplit > 1: split key walks whose partials go to part
+  // (nsplit * B * H * Mq * (D + 1) floats: O / l, then lse) for a merge.
+  int stack = 0;
+  int nsplit = 1;
+  float* part = nullptr;
 };
+// Whether the forward for a query window of Mq rows would stack two heads
+// per tile (the launch's slot count follows the GQA group as in
+// launch_fwd_sm100).
+bool fwd_qwin_stacks(int H, int Hkv, int Mq);
 // qt_lo / qt_hi (token-level, d == 1, no query window): launch only the
 // query tiles [qt_lo, qt_hi) of the sequence (qt_hi < 0: all).
 int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, float* lse,

@@ -550,7 +550,7 @@ __global__ void __launch_bounds__(kThreadsR, (NQ <= 4 ? 3 : 1))
 
 // ------------------------------------------------------------ workspaces
 // Per device and per user (0: decode, 1: unused, 2: paged decode,
-// 3: chunked append, 4: the staged key sequence of a tensor-core append):
+// 3: chunked append, 4: the split partials of a tensor-core append):
 // split counters and
 // split partials in separate buffers.  Every merge resets its counter to
 // zero, so between complete calls all counters are zero; the counter buffer
@@ -563,7 +563,7 @@ struct Workspace {
   size_t part_bytes = 0;
 };
 constexpr int kMaxDev = 64;
-Workspace g_ws[kMaxDev][5];  // users: decode, (unused), paged, append, append staging
+Workspace g_ws[kMaxDev][5];  // users: decode, (unused), paged, append, tensor-core append
 std::mutex g_ws_mu;
 
 bool get_workspace(int which, size_t cnt_bytes, size_t part_bytes, cudaStream_t stream,
@@ -693,36 +693,51 @@ __global__ void ring_store_kernel(const uint4* __restrict__ k_new, const uint4* 
   v_ring[dst] = v_new[src];
 }
 
-// Stages the key / value sequence of a chunked append for the tensor-core
-// forward: row v holds position pos0[b] - (W - 1) + v, taken from the ring
-// (slot position % W) below pos0 and from the chunk from pos0 on; rows of
-// negative positions are zeros (the forward masks them).  16 B per thread.
-__global__ void append_stage_kernel(const uint4* __restrict__ k_ring,
-                                    const uint4* __restrict__ v_ring,
-                                    const uint4* __restrict__ k_new,
-                                    const uint4* __restrict__ v_new, uint4* __restrict__ ks,
-                                    uint4* __restrict__ vs, const int64_t* __restrict__ pos0,
-                                    int B, int C, int W, int Nv, int row_vecs) {
-  const long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= (long long)B * Nv * row_vecs) return;
-  const int i = (int)(t % row_vecs);
-  const int v = (int)((t / row_vecs) % Nv);
-  const int b = (int)(t / ((long long)row_vecs * Nv));
-  const long long p0 = pos0[b];
-  const long long pos = p0 - (W - 1) + v;
-  uint4 kk = make_uint4(0u, 0u, 0u, 0u), vv = kk;
-  if (pos >= p0) {
-    const long src = ((long)b * C + (pos - p0)) * row_vecs + i;
-    kk = k_new[src];
-    vv = v_new[src];
-  } else if (pos >= 0) {
-    const long src = ((long)b * W + pos % W) * row_vecs + i;
-    kk = k_ring[src];
-    vv = v_ring[src];
+// Combines the split key walks of a chunked append: row (b, c, h) has
+// nsplit partial results O_i / l_i (fp32) with lse_i; with m = max lse_i
+// and w_i = exp(lse_i - m), out = sum w_i O_i / sum w_i (bf16) and lse = m +
+// ln sum w_i (the lse identity of split softmax).  One warp per row, D / 32
+// columns per lane.
+template <int D>
+__global__ void __launch_bounds__(256) append_merge_kernel(const float* __restrict__ part_o,
+                                                           const float* __restrict__ part_lse,
+                                                           uint16_t* __restrict__ out,
+                                                           float* __restrict__ lse, int nsplit,
+                                                           int B, int C, int H) {
+  constexpr int kPer = D / 32;
+  const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const long long rows = (long long)B * H * C;
+  if (row >= rows) return;
+  // part index ((sp * B + b) * H + h) * C + c = sp * rows + row
+  const int c = (int)(row % C);
+  const long long bh = row / C;  // b * H + h
+  const int h = (int)(bh % H);
+  const int b = (int)(bh / H);
+  float m = -INFINITY;
+  for (int sp = 0; sp < nsplit; ++sp) m = fmaxf(m, part_lse[(long long)sp * rows + row]);
+  float acc[kPer];
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  for (int sp = 0; sp < nsplit; ++sp) {
+    // a part holding none of the row's keys has lse = -inf: skipped
+    const float li = part_lse[(long long)sp * rows + row];
+    if (li == -INFINITY) continue;
+    const float w = __expf(li - m);
+    wsum += w;
+    const float* src = part_o + ((long long)sp * rows + row) * D + lane * kPer;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] += w * src[e];
   }
-  const long dst = ((long)b * Nv + v) * row_vecs + i;
-  ks[dst] = kk;
-  vs[dst] = vv;
+  const float inv = 1.f / wsum;
+  uint16_t* dst = out + (((long long)b * C + c) * H + h) * D + lane * kPer;
+#pragma unroll
+  for (int e = 0; e < kPer; e += 2) {
+    const __nv_bfloat162 v2 = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
+    *reinterpret_cast<__nv_bfloat162*>(dst + e) = v2;
+  }
+  if (lse && lane == 0) lse[bh * C + c] = m + __logf(wsum);
 }
 
 }  // namespace
@@ -810,45 +825,66 @@ int ring_store(const void* k_new, const void* v_new, void* k_ring, void* v_ring,
 }  // namespace
 
 namespace {
+int append_merge(const float* part, void* out, float* lse, int nsplit, int B, int C, int H, int D,
+                 cudaStream_t stream) {
+  const long long rows = (long long)B * H * C;
+  const float* part_lse = part + (size_t)nsplit * rows * D;
+  const long long blocks = (rows + 7) / 8;
+  if (blocks > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  if (D == 128)
+    append_merge_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
+        part, part_lse, static_cast<uint16_t*>(out), lse, nsplit, B, C, H);
+  else
+    append_merge_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
+        part, part_lse, static_cast<uint16_t*>(out), lse, nsplit, B, C, H);
+  return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
+}
+
 // Chunks of 32 tokens and more: the tcgen05 forward with a causal window of
-// W keys over the ring history below pos0 followed by the chunk, its
-// queries being the chunk's C rows.  With W a multiple of 64 it reads the
-// ring and the chunk in place; otherwise it first stages the key sequence
-// contiguously.  Shorter chunks would leave most of a 128-row query tile
-// idle and take the row kernel below.
+// W keys over the ring history below pos0 followed by the chunk (both read
+// in place), its queries being the chunk's C rows.  Shorter chunks would
+// leave most of a 128-row query tile idle and take the row kernel below.
 int append_attention_tc(const void* q, const void* k_new, const void* v_new, const void* k_ring,
                         const void* v_ring, void* out, float* lse, const int64_t* pos0, int B,
                         int C, int H, int Hkv, int D, int W, float scale, cudaStream_t stream) {
-  if (W % 64 == 0 && (long long)W + 64 + C <= 0x7fffffffLL) {
-    // read the ring and the chunk in place: every 64-row key box then lies
-    // inside one of them (the kernel's per-batch layout), no staged copy
-    QueryWindow qw{pos0, 0, C, W};
-    qw.kn = k_new;
-    qw.vn = v_new;
-    return launch_fwd_sm100(q, k_ring, v_ring, out, lse, B, H, Hkv, W + 64 + C, D, W - 1, 0, 1,
-                            0, nullptr, 0, scale, stream, &qw);
+  // Work items: query tiles x head groups (four heads per CTA when two are
+  // stacked per tile, else two or one); when they do not fill the SMs the
+  // key walks are split (the partials merged after), at least two key
+  // tiles per part.
+  int nsm = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || nsm <= 0)
+    return SWA_ERR_CUDA;
+  const int grp = H / Hkv;
+  const bool stack = fwd_qwin_stacks(H, Hkv, C);
+  const int per_cta = stack ? 4 : (grp % 2 == 0 ? 2 : 1);
+  const long long items = (long long)B * ((H + per_cta - 1) / per_cta) * ((C + 127) / 128);
+  const int per_sm = (D == 64 && per_cta == 1) ? 2 : 1;
+  const int walk = (W + C + 127) / 128 + 1;  // key tiles of a query tile, at most
+  int nsplit = (int)((long long)nsm * per_sm / (items > 0 ? items : 1));
+  nsplit = nsplit < 1 ? 1 : (nsplit > 8 ? 8 : nsplit);
+  while (nsplit > 1 && walk / nsplit < 2) --nsplit;
+  QueryWindow qw{pos0, W - 1, C, W};
+  qw.stack = stack ? 1 : 0;
+  qw.nsplit = nsplit;
+  const size_t part_bytes =
+      nsplit > 1 ? (size_t)nsplit * B * H * C * (D + 1) * sizeof(float) : 0;
+  // the ring and the chunk are read in place: with W a multiple of 64
+  // (swa_append requires it) every 64-row key box lies inside one of them
+  // (the kernel's per-batch layout), so no staged copy is needed
+  if (W % 64 != 0 || (long long)W + 64 + C > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  if (part_bytes) {
+    int* cnt = nullptr;
+    void* part = nullptr;
+    if (!get_workspace(4, 256, part_bytes, stream, &cnt, &part)) return SWA_ERR_NOMEM;
+    qw.part = static_cast<float*>(part);
   }
-  const long long Nv = (long long)W - 1 + C;
-  if (Nv > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
-  const size_t half = (size_t)B * Nv * Hkv * D * 2;
-  int* cnt = nullptr;
-  void* part = nullptr;
-  if (!get_workspace(4, 256, 2 * half, stream, &cnt, &part)) return SWA_ERR_NOMEM;
-  uint8_t* ks = static_cast<uint8_t*>(part);
-  uint8_t* vs = ks + half;
-  const int row_vecs = Hkv * D / 8;
-  const long long n = (long long)B * Nv * row_vecs;
-  const long long blocks = (n + 255) / 256;
-  if (blocks > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
-  append_stage_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
-      static_cast<const uint4*>(k_ring), static_cast<const uint4*>(v_ring),
-      static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new),
-      reinterpret_cast<uint4*>(ks), reinterpret_cast<uint4*>(vs), pos0, B, C, W, (int)Nv,
-      row_vecs);
-  if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
-  const QueryWindow qw{pos0, W - 1, C, W};
-  return launch_fwd_sm100(q, ks, vs, out, lse, B, H, Hkv, (int)Nv, D, W - 1, 0, 1, 0, nullptr, 0,
-                          scale, stream, &qw);
+  qw.kn = k_new;
+  qw.vn = v_new;
+  const int st = launch_fwd_sm100(q, k_ring, v_ring, out, lse, B, H, Hkv, W + 64 + C, D, W - 1,
+                                  0, 1, 0, nullptr, 0, scale, stream, &qw);
+  if (st != SWA_OK || nsplit == 1) return st;
+  return append_merge(qw.part, out, lse, nsplit, B, C, H, D, stream);
 }
 }  // namespace
 

@@ -143,6 +143,12 @@ def test_append_configs(swa, name):
     # inside the chunk (C > W), positions below W
     (3, 100, 4, 2, 128, 64, [62, 63, 65]),
     (2, 150, 4, 4, 64, 128, [129, 64]),
+    # four heads per CTA (two stacked per tile, GQA 4 and 8) with split key
+    # walks, one at D = 64, one with positions below W
+    (2, 64, 16, 4, 128, 1024, [5000, 700]),
+    (1, 48, 16, 2, 128, 2048, [3000]),
+    (2, 50, 8, 2, 128, 1024, [1500, 20]),
+    (2, 64, 8, 2, 64, 512, [600, 511]),
 ])
 def test_append_shapes(swa, B, C, H, Hkv, D, W, pos0):
     q = inputs.normal((B, C, H, D), C + W, 0)
