@@ -27,6 +27,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "swa_internal.h"
 #include "swa_ptx.cuh"
@@ -704,7 +705,9 @@ __global__ void __launch_bounds__(256) append_merge_kernel(const float* __restri
                                                            uint16_t* __restrict__ out,
                                                            float* __restrict__ lse, int nsplit,
                                                            int B, int C, int H) {
-  constexpr int kPer = D / 32;
+  constexpr int kPer = D / 32;  // 4 (D = 128) or 2 (D = 64) columns per lane
+  constexpr int kMaxSplit = 8;
+  using Vec = typename std::conditional<kPer == 4, float4, float2>::type;
   const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const long long rows = (long long)B * H * C;
@@ -714,29 +717,41 @@ __global__ void __launch_bounds__(256) append_merge_kernel(const float* __restri
   const long long bh = row / C;  // b * H + h
   const int h = (int)(bh % H);
   const int b = (int)(bh / H);
+  // every load issued before any is used
+  float li[kMaxSplit];
+  Vec o[kMaxSplit];
+#pragma unroll
+  for (int sp = 0; sp < kMaxSplit; ++sp) {
+    if (sp < nsplit) {
+      li[sp] = __ldg(part_lse + (long long)sp * rows + row);
+      o[sp] = __ldg(reinterpret_cast<const Vec*>(part_o + ((long long)sp * rows + row) * D) + lane);
+    }
+  }
   float m = -INFINITY;
-  for (int sp = 0; sp < nsplit; ++sp) m = fmaxf(m, part_lse[(long long)sp * rows + row]);
-  float acc[kPer];
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+  for (int sp = 0; sp < kMaxSplit; ++sp)
+    if (sp < nsplit) m = fmaxf(m, li[sp]);
+  float acc[kPer] = {};
   float wsum = 0.f;
-  for (int sp = 0; sp < nsplit; ++sp) {
-    // a part holding none of the row's keys has lse = -inf: skipped
-    const float li = part_lse[(long long)sp * rows + row];
-    if (li == -INFINITY) continue;
-    const float w = __expf(li - m);
-    wsum += w;
-    const float* src = part_o + ((long long)sp * rows + row) * D + lane * kPer;
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) acc[e] += w * src[e];
+  for (int sp = 0; sp < kMaxSplit; ++sp) {
+    // a part holding none of the row's keys has lse = -inf: skipped
+    if (sp >= nsplit || li[sp] == -INFINITY) continue;
+    const float w = __expf(li[sp] - m);
+    wsum += w;
+    const float* f = reinterpret_cast<const float*>(&o[sp]);
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] += w * f[e];
   }
   const float inv = 1.f / wsum;
   uint16_t* dst = out + (((long long)b * C + c) * H + h) * D + lane * kPer;
+  uint32_t pk[kPer / 2];
 #pragma unroll
-  for (int e = 0; e < kPer; e += 2) {
-    const __nv_bfloat162 v2 = __floats2bfloat162_rn(acc[e] * inv, acc[e + 1] * inv);
-    *reinterpret_cast<__nv_bfloat162*>(dst + e) = v2;
-  }
+  for (int e = 0; e < kPer; e += 2) pk[e / 2] = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+  if (kPer == 4)
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[kPer / 2 - 1]);
+  else
+    *reinterpret_cast<uint32_t*>(dst) = pk[0];
   if (lse && lane == 0) lse[bh * C + c] = m + __logf(wsum);
 }
 
