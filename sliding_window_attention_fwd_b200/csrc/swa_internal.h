@@ -80,6 +80,20 @@ int launch_fwd_sm100(const void* q, const void* k, const void* v, void* out, flo
 int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* out,
                   float* lse, const int64_t* pos, int B, int H, int Hkv, int D, int W,
                   float scale, cudaStream_t stream);
+// The tensor-core decode (D = 128, GQA group <= 8; SWA_ERR_UNSUPPORTED
+// otherwise, launching nothing).
+int launch_decode_tc(const void* q, const void* k_ring, const void* v_ring, void* out,
+                     float* lse, const int64_t* pos, int B, int H, int Hkv, int D, int W,
+                     float scale, cudaStream_t stream);
+// Library workspace `which` (one per device and use) of at least `bytes`.
+bool split_workspace(int which, size_t bytes, cudaStream_t stream, float** part);
+// Tensor map of a [B, rows, Hkv, D] bf16 tensor: 64-column x 64-row boxes,
+// 128-byte swizzle.
+int encode_kv_map(CUtensorMap* m, const void* base, int D, int Hkv, int rows, int B);
+// Merges nsplit partial results: part = O / l [nsplit, B*H*C, D] fp32, then
+// lse [nsplit, B*H*C]; out [B, C, H, D] bf16, lse [B, H, C] (may be NULL).
+int split_merge(const float* part, void* out, float* lse, int nsplit, int B, int C, int H, int D,
+                cudaStream_t stream);
 
 // Decode with its split partials in a fixed file-scope device array (no
 // allocation by the library).

@@ -694,19 +694,20 @@ __global__ void ring_store_kernel(const uint4* __restrict__ k_new, const uint4* 
   v_ring[dst] = v_new[src];
 }
 
-// Combines the split key walks of a chunked append: row (b, c, h) has
-// nsplit partial results O_i / l_i (fp32) with lse_i; with m = max lse_i
+// Combines split key walks (the parts of a tensor-core append or decode):
+// row (b, c, h) has nsplit partial results O_i / l_i (fp32) with lse_i
+// (any number of parts, taken eight at a time); with m = max lse_i
 // and w_i = exp(lse_i - m), out = sum w_i O_i / sum w_i (bf16) and lse = m +
 // ln sum w_i (the lse identity of split softmax).  One warp per row, D / 32
 // columns per lane.
 template <int D>
-__global__ void __launch_bounds__(256) append_merge_kernel(const float* __restrict__ part_o,
+__global__ void __launch_bounds__(256) split_merge_kernel(const float* __restrict__ part_o,
                                                            const float* __restrict__ part_lse,
                                                            uint16_t* __restrict__ out,
                                                            float* __restrict__ lse, int nsplit,
                                                            int B, int C, int H) {
   constexpr int kPer = D / 32;  // 4 (D = 128) or 2 (D = 64) columns per lane
-  constexpr int kMaxSplit = 8;
+  constexpr int kBatch = 8;     // parts whose loads are in flight together
   using Vec = typename std::conditional<kPer == 4, float4, float2>::type;
   const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
@@ -717,31 +718,34 @@ __global__ void __launch_bounds__(256) append_merge_kernel(const float* __restri
   const long long bh = row / C;  // b * H + h
   const int h = (int)(bh % H);
   const int b = (int)(bh / H);
-  // every load issued before any is used
-  float li[kMaxSplit];
-  Vec o[kMaxSplit];
-#pragma unroll
-  for (int sp = 0; sp < kMaxSplit; ++sp) {
-    if (sp < nsplit) {
-      li[sp] = __ldg(part_lse + (long long)sp * rows + row);
-      o[sp] = __ldg(reinterpret_cast<const Vec*>(part_o + ((long long)sp * rows + row) * D) + lane);
-    }
-  }
   float m = -INFINITY;
+  for (int sp = lane; sp < nsplit; sp += 32) m = fmaxf(m, __ldg(part_lse + (long long)sp * rows + row));
 #pragma unroll
-  for (int sp = 0; sp < kMaxSplit; ++sp)
-    if (sp < nsplit) m = fmaxf(m, li[sp]);
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float acc[kPer] = {};
   float wsum = 0.f;
+  for (int sp0 = 0; sp0 < nsplit; sp0 += kBatch) {
+    // a batch of parts: every load issued before any is used
+    float li[kBatch];
+    Vec o[kBatch];
 #pragma unroll
-  for (int sp = 0; sp < kMaxSplit; ++sp) {
-    // a part holding none of the row's keys has lse = -inf: skipped
-    if (sp >= nsplit || li[sp] == -INFINITY) continue;
-    const float w = __expf(li[sp] - m);
-    wsum += w;
-    const float* f = reinterpret_cast<const float*>(&o[sp]);
+    for (int i = 0; i < kBatch; ++i) {
+      if (sp0 + i < nsplit) {
+        const long long pr = (long long)(sp0 + i) * rows + row;
+        li[i] = __ldg(part_lse + pr);
+        o[i] = __ldg(reinterpret_cast<const Vec*>(part_o + pr * D) + lane);
+      }
+    }
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) acc[e] += w * f[e];
+    for (int i = 0; i < kBatch; ++i) {
+      // a part holding none of the row's keys has lse = -inf: skipped
+      if (sp0 + i >= nsplit || li[i] == -INFINITY) continue;
+      const float w = __expf(li[i] - m);
+      wsum += w;
+      const float* f = reinterpret_cast<const float*>(&o[i]);
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] += w * f[e];
+    }
   }
   const float inv = 1.f / wsum;
   uint16_t* dst = out + (((long long)b * C + c) * H + h) * D + lane * kPer;
@@ -757,9 +761,28 @@ __global__ void __launch_bounds__(256) append_merge_kernel(const float* __restri
 
 }  // namespace
 
+bool split_workspace(int which, size_t bytes, cudaStream_t stream, float** part) {
+  int* cnt = nullptr;
+  void* p = nullptr;
+  if (!get_workspace(which, 256, bytes, stream, &cnt, &p)) return false;
+  *part = static_cast<float*>(p);
+  return true;
+}
+
+int encode_kv_map(CUtensorMap* m, const void* base, int D, int Hkv, int rows, int B) {
+  return encode_kv(m, base, D, Hkv, rows, B);
+}
+
 int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* out, float* lse,
                   const int64_t* pos, int B, int H, int Hkv, int D, int W, float scale,
                   cudaStream_t stream) {
+  // D = 128: the tensor-core decode (swa_decode_tc.cu); other sizes the
+  // split-KV row kernel below
+  if (D == 128) {
+    const int st = launch_decode_tc(q, k_ring, v_ring, out, lse, pos, B, H, Hkv, D, W, scale,
+                                    stream);
+    if (st != SWA_ERR_UNSUPPORTED) return st;
+  }
   RowParams p;
   std::memset(&p, 0, sizeof(p));
   if (encode_kv(&p.tmK, k_ring, D, Hkv, W, B) != SWA_OK ||
@@ -840,17 +863,17 @@ int ring_store(const void* k_new, const void* v_new, void* k_ring, void* v_ring,
 }  // namespace
 
 namespace {
-int append_merge(const float* part, void* out, float* lse, int nsplit, int B, int C, int H, int D,
+int merge_parts(const float* part, void* out, float* lse, int nsplit, int B, int C, int H, int D,
                  cudaStream_t stream) {
   const long long rows = (long long)B * H * C;
   const float* part_lse = part + (size_t)nsplit * rows * D;
   const long long blocks = (rows + 7) / 8;
   if (blocks > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
   if (D == 128)
-    append_merge_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
+    split_merge_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
         part, part_lse, static_cast<uint16_t*>(out), lse, nsplit, B, C, H);
   else
-    append_merge_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
+    split_merge_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
         part, part_lse, static_cast<uint16_t*>(out), lse, nsplit, B, C, H);
   return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
@@ -899,9 +922,14 @@ int append_attention_tc(const void* q, const void* k_new, const void* v_new, con
   const int st = launch_fwd_sm100(q, k_ring, v_ring, out, lse, B, H, Hkv, W + 64 + C, D, W - 1,
                                   0, 1, 0, nullptr, 0, scale, stream, &qw);
   if (st != SWA_OK || nsplit == 1) return st;
-  return append_merge(qw.part, out, lse, nsplit, B, C, H, D, stream);
+  return merge_parts(qw.part, out, lse, nsplit, B, C, H, D, stream);
 }
 }  // namespace
+
+int split_merge(const float* part, void* out, float* lse, int nsplit, int B, int C, int H, int D,
+                cudaStream_t stream) {
+  return merge_parts(part, out, lse, nsplit, B, C, H, D, stream);
+}
 
 int launch_append(const void* q, const void* k_new, const void* v_new, void* k_ring, void* v_ring,
                   void* out, float* lse, const int64_t* pos0, int B, int C, int H, int Hkv, int D,

@@ -53,7 +53,8 @@ def test_ring_decode_partial_cache(swa):
 
 
 @pytest.mark.parametrize("B,H,Hkv,D,W", [(3, 8, 8, 128, 300), (2, 16, 2, 64, 1000),
-                                         (4, 6, 2, 128, 777), (1, 2, 1, 64, 64)])
+                                         (4, 6, 2, 128, 777), (1, 2, 1, 64, 64),
+                                         (3, 16, 2, 128, 2500), (2, 4, 4, 128, 4096)])
 def test_ring_decode_shapes(swa, B, H, Hkv, D, W):
     q = inputs.normal((B, H, D), 9, 0)
     kr = inputs.normal((B, W, Hkv, D), 9, 1)
@@ -92,3 +93,14 @@ def test_workspace_reuse_across_sizes(swa):
     vr = inputs.normal((2, 2048, 4, 128), 17, 2)
     check(swa, q, kr, vr, torch.tensor([5000, 100], dtype=torch.int64))
     check(swa, *big)
+
+
+def test_ring_decode_parts_of_a_short_cache(swa):
+    """A long ring holding few tokens: parts of the ring past the filled slots
+    are empty and must not contribute (D = 128, GQA 4, positions below one
+    part, at a part boundary and past the first part)."""
+    B, H, Hkv, D, W = 4, 8, 2, 128, 4096
+    q = inputs.normal((B, H, D), 21, 0)
+    kr = inputs.normal((B, W, Hkv, D), 21, 1)
+    vr = inputs.normal((B, W, Hkv, D), 21, 2)
+    check(swa, q, kr, vr, torch.tensor([10, 1023, 1024, 2900], dtype=torch.int64))
