@@ -385,7 +385,7 @@ def run_ours(args, rank, world, local_rank):
               "ms_per_step": d_ms, "workload": dcfg.name,
               "roofline": {"bound": "hbm", "achieved": d_gbs, "peak": peaks["hbm_gbs"],
                            "unit": "GB/s", "frac": d_gbs / peaks["hbm_gbs"],
-                           "traffic": captured_traffic("swa_rowattn_kernel<128,4,0>"),
+                           "traffic": captured_traffic("swa_decode_tc_kernel"),
                            "peak_source": peak_src}}
     del dq, dk, dv
 

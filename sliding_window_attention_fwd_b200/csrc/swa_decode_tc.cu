@@ -11,10 +11,12 @@
 // zero rows of Q.  TMEM lane k of S^T is key k of the tile, so thread k of
 // the softmax warpgroup owns that key's scores; lane d of O^T is dimension d.
 // The key order does not matter to softmax, so the keys are walked in ring
-// slot order (slots >= min(pos + 1, W) are empty and masked).  A CTA takes a
-// 1024-slot part of one (batch, kv head)'s ring, streams its K and V tiles
-// through a three-slot TMA ring (128-byte swizzle), and writes O / l and
-// the lse of its part; a merge kernel combines the parts (lse identity).
+// slot order (slots >= min(pos + 1, W) are empty and masked).  Over a paged
+// cache the keys are the window's positions from a 64-aligned start, each
+// 64-row box looked up in the block table.  A CTA takes a part of about
+// 1024 keys of one (batch, kv head), streams its K and V tiles through a
+// three-slot TMA ring (128-byte swizzle), and writes O / l and the lse of
+// its part; a merge kernel combines the parts (lse identity).
 //
 // Warp roles (192 threads, two CTAs per SM): warp 0 TMA producer, warp 1
 // MMA issuer (and TMEM owner), warps 2-5 softmax (their lane quadrants
@@ -37,7 +39,7 @@ namespace swa {
 namespace {
 
 constexpr int kTK = 128;        // keys per tile (MMA M)
-constexpr int kPart = 1024;     // ring slots per CTA
+constexpr int kPart = 1024;     // key indices per CTA, about
 constexpr int kNQ = 8;          // query vectors of a GQA group, at most
 constexpr int kN = 16;          // MMA N: the group padded with zero rows
 constexpr int kRingSlots = 3;   // TMA ring (each slot one K or one V tile)
@@ -45,13 +47,20 @@ constexpr int kDecChunk = kTK * 128;  // one 64-column slice of a 128-row tile (
 constexpr float kLazy = 8.0f;   // log2 units
 
 struct DecParams {
-  CUtensorMap tmK, tmV;  // rings [B, W, Hkv, D]: dims {D, Hkv, W, B}, 64 x 64 boxes
+  // rings [B, W, Hkv, D] (dims {D, Hkv, W, B}), or the page pools
+  // [num_pages * page_size, Hkv, D] (batch dimension 1); 64 x 64 boxes
+  CUtensorMap tmK, tmV;
   const uint16_t* q;     // [B, H, D]
   const int64_t* pos;    // [B]
+  // paged cache: logical page lp of sequence b is physical page
+  // table[b * max_pages + lp] (page_size a multiple of 64)
+  const int32_t* table;
+  int paged, page_size, max_pages;
   float* part_o;         // [nsplit, B, H, D]: O / l of each part
   float* part_lse;       // [nsplit, B, H]: ln-sum-exp of each part (-inf: empty)
   int* err;
   int B, H, Hkv, W, grp, nsplit;
+  int part_keys;  // key indices per CTA (a multiple of 128)
   float scale_log2;
 };
 
@@ -111,9 +120,22 @@ __global__ void __launch_bounds__(DecCfg::kThreads, 2)
   const int g = x % p.Hkv;
   const int b = x / p.Hkv;
   const long long pb = p.pos[b];
-  const int nvalid = pb + 1 < (long long)p.W ? (int)(pb + 1) : p.W;  // filled slots
-  const int s0 = part * kPart;
-  const int s1 = min(s0 + kPart, nvalid);
+  // key index space of the CTA's part: ring slots [0, min(pos + 1, W)), or,
+  // paged, positions a64 + idx for idx in [0, pos - a64] from the window's
+  // first position a rounded down to 64 (so no 64-row box crosses a page),
+  // the positions below a masked
+  long long a64 = 0;
+  int lo_idx = 0, n_idx;
+  if (p.paged) {
+    const long long a = pb - p.W + 1 > 0 ? pb - p.W + 1 : 0;
+    a64 = a & ~63LL;
+    lo_idx = (int)(a - a64);
+    n_idx = (int)(pb - a64 + 1);
+  } else {
+    n_idx = pb + 1 < (long long)p.W ? (int)(pb + 1) : p.W;  // filled slots
+  }
+  const int s0 = part * p.part_keys;
+  const int s1 = min(s0 + p.part_keys, n_idx);
   const int ntiles = s1 > s0 ? (s1 - s0 + kTK - 1) / kTK : 0;
   const int nq = p.grp;
 
@@ -180,10 +202,23 @@ __global__ void __launch_bounds__(DecCfg::kThreads, 2)
         const CUtensorMap* m = kv ? &p.tmV : &p.tmK;
         uint8_t* dst = smem + C::kRing + st * C::kTile;
         mbar_arrive_expect_tx(&full[st], C::kTile);
-        for (int cc = 0; cc < D / 64; ++cc)
-          for (int hh = 0; hh < 2; ++hh)
+        for (int hh = 0; hh < 2; ++hh) {
+          // source row of the 64 keys from index idx0: a ring slot, or a row
+          // of the page pool (a page id past the table reads as zeros,
+          // masked below)
+          const int idx0 = s0 + t * kTK + hh * 64;
+          int row = idx0, bc = b;
+          if (p.paged) {
+            const long long t0 = a64 + idx0;
+            const long long lp = t0 / p.page_size;
+            const long long page = lp < p.max_pages ? p.table[(long)b * p.max_pages + lp] : -1;
+            row = page < 0 ? -64 : (int)(page * p.page_size + t0 % p.page_size);
+            bc = 0;
+          }
+          for (int cc = 0; cc < D / 64; ++cc)
             tma_load_4d(dst + cc * kDecChunk + hh * (kDecChunk / 2), m, &full[st], cc * 64, g,
-                        s0 + t * kTK + hh * 64, b);
+                        row, bc);
+        }
       }
 #ifdef SWA_TEST_WITHHOLD_TILE
       const int skip = 2 * SWA_TEST_WITHHOLD_TILE;
@@ -262,7 +297,8 @@ __global__ void __launch_bounds__(DecCfg::kThreads, 2)
       uint32_t sv[16];
       tmem_ld16(tmem + 16u * (t & 1) + lane_off, sv);
       tmem_wait_ld();
-      const bool valid = s0 + t * kTK + r < s1;
+      const int idx = s0 + t * kTK + r;
+      const bool valid = idx < s1 && idx >= lo_idx;
       float xs[kNQ];
 #pragma unroll
       for (int n = 0; n < kNQ; ++n) xs[n] = valid ? __uint_as_float(sv[n]) * sl2 : -INFINITY;
@@ -376,20 +412,16 @@ __global__ void __launch_bounds__(DecCfg::kThreads, 2)
 
 }  // namespace
 
-int launch_decode_tc(const void* q, const void* k_ring, const void* v_ring, void* out, float* lse,
-                     const int64_t* pos, int B, int H, int Hkv, int D, int W, float scale,
-                     cudaStream_t stream) {
-  const int grp = H / Hkv;
-  if (D != 128 || grp > kNQ || grp < 1) return SWA_ERR_UNSUPPORTED;
+namespace {
+int launch_tc(DecParams& p, const void* q, void* out, float* lse, const int64_t* pos, int B,
+              int H, int Hkv, int D, int W, int span, float scale, cudaStream_t stream) {
   static std::atomic<unsigned long long> attr{0};
   if (!smem_attr_once(reinterpret_cast<const void*>(swa_decode_tc_kernel), DecCfg::kAlloc, attr))
     return SWA_ERR_CUDA;
-  DecParams p;
-  std::memset(&p, 0, sizeof(p));
-  if (encode_kv_map(&p.tmK, k_ring, D, Hkv, W, B) != SWA_OK ||
-      encode_kv_map(&p.tmV, v_ring, D, Hkv, W, B) != SWA_OK)
-    return SWA_ERR_CUDA;
+  // about kPart keys per CTA: as many parts as W needs, the span (W, or
+  // W + 63 from a 64-aligned start) shared evenly in whole 128-key tiles
   p.nsplit = (W + kPart - 1) / kPart;
+  p.part_keys = ((span + p.nsplit - 1) / p.nsplit + kTK - 1) / kTK * kTK;
   const size_t rows = (size_t)B * H;
   float* part = nullptr;
   if (!split_workspace(1, (size_t)p.nsplit * rows * (D + 1) * sizeof(float), stream, &part))
@@ -404,13 +436,48 @@ int launch_decode_tc(const void* q, const void* k_ring, const void* v_ring, void
   p.H = H;
   p.Hkv = Hkv;
   p.W = W;
-  p.grp = grp;
+  p.grp = H / Hkv;
   p.scale_log2 = scale * 1.4426950408889634f;
   const long long grid = (long long)B * Hkv * p.nsplit;
   if (grid > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
   swa_decode_tc_kernel<<<(unsigned)grid, DecCfg::kThreads, DecCfg::kAlloc, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SWA_ERR_CUDA;
   return split_merge(part, out, lse, p.nsplit, B, 1, H, D, stream);
+}
+}  // namespace
+
+int launch_decode_tc(const void* q, const void* k_ring, const void* v_ring, void* out, float* lse,
+                     const int64_t* pos, int B, int H, int Hkv, int D, int W, float scale,
+                     cudaStream_t stream) {
+  const int grp = H / Hkv;
+  if (D != 128 || grp > kNQ || grp < 1) return SWA_ERR_UNSUPPORTED;
+  DecParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (encode_kv_map(&p.tmK, k_ring, D, Hkv, W, B) != SWA_OK ||
+      encode_kv_map(&p.tmV, v_ring, D, Hkv, W, B) != SWA_OK)
+    return SWA_ERR_CUDA;
+  return launch_tc(p, q, out, lse, pos, B, H, Hkv, D, W, W, scale, stream);
+}
+
+int launch_decode_paged_tc(const void* q, const void* k_pages, const void* v_pages, void* out,
+                           float* lse, const int32_t* table, const int64_t* pos, int B, int H,
+                           int Hkv, int D, int page_size, int num_pages, int max_pages, int W,
+                           float scale, cudaStream_t stream) {
+  const int grp = H / Hkv;
+  if (D != 128 || grp > kNQ || grp < 1 || page_size % 64 != 0) return SWA_ERR_UNSUPPORTED;
+  const long long pool_rows = (long long)num_pages * page_size;
+  if (pool_rows > 0x7fffffffLL || (long long)W + 64 > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  DecParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (encode_kv_map(&p.tmK, k_pages, D, Hkv, (int)pool_rows, 1) != SWA_OK ||
+      encode_kv_map(&p.tmV, v_pages, D, Hkv, (int)pool_rows, 1) != SWA_OK)
+    return SWA_ERR_CUDA;
+  p.paged = 1;
+  p.table = table;
+  p.page_size = page_size;
+  p.max_pages = max_pages;
+  // the window's positions from a 64-aligned start: at most W + 63 indices
+  return launch_tc(p, q, out, lse, pos, B, H, Hkv, D, W, W + 63, scale, stream);
 }
 
 }  // namespace swa

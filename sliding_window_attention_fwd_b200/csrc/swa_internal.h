@@ -85,6 +85,11 @@ int launch_decode(const void* q, const void* k_ring, const void* v_ring, void* o
 int launch_decode_tc(const void* q, const void* k_ring, const void* v_ring, void* out,
                      float* lse, const int64_t* pos, int B, int H, int Hkv, int D, int W,
                      float scale, cudaStream_t stream);
+// The same over a paged cache (page_size a multiple of 64).
+int launch_decode_paged_tc(const void* q, const void* k_pages, const void* v_pages, void* out,
+                           float* lse, const int32_t* table, const int64_t* pos, int B, int H,
+                           int Hkv, int D, int page_size, int num_pages, int max_pages, int W,
+                           float scale, cudaStream_t stream);
 // Library workspace `which` (one per device and use) of at least `bytes`.
 bool split_workspace(int which, size_t bytes, cudaStream_t stream, float** part);
 // Tensor map of a [B, rows, Hkv, D] bf16 tensor: 64-column x 64-row boxes,

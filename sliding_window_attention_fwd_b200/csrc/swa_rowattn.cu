@@ -813,6 +813,11 @@ int launch_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                         float* lse, const int32_t* table, const int64_t* pos, int B, int H,
                         int Hkv, int D, int page_size, int num_pages, int max_pages, int W,
                         float scale, cudaStream_t stream) {
+  if (D == 128) {
+    const int st = launch_decode_paged_tc(q, k_pages, v_pages, out, lse, table, pos, B, H, Hkv,
+                                          D, page_size, num_pages, max_pages, W, scale, stream);
+    if (st != SWA_ERR_UNSUPPORTED) return st;
+  }
   RowParams p;
   std::memset(&p, 0, sizeof(p));
   const long long rows = (long long)num_pages * page_size;
