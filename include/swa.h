@@ -255,7 +255,9 @@ SWA_API int swa_forward_f32(const float* q, const float* k, const float* v,
  * the caller has already written its k/v into slot pos[b] % W.  The query
  * attends positions max(0, pos-W+1) .. pos, i.e. ring slots
  * 0 .. min(pos, W-1) (all W slots once pos >= W-1).  scale is 1/sqrt(D).
- * D must be 128 or 64; H % Hkv == 0 and H / Hkv <= 8.
+ * D must be 128 or 64; H % Hkv == 0 and H / Hkv <= 8.  Launches on
+ * `stream`: at D = 128 a tensor-core kernel over parts of about 1024 slots
+ * and a kernel merging the parts; at D = 64 the split-KV row kernel.
  * The first call on a device allocates a small library-owned workspace
  * (split partials and counters, kept until swa_release); make that first
  * call before capturing a CUDA graph.  Calls on different streams of one
