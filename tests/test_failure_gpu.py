@@ -5,8 +5,8 @@
   usable afterwards.
 * The same inside the production kernels: a test-only build of the library
   (SWA_TEST_WITHHOLD_TILE) never loads one K/V tile, and lowers the bound on
-  every wait to 5 ms.  The fused forward and the split-KV row kernel must
-  then time out, leave their abort path (in-flight copies drained, TMEM
+  every wait to 5 ms.  The fused forward, the tensor-core decode and the
+  split-KV row kernel must then time out, leave their abort path (in-flight copies drained, TMEM
   released) and return; a problem that needs no withheld tile still gives
   the oracle's result with the same library, so the context and the SM
   resources (TMEM) are intact.
@@ -97,9 +97,12 @@ def test_forward_abort_path(withheld_lib):
     compare(lse2.cpu().numpy(), ref_l, LSE_ABS, what="lse")
 
 
-def test_row_kernel_abort_path(withheld_lib):
+@pytest.mark.parametrize("D", [128, 64])
+def test_decode_abort_path(withheld_lib, D):
+    """D = 128: the tensor-core decode (K tile 1 of every part withheld);
+    D = 64: the split-KV row kernel (its 64-row stage 1 withheld)."""
     lib = withheld_lib
-    B, H, Hkv, D, W = 2, 8, 2, 128, 4096  # 1024 keys = 16 stages per CTA
+    B, H, Hkv, W = 2, 8, 2, 4096  # 1024 keys per CTA: 8 tiles / 16 stages
     q = inputs.normal((B, H, D), 43, 0).cuda()
     kr = inputs.normal((B, W, Hkv, D), 43, 1).cuda()
     vr = inputs.normal((B, W, Hkv, D), 43, 2).cuda()
