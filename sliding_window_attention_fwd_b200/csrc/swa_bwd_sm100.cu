@@ -65,6 +65,9 @@ static_assert(kGroupsB == 1 || kGroupsB == 2 || kGroupsB == 4, "1, 2 or 4 comput
 // (16 elements) of a P / dS operand written in place over fp32 scores: chunk
 // ch of 32 scores (group g = ch / kCpg, its i-th chunk) is packed into the 16
 // columns 32 kCpg g + 16 i, inside the group's own (already read) columns.
+// dq kernel: TMEM column of step it's S buffer
+__device__ __forceinline__ uint32_t sbuf(int it) { return (it & 1) ? 384u : 0u; }
+
 __device__ __forceinline__ uint32_t pcol(int k) {
   const int ch = k / 2, g = ch / kCpg, i = ch % kCpg;
   return (uint32_t)(32 * kCpg * g + 16 * i + 8 * (k % 2));
@@ -101,13 +104,14 @@ struct BCfg {
   static constexpr int kStageBytes = 2 * kTile;
   static constexpr int kVec = kRing + kStages * kStageBytes;  // dkdv: [stage][lse2 | delta][128]
   static constexpr int kBar = kVec + kStages * 2 * kTileM * 4;
-  static constexpr int kNumBars = 1 + 2 * kStages + 2 * kStages + 4;
+  static constexpr int kNumBars = 1 + 2 * kStages + 2 * kStages + 5;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16 + 1024;  // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory budget");
   static_assert(2 * kStages >= kGroupsB, "dq kernel: the Delta parts fit in the vector area");
   // TMEM columns: S (or S^T) [0, 128), dP (or dP^T) [128, 256), then the
-  // accumulators: dq kernel dQ [256, 256 + D); dkdv kernel dV, dK.
+  // accumulators: dq kernel dQ [256, 256 + D) and its second S buffer
+  // [384, 512); dkdv kernel dV, dK.
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -154,8 +158,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   uint64_t* full_v = full_k + S_;       // [S_]
   uint64_t* empty_k = full_v + S_;      // [S_]
   uint64_t* empty_v = empty_k + S_;     // [S_]
-  uint64_t* s_full = empty_v + S_;      // S of the step in TMEM
-  uint64_t* dp_full = s_full + 1;       // dP of the step in TMEM
+  uint64_t* s_full = empty_v + S_;      // [it & 1]: S of step it in its TMEM buffer
+  uint64_t* dp_full = s_full + 2;       // dP of the step in TMEM
   uint64_t* ds_full = dp_full + 1;      // dS of the step written (128 arrivals)
   uint64_t* done = ds_full + 1;         // every MMA finished
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
@@ -189,7 +193,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       mbar_init(&empty_k[s], 1);
       mbar_init(&empty_v[s], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     mbar_init(dp_full, 1);
     mbar_init(ds_full, 128 * kGroupsB);
     mbar_init(done, 1);
@@ -249,20 +254,24 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       const uint64_t dkmn0 = sdesc_sw128(ring_addr, kChunkB, 1024);         // K, MN-major
       const uint64_t dv0 = sdesc_sw128(ring_addr + C::kTile, 16, 1024);     // V, K-major
       constexpr uint64_t kStageStep = C::kStageBytes >> 4;
-      bool ok = mbar_wait(full_q, 0, p.err, abort_flag);
-      for (int it = 0; ok && it < n_tiles; ++it) {
+      // S of step it goes to TMEM buffer it & 1 ([0, 128) or [384, 512)), so
+      // S(it + 1) is issued before dQ(it) reads dS(it) from the other one;
+      // order: S(0), dP(0), then per step S(it + 1), dQ(it), dP(it + 1)
+      auto issue_s = [&](int it) -> bool {
         const int st = it % S_;
-        const uint32_t ph = (uint32_t)(it / S_) & 1u;
-        // S = Q K^T (the previous step's dQ MMA, issued before, has read dS)
-        if (!mbar_wait(&full_k[st], ph, p.err, abort_flag)) break;
+        if (!mbar_wait(&full_k[st], (uint32_t)(it / S_) & 1u, p.err, abort_flag)) return false;
         tc_fence_after();
         const uint64_t dk = dk0 + (uint64_t)st * kStageStep;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          mma_ss(tmem, dq_ + kmajor_off(k), dk + kmajor_off(k), idesc_s, k > 0 ? 1u : 0u);
-        tc_commit(s_full);
-        // dP = dO V^T
-        if (!mbar_wait(&full_v[st], ph, p.err, abort_flag)) break;
+          mma_ss(tmem + sbuf(it), dq_ + kmajor_off(k), dk + kmajor_off(k), idesc_s,
+                 k > 0 ? 1u : 0u);
+        tc_commit(&s_full[it & 1]);
+        return true;
+      };
+      auto issue_dp = [&](int it) -> bool {
+        const int st = it % S_;
+        if (!mbar_wait(&full_v[st], (uint32_t)(it / S_) & 1u, p.err, abort_flag)) return false;
         tc_fence_after();
         const uint64_t dv = dv0 + (uint64_t)st * kStageStep;
 #pragma unroll
@@ -271,15 +280,23 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                  k > 0 ? 1u : 0u);
         tc_commit(dp_full);
         tc_commit(&empty_v[st]);
-        // dQ += dS K, dS (bf16) over S's columns
+        return true;
+      };
+      bool ok = mbar_wait(full_q, 0, p.err, abort_flag) && issue_s(0) && issue_dp(0);
+      for (int it = 0; ok && it < n_tiles; ++it) {
+        const int st = it % S_;
+        if (it + 1 < n_tiles && !issue_s(it + 1)) break;
+        // dQ += dS K, dS (bf16) over S's columns; then dP of the next step
+        // (the compute warps have read dP(it))
         if (!mbar_wait(ds_full, (uint32_t)it & 1u, p.err, abort_flag)) break;
         tc_fence_after();
         const uint64_t dkmn = dkmn0 + (uint64_t)st * kStageStep;
 #pragma unroll
         for (int k = 0; k < kTileN / 16; ++k)
-          mma_ts(tmem + 256u, tmem + pcol(k), dkmn + (uint64_t)((k * 2048) >> 4), idesc_dq,
-                 (it > 0 || k > 0) ? 1u : 0u);
+          mma_ts(tmem + 256u, tmem + sbuf(it) + pcol(k), dkmn + (uint64_t)((k * 2048) >> 4),
+                 idesc_dq, (it > 0 || k > 0) ? 1u : 0u);
         tc_commit(&empty_k[st]);
+        if (it + 1 < n_tiles && !issue_dp(it + 1)) break;
       }
       tc_commit(done);  // also on the abort path: TMEM quiescent before it is freed
     }
@@ -291,7 +308,6 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off;
     const uint32_t tP = tmem + 128u + lane_off;
     const uint32_t tQ = tmem + 256u + lane_off;
     const int m_v = qt * kTileM + r;
@@ -342,7 +358,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       const int t = tr.kv_begin + it;
       const bool edge = !(t >= int_lo && t <= int_hi);
       // P as soon as S is in TMEM (dP is still being computed)
-      bool w = mbar_wait(s_full, ph, p.err, abort_flag);
+      const uint32_t tS = tmem + sbuf(it) + lane_off;
+      bool w = mbar_wait(&s_full[it & 1], (uint32_t)(it >> 1) & 1u, p.err, abort_flag);
       if (!__all_sync(0xffffffffu, w)) {
         ok = false;
         break;
@@ -563,24 +580,34 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       const uint64_t ddomn0 = sdesc_sw128(ring_addr + C::kTile, kChunkB, 1024);
       constexpr uint64_t kStageStep = C::kStageBytes >> 4;
       const uint32_t t_dv = tmem + 256u, t_dk = tmem + 256u + (uint32_t)D;
-      bool ok = mbar_wait(full_kv, 0, p.err, abort_flag);
-      for (int s = 0; ok && s < n_steps; ++s) {
+      // order: S^T(0), dP^T(0), then per step dV(s), S^T(s + 1), dK(s),
+      // dP^T(s + 1): each of S^T(s + 1) / dP^T(s + 1) right after the MMA that
+      // reads the columns it overwrites (P^T(s) / dS^T(s)), so the compute
+      // warps get the next S^T one MMA group sooner
+      auto issue_st = [&](int s) -> bool {
         const int st = s % S_;
-        const uint32_t ph = (uint32_t)(s / S_) & 1u;
-        if (!mbar_wait(&full[st], ph, p.err, abort_flag)) break;
+        if (!mbar_wait(&full[st], (uint32_t)(s / S_) & 1u, p.err, abort_flag)) return false;
         tc_fence_after();
         const uint64_t sq = (uint64_t)st * kStageStep;
-        // S^T = K Q^T and dP^T = V dO^T (the previous step's dV / dK MMAs,
-        // issued before, have read P^T and dS^T)
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
           mma_ss(tmem, dk_ + kmajor_off(k), dq0 + sq + kmajor_off(k), idesc_s, k > 0 ? 1u : 0u);
         tc_commit(st_full);
+        return true;
+      };
+      auto issue_dpt = [&](int s) {  // after issue_st(s): the stage is full
+        const uint64_t sq = (uint64_t)(s % S_) * kStageStep;
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
           mma_ss(tmem + 128u, dv_ + kmajor_off(k), ddo0 + sq + kmajor_off(k), idesc_s,
                  k > 0 ? 1u : 0u);
         tc_commit(dpt_full);
+      };
+      bool ok = mbar_wait(full_kv, 0, p.err, abort_flag) && issue_st(0);
+      if (ok) issue_dpt(0);
+      for (int s = 0; ok && s < n_steps; ++s) {
+        const int st = s % S_;
+        const uint64_t sq = (uint64_t)st * kStageStep;
         // dV += P^T dO, dK += dS^T Q
         if (!mbar_wait(pt_full, (uint32_t)s & 1u, p.err, abort_flag)) break;
         tc_fence_after();
@@ -588,11 +615,14 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         for (int k = 0; k < kTileM / 16; ++k)
           mma_ts(t_dv, tmem + pcol(k), ddomn0 + sq + (uint64_t)((k * 2048) >> 4), idesc_o,
                  (s > 0 || k > 0) ? 1u : 0u);
+        const bool next = s + 1 < n_steps;
+        if (next && !issue_st(s + 1)) break;
 #pragma unroll
         for (int k = 0; k < kTileM / 16; ++k)
           mma_ts(t_dk, tmem + 128u + pcol(k), dqmn0 + sq + (uint64_t)((k * 2048) >> 4), idesc_o,
                  (s > 0 || k > 0) ? 1u : 0u);
         tc_commit(&empty[st]);
+        if (next) issue_dpt(s + 1);
       }
       tc_commit(done);
     }
