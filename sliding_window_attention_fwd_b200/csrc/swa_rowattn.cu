@@ -718,10 +718,15 @@ __global__ void __launch_bounds__(256) split_merge_kernel(const float* __restric
   const long long bh = row / C;  // b * H + h
   const int h = (int)(bh % H);
   const int b = (int)(bh / H);
+  // m = max lse_i: with at most kBatch parts it comes from the batch loaded
+  // below (one pass, every load in flight at once); otherwise a first pass
   float m = -INFINITY;
-  for (int sp = lane; sp < nsplit; sp += 32) m = fmaxf(m, __ldg(part_lse + (long long)sp * rows + row));
+  if (nsplit > kBatch) {
+    for (int sp = lane; sp < nsplit; sp += 32)
+      m = fmaxf(m, __ldg(part_lse + (long long)sp * rows + row));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  }
   float acc[kPer] = {};
   float wsum = 0.f;
   for (int sp0 = 0; sp0 < nsplit; sp0 += kBatch) {
@@ -735,6 +740,11 @@ __global__ void __launch_bounds__(256) split_merge_kernel(const float* __restric
         li[i] = __ldg(part_lse + pr);
         o[i] = __ldg(reinterpret_cast<const Vec*>(part_o + pr * D) + lane);
       }
+    }
+    if (nsplit <= kBatch) {
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i)
+        if (i < nsplit) m = fmaxf(m, li[i]);
     }
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
