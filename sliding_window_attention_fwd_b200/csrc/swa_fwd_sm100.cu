@@ -734,6 +734,14 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
         tmem_st16(tS + pcol + jj * 16, pk);
       }
     };
+    // zeros as the P of a key half (32 columns of bf16 pairs from pcol)
+    auto zero_p = [&](int pcol) {
+      uint32_t z[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) z[i] = 0u;
+      tmem_st16(tS + pcol, z);
+      tmem_st16(tS + pcol + 16, z);
+    };
     // Multiplies O (and l) by 2^(m_from - m_to) and adopts m_to; O holds
     // P_0..P_{it-1} V, whose MMAs are complete once o_done says so.
     auto rescale_o = [&](int it, bool mine, float m_to) -> bool {
@@ -796,9 +804,15 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       bool w_ok = mbar_wait(&se_full[slot], ph, p.err, abort_flag);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
+      // key halves of a global-key tile past the last global key hold no
+      // key of any row: no scores to read, P = 0 (the same for every row)
+      const bool gskip_e = glob && it >= n_band && (it - n_band) * kTileN + 64 * e >= p.n_global;
+      float tmax = -INFINITY;
+      if (gskip_e) {
+        zero_p(64 * e);
+      } else {
       read_half(e, sv);
       mask_half(it, e, edge, sv);
-      float tmax;
       if (!__any_sync(0xffffffffu, m_used == -INFINITY)) {
         // optimistic: exponentiate against the running max while the half's
         // max is found (no dependence between the two); a jump (rare)
@@ -824,6 +838,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
         }
         exp_half(64 * e, sv, m_used == -INFINITY ? 0.f : m_used, ls);
       }
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&pe_full[slot]);
@@ -832,6 +847,13 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       w_ok = mbar_wait(&sl_full[slot], ph, p.err, abort_flag);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
+      const bool gskip_l =
+          glob && it >= n_band && (it - n_band) * kTileN + 64 * (e ^ 1) >= p.n_global;
+      if (gskip_l) {
+        tc_fence_before();
+        mbar_arrive(&l_free[slot]);
+        zero_p(64 * e + 32);
+      } else {
       read_half(e ^ 1, sv);
       // these columns now belong to the early half of the next tile
       tc_fence_before();
@@ -878,6 +900,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
           for (int j = 0; j < 4; ++j) ls[j] = make_float2(ls[j].x * f, ls[j].y * f);
         }
         exp_half(64 * e + 32, sv, m_used == -INFINITY ? 0.f : m_used, ls);
+      }
       }
       {
         const float2 a2 = add2(add2(ls[0], ls[1]), add2(ls[2], ls[3]));
