@@ -539,6 +539,21 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       const uint32_t ph = (uint32_t)(s / S_) & 1u;
       const int qt = qr.kv_begin + s / grp;
       const int h = g_kv * grp + s % grp;
+      // lse (log2 units) and Delta of the tile's 128 query rows, loaded into
+      // registers before the wait for the stage so their latency overlaps it;
+      // rows past the class end get lse = +inf (P = 0)
+      float l2[kTileM / 32], dl[kTileM / 32];
+#pragma unroll
+      for (int u = 0; u < kTileM / 32; ++u) {
+        const int m = qt * kTileM + lane + 32 * u;
+        l2[u] = INFINITY;
+        dl[u] = 0.f;
+        if (m < Mv) {
+          const size_t li = ((size_t)b * p.H + h) * p.N + phys_row(geo, c, m);
+          l2[u] = __ldg(p.lse + li) * kLog2e;
+          dl[u] = p.delta[li];
+        }
+      }
       if (s >= S_ && !mbar_wait(&empty[st], ph ^ 1u, p.err, abort_flag)) break;
       if (lane == 0) {
         uint8_t* qb = smem + C::kRing + st * C::kStageBytes;
@@ -546,19 +561,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         load_tile<D>(qb, &p.tmQ[map_idx], &full[st], p, c, h, qt * kTileM, b);
         load_tile<D>(qb + C::kTile, &p.tmDO[map_idx], &full[st], p, c, h, qt * kTileM, b);
       }
-      // lse (log2 units) and Delta of the tile's 128 query rows; rows past the
-      // class end get lse = +inf (P = 0)
       float* vl = vec + st * 2 * kTileM;
-      for (int e = lane; e < kTileM; e += 32) {
-        const int m = qt * kTileM + e;
-        float l2 = INFINITY, dl = 0.f;
-        if (m < Mv) {
-          const size_t li = ((size_t)b * p.H + h) * p.N + phys_row(geo, c, m);
-          l2 = __ldg(p.lse + li) * kLog2e;
-          dl = p.delta[li];
-        }
-        vl[e] = l2;
-        vl[kTileM + e] = dl;
+#pragma unroll
+      for (int u = 0; u < kTileM / 32; ++u) {
+        vl[lane + 32 * u] = l2[u];
+        vl[kTileM + lane + 32 * u] = dl[u];
       }
       mbar_arrive(&full[st]);
       last = s;
