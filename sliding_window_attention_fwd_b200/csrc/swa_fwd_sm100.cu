@@ -119,6 +119,19 @@ struct FwdParams {
   int nsplit;
   float* part_o;
   float* part_lse;
+  // Paired parts (nsplit == 2, launched as clusters of two CTAs whose rank
+  // is the part): the two parts merge through distributed shared memory and
+  // write out / lse themselves, with no partials and no merge kernel.
+  // ring_store (paired, in place, one query tile, every head of the kv head
+  // in one item, so the cluster holds every reader of the kv head's ring
+  // rows): once both parts' MMAs are done, the chunk's keys (part 0) and
+  // values (part 1) enter their ring slots (pos0 + c) % win.
+  int pair;
+  int ring_store;
+  uint4* k_ring;
+  uint4* v_ring;
+  const uint4* kn_raw;
+  const uint4* vn_raw;
 };
 
 template <int D, int NSLOT, int NSTREAM>
@@ -142,12 +155,17 @@ struct Cfg {
   static constexpr int kRing = kQ + kQBytes;
   static constexpr int kBar = kRing + kStages * kStageBytes;
   // full_q, full_k[S], empty_k[S], full_v[S], empty_v[S],
-  // se_full[2], sl_full[2], l_free[2], p_full[2], o_done[2], o_final[2]
-  static constexpr int kNumBars = 1 + 4 * kStages + 16;
+  // se_full[2], sl_full[2], l_free[2], p_full[2], o_done[2], o_final[2],
+  // pe_full[2], oe_done[2], peer_free, xfer
+  static constexpr int kNumBars = 1 + 4 * kStages + 18;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kTotal = kMisc + 16;
   static constexpr int kAlloc = kTotal + 1024;  // slack for 1024-byte alignment
   static_assert(kAlloc <= 232448, "shared memory budget");
+  // paired parts: the half of O the other part writes (fp32, NSLOT x 128
+  // rows of D / 2) and its (m, l) per row land in the ring
+  static constexpr int kRxO = NSLOT * 128 * (D / 2) * 4;
+  static_assert(kRxO + NSLOT * 128 * 8 <= kStages * kStageBytes, "pair exchange area");
 };
 
 // KIND (compile-time, so each form carries only its own code): 0 band (and
@@ -176,6 +194,10 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
   uint64_t* o_final = o_done + 2;
   uint64_t* pe_full = o_final + 2;  // [slot]: P of the early half written
   uint64_t* oe_done = pe_full + 2;  // [slot]: PV of the early half done
+  // paired parts: the other part's MMAs are done (its ring may be
+  // written); the other part's half of O and (m, l) have landed here
+  uint64_t* peer_free = oe_done + 2;
+  uint64_t* xfer = peer_free + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
 
@@ -351,6 +373,8 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       mbar_init(&pe_full[s], 128);
       mbar_init(&oe_done[s], 1);
     }
+    mbar_init(peer_free, 128 * NSLOT);
+    mbar_init(xfer, 128 * NSLOT);
     fence_mbar_init();
     // (an empty part of a split key walk loads nothing: no copy may still
     // be landing in shared memory when the CTA exits)
@@ -374,6 +398,10 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // paired parts: this CTA's barriers exist (the other part waits for this
+  // arrival before its first access to them)
+  const bool pair = qwin && p.pair;
+  if (pair) cluster_arrive_relaxed();
   const uint32_t tmem = *tmem_holder;
   // TMEM columns: slot s has S/P at [128 s, 128 s + 128) and O at 256 + 128 s.
   const uint32_t q_addr = smem_u32(smem + C::kQ);
@@ -915,7 +943,7 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
 
     // split key walk: this CTA's part goes to the partials (fp32 O / l and
     // lse); an empty part contributes nothing (lse = -inf)
-    const bool split = qwin && p.nsplit > 1;
+    const bool split = qwin && p.nsplit > 1 && !pair;
     const size_t prow = (((size_t)sp * p.B + b) * p.H + h) * (size_t)Mq + m_row;
     if (split && ok && n_tiles == 0 && row_valid && !warp_idle) {
       float4* dst = reinterpret_cast<float4*>(p.part_o + prow * D);
@@ -924,7 +952,109 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
     }
     bool fin = ok && n_tiles > 0 && !warp_idle;
     if (fin) fin = mbar_wait(&o_final[slot], 0, p.err, abort_flag);
-    if (__all_sync(0xffffffffu, fin)) {
+    if (pair) {
+      // The two parts of the key walk merge through distributed shared
+      // memory.  Once both have finished their MMAs (each tells the other
+      // on peer_free), each sends the other the half of its O columns that
+      // the other writes, with its (m, l), and merges the half it keeps:
+      // with M = max(m_0, m_1) and a_i = 2^(m_i - M), out = (a_0 O_0 + a_1
+      // O_1) / (a_0 l_0 + a_1 l_1) (the split softmax's lse identity).
+      constexpr int kHalf = D / 2;  // columns a part writes
+      constexpr int kV4 = kHalf / 4;
+      const uint32_t peer = (uint32_t)(sp ^ 1);
+      const int rrow = slot * 128 + r;
+      // receive area (the ring, free once this CTA's MMAs are done): row
+      // rrow's kV4 float4, XOR-swizzled by the row against bank conflicts,
+      // then (m, l) per row
+      const uint32_t rx_o = smem_u32(smem + C::kRing) + (uint32_t)(rrow * kV4 * 16);
+      const uint32_t rx_ml = smem_u32(smem + C::kRing) + (uint32_t)(C::kRxO + rrow * 8);
+      // O in TMEM is complete (an empty part, or one that gave up, sends
+      // zeros with m = -inf)
+      const bool have = __all_sync(0xffffffffu, fin);
+      const float m_me = have ? m_used : -INFINITY, l_me = have ? l : 0.f;
+      __syncwarp();
+      cluster_wait();  // the other part's barriers exist
+      mbar_arrive_cluster(map_shared_rank(smem_u32(peer_free), peer));
+      const bool go = __all_sync(0xffffffffu, mbar_wait<true>(peer_free, 0, p.err, abort_flag));
+      if (go) {
+        const uint32_t dst = map_shared_rank(rx_o, peer);
+#pragma unroll
+        for (int j = 0; j < kHalf / 32; ++j) {
+          uint32_t v[32];
+          if (have) {
+            tmem_ld32(tO + (uint32_t)(peer * kHalf + 32 * j), v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4)
+            st_cluster_f4(dst + (uint32_t)(((j * 8 + e4) ^ (r & 7)) * 16),
+                          __uint_as_float(v[4 * e4]), __uint_as_float(v[4 * e4 + 1]),
+                          __uint_as_float(v[4 * e4 + 2]), __uint_as_float(v[4 * e4 + 3]));
+        }
+        st_cluster_f2(map_shared_rank(rx_ml, peer), m_me, l_me);
+      }
+      mbar_arrive_cluster(map_shared_rank(smem_u32(xfer), peer));
+      // both parts' MMAs are done, so every read of this kv head's ring rows
+      // is: the chunk enters the ring (keys from part 0, values from part 1)
+      if (p.ring_store && go && (have || n_tiles == 0)) {
+        const long long p0 = p.pos0[b];
+        constexpr int kRv = D / 8;  // 16-byte vectors per row
+        const int c_first = Mq > p.win ? Mq - p.win : 0;
+        const uint4* src = sp == 0 ? p.kn_raw : p.vn_raw;
+        uint4* dst = sp == 0 ? p.k_ring : p.v_ring;
+        const int kv = kvh[0];
+        if (p0 >= 0) {
+          for (int t = (int)threadIdx.x - 128; t < (Mq - c_first) * kRv; t += 128 * NSLOT) {
+            const int cc = c_first + t / kRv, i = t % kRv;
+            const long long slot_r = (p0 + cc) % p.win;
+            dst[(((long long)b * p.win + slot_r) * p.Hkv + kv) * kRv + i] =
+                __ldg(src + (((long long)b * Mq + cc) * p.Hkv + kv) * kRv + i);
+          }
+        }
+      }
+      const bool got = __all_sync(0xffffffffu, mbar_wait<true>(xfer, 0, p.err, abort_flag));
+      if (got) {
+        const float2 mlp = ld_shared_f2(rx_ml);
+        const float M = fmaxf(m_me, mlp.x);
+        const float a_me = m_me == -INFINITY ? 0.f : ex2_approx(m_me - M);
+        const float a_pe = mlp.x == -INFINITY ? 0.f : ex2_approx(mlp.x - M);
+        const float L_ = a_me * l_me + a_pe * mlp.y;
+        const float inv = L_ > 0.f ? 1.f / L_ : 0.f;
+        const float c_me = a_me * inv, c_pe = a_pe * inv;
+        uint16_t* orow = p.out + (((size_t)b * Mq + m_row) * p.H + h) * D + sp * kHalf;
+#pragma unroll
+        for (int j = 0; j < kHalf / 32; ++j) {
+          uint32_t v[32];
+          if (have) {
+            tmem_ld32(tO + (uint32_t)(sp * kHalf + 32 * j), v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 o = ld_shared_f4(rx_o + (uint32_t)(((j * 8 + e4) ^ (r & 7)) * 16));
+            pk[2 * e4] = pack_bf16x2(__uint_as_float(v[4 * e4]) * c_me + o.x * c_pe,
+                                     __uint_as_float(v[4 * e4 + 1]) * c_me + o.y * c_pe);
+            pk[2 * e4 + 1] = pack_bf16x2(__uint_as_float(v[4 * e4 + 2]) * c_me + o.z * c_pe,
+                                         __uint_as_float(v[4 * e4 + 3]) * c_me + o.w * c_pe);
+          }
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + 32 * j);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+          }
+        }
+        if (row_valid && sp == 0 && p.lse)
+          p.lse[((size_t)b * p.H + h) * Mq + m_row] = (M + __log2f(L_)) * 0.69314718055994531f;
+      }
+    } else if (__all_sync(0xffffffffu, fin)) {
       tc_fence_after();
       // (l == 0: a part of a split walk with none of the row's keys; its
       // lse is -inf and the merge skips it)
@@ -989,6 +1119,43 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }
+  // paired parts: neither CTA exits while the other may still write its
+  // shared memory (the softmax warps waited on the first cluster barrier
+  // in their epilogue, the others do here)
+  if (pair) {
+    if (warp < 4) cluster_wait();
+    cluster_arrive();
+    cluster_wait();
+  }
+}
+
+// Whether the device can place clusters of two CTAs of the query-window
+// form (paired parts); asked once per form.
+template <int D, int NSLOT, int NSTREAM>
+bool pair_clusters_fit() {
+  using C = Cfg<D, NSLOT, NSTREAM>;
+  static std::atomic<int> known{0};  // 0 not asked, 1 yes, -1 no
+  int k = known.load(std::memory_order_acquire);
+  if (k == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kAlloc;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(
+        &n, reinterpret_cast<const void*>(swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 1>), &cfg);
+    if (e != cudaSuccess) cudaGetLastError();
+    k = (e == cudaSuccess && n > 0) ? 1 : -1;
+    known.store(k, std::memory_order_release);
+  }
+  return k > 0;
 }
 
 template <int D, int NSLOT, int NSTREAM>
@@ -1067,11 +1234,25 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
       p.inplace = inplace ? 1 : 0;
       p.stack = (NSLOT == 2 && qw->stack) ? 1 : 0;
       p.nsplit = qw->nsplit > 1 ? qw->nsplit : 1;
-      if (p.nsplit > 1) {
+      p.pair = (p.nsplit == 2 && qw->pair && pair_clusters_fit<D, NSLOT, NSTREAM>()) ? 1 : 0;
+      if (p.nsplit > 1 && !p.pair) {
         if (!qw->part) return SWA_ERR_ARG;
         p.part_o = qw->part;
         p.part_lse = qw->part + (size_t)p.nsplit * B * H * qw->Mq * D;
       }
+      // the chunk enters the rings inside the launch when each cluster holds
+      // every reader of its kv head's ring rows: one query tile and all the
+      // kv head's query heads in one item
+      const int heads_per_item = p.stack ? 2 * NSLOT : NSLOT;
+      if (p.pair && inplace && qw->ring_k && qw->ring_v && p.nclass == 1 &&
+          p.qtile_prefix[1] == 1 && heads_per_item == H / Hkv) {
+        p.ring_store = 1;
+        p.k_ring = static_cast<uint4*>(qw->ring_k);
+        p.v_ring = static_cast<uint4*>(qw->ring_v);
+        p.kn_raw = static_cast<const uint4*>(qw->kn);
+        p.vn_raw = static_cast<const uint4*>(qw->vn);
+      }
+      if (qw->done) *qw->done = p.pair | (p.ring_store << 1);
     }
     const uint32_t box[4] = {64, 1, (uint32_t)kBlockRows, 1};
     const int nmaps = block_mode ? 1 : p.nclass;
@@ -1131,7 +1312,23 @@ int launch_impl(const void* q, const void* k, const void* v, void* out, float* l
                                              (qw ? p.nsplit : 1);
     if (grid <= 0) continue;
     if (grid > 0x7fffffffL) return SWA_ERR_UNSUPPORTED;
-    if (kind == 1)
+    if (kind == 1 && p.pair) {
+      // clusters of two: the two parts of an item are consecutive CTAs
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)grid);
+      cfg.blockDim = dim3(C::kThreads);
+      cfg.dynamicSmemBytes = C::kAlloc;
+      cfg.stream = stream;
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      if (cudaLaunchKernelEx(&cfg, swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 1>, p) != cudaSuccess)
+        return SWA_ERR_CUDA;
+    } else if (kind == 1)
       swa_fwd_sm100_kernel<D, NSLOT, NSTREAM, 1><<<(unsigned)grid, C::kThreads, C::kAlloc,
                                                    stream>>>(p);
     else if (kind == 2)

@@ -65,6 +65,16 @@ struct QueryWindow {
   int stack = 0;
   int nsplit = 1;
   float* part = nullptr;
+  // pair: with nsplit == 2, let the two parts merge each other through a
+  // cluster of two CTAs (no partials written) when the device can place the
+  // clusters; ring_k / ring_v (in place): the rings the chunk kn / vn then
+  // enters from inside the launch, when one cluster holds every reader of a
+  // kv head's ring rows.  *done (if given) reports what the launch did:
+  // bit 0 merged in pairs, bit 1 stored the chunk into the rings.
+  int pair = 0;
+  void* ring_k = nullptr;
+  void* ring_v = nullptr;
+  int* done = nullptr;
 };
 // Whether the forward for a query window of Mq rows would stack two heads
 // per tile (the launch's slot count follows the GQA group as in

@@ -694,21 +694,52 @@ __global__ void ring_store_kernel(const uint4* __restrict__ k_new, const uint4* 
   v_ring[dst] = v_new[src];
 }
 
+// The chunk of an append entering its ring slots (pos0 + c) % W: the rows
+// c >= c_first of k_new / v_new, row_vecs 16-byte vectors each.
+struct RingStore {
+  const uint4* k_new = nullptr;
+  const uint4* v_new = nullptr;
+  uint4* k_ring = nullptr;
+  uint4* v_ring = nullptr;
+  const int64_t* pos0 = nullptr;
+  int B = 0, C = 0, W = 0, row_vecs = 0, c_first = 0;
+};
+
 // Combines split key walks (the parts of a tensor-core append or decode):
 // row (b, c, h) has nsplit partial results O_i / l_i (fp32) with lse_i
 // (any number of parts, taken eight at a time); with m = max lse_i
 // and w_i = exp(lse_i - m), out = sum w_i O_i / sum w_i (bf16) and lse = m +
 // ln sum w_i (the lse identity of split softmax).  One warp per row, D / 32
-// columns per lane.
+// columns per lane.  An append also hands its ring store to this launch
+// (every key walk has read the ring by then): the grid's threads copy the
+// chunk's vectors into their slots before merging.
 template <int D>
 __global__ void __launch_bounds__(256) split_merge_kernel(const float* __restrict__ part_o,
                                                            const float* __restrict__ part_lse,
                                                            uint16_t* __restrict__ out,
                                                            float* __restrict__ lse, int nsplit,
-                                                           int B, int C, int H) {
+                                                           int B, int C, int H, RingStore rs) {
   constexpr int kPer = D / 32;  // 4 (D = 128) or 2 (D = 64) columns per lane
   constexpr int kBatch = 8;     // parts whose loads are in flight together
   using Vec = typename std::conditional<kPer == 4, float4, float2>::type;
+  if (rs.k_new) {
+    const long long per_b = (long long)(rs.C - rs.c_first) * rs.row_vecs;
+    const long long total = per_b * rs.B;
+    const long long nthr = (long long)gridDim.x * blockDim.x;
+    for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += nthr) {
+      const int b = (int)(t / per_b);
+      const long long rem = t - (long long)b * per_b;
+      const int c = rs.c_first + (int)(rem / rs.row_vecs);
+      const int i = (int)(rem % rs.row_vecs);
+      const long long p0 = rs.pos0[b];
+      if (p0 < 0) continue;
+      const long long slot = (p0 + c) % rs.W;
+      const long long src = ((long long)b * rs.C + c) * rs.row_vecs + i;
+      const long long dst = ((long long)b * rs.W + slot) * rs.row_vecs + i;
+      rs.k_ring[dst] = __ldg(rs.k_new + src);
+      rs.v_ring[dst] = __ldg(rs.v_new + src);
+    }
+  }
   const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const long long rows = (long long)B * H * C;
@@ -879,17 +910,17 @@ int ring_store(const void* k_new, const void* v_new, void* k_ring, void* v_ring,
 
 namespace {
 int merge_parts(const float* part, void* out, float* lse, int nsplit, int B, int C, int H, int D,
-                 cudaStream_t stream) {
+                 cudaStream_t stream, const RingStore& rs = RingStore()) {
   const long long rows = (long long)B * H * C;
   const float* part_lse = part + (size_t)nsplit * rows * D;
   const long long blocks = (rows + 7) / 8;
   if (blocks > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
   if (D == 128)
     split_merge_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
-        part, part_lse, static_cast<uint16_t*>(out), lse, nsplit, B, C, H);
+        part, part_lse, static_cast<uint16_t*>(out), lse, nsplit, B, C, H, rs);
   else
     split_merge_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
-        part, part_lse, static_cast<uint16_t*>(out), lse, nsplit, B, C, H);
+        part, part_lse, static_cast<uint16_t*>(out), lse, nsplit, B, C, H, rs);
   return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
@@ -897,9 +928,9 @@ int merge_parts(const float* part, void* out, float* lse, int nsplit, int B, int
 // W keys over the ring history below pos0 followed by the chunk (both read
 // in place), its queries being the chunk's C rows.  Shorter chunks would
 // leave most of a 128-row query tile idle and take the row kernel below.
-int append_attention_tc(const void* q, const void* k_new, const void* v_new, const void* k_ring,
-                        const void* v_ring, void* out, float* lse, const int64_t* pos0, int B,
-                        int C, int H, int Hkv, int D, int W, float scale, cudaStream_t stream) {
+int append_attention_tc(const void* q, const void* k_new, const void* v_new, void* k_ring,
+                        void* v_ring, void* out, float* lse, const int64_t* pos0, int B, int C,
+                        int H, int Hkv, int D, int W, float scale, cudaStream_t stream) {
   // Work items: query tiles x head groups (four heads per CTA when two are
   // stacked per tile, else two or one); when they do not fill the SMs the
   // key walks are split (the partials merged after), at least two key
@@ -934,10 +965,32 @@ int append_attention_tc(const void* q, const void* k_new, const void* v_new, con
   }
   qw.kn = k_new;
   qw.vn = v_new;
+  // two parts merge each other inside the launch (clusters of two CTAs),
+  // which can also store the chunk into the ring
+  qw.pair = nsplit == 2 ? 1 : 0;
+  qw.ring_k = k_ring;
+  qw.ring_v = v_ring;
+  int done = 0;
+  qw.done = &done;
   const int st = launch_fwd_sm100(q, k_ring, v_ring, out, lse, B, H, Hkv, W + 64 + C, D, W - 1,
                                   0, 1, 0, nullptr, 0, scale, stream, &qw);
-  if (st != SWA_OK || nsplit == 1) return st;
-  return merge_parts(qw.part, out, lse, nsplit, B, C, H, D, stream);
+  if (st != SWA_OK) return st;
+  if (done & 2) return SWA_OK;
+  if (nsplit == 1 || (done & 1))
+    return ring_store(k_new, v_new, k_ring, v_ring, pos0, B, C, Hkv, D, W, stream);
+  // the merge launch also stores the chunk into the ring
+  RingStore rs;
+  rs.k_new = static_cast<const uint4*>(k_new);
+  rs.v_new = static_cast<const uint4*>(v_new);
+  rs.k_ring = static_cast<uint4*>(k_ring);
+  rs.v_ring = static_cast<uint4*>(v_ring);
+  rs.pos0 = pos0;
+  rs.B = B;
+  rs.C = C;
+  rs.W = W;
+  rs.row_vecs = Hkv * D / 8;
+  rs.c_first = C > W ? C - W : 0;
+  return merge_parts(qw.part, out, lse, nsplit, B, C, H, D, stream, rs);
 }
 }  // namespace
 
@@ -949,12 +1002,9 @@ int split_merge(const float* part, void* out, float* lse, int nsplit, int B, int
 int launch_append(const void* q, const void* k_new, const void* v_new, void* k_ring, void* v_ring,
                   void* out, float* lse, const int64_t* pos0, int B, int C, int H, int Hkv, int D,
                   int W, float scale, cudaStream_t stream) {
-  if (C >= 32) {
-    const int st = append_attention_tc(q, k_new, v_new, k_ring, v_ring, out, lse, pos0, B, C, H,
-                                       Hkv, D, W, scale, stream);
-    if (st != SWA_OK) return st;
-    return ring_store(k_new, v_new, k_ring, v_ring, pos0, B, C, Hkv, D, W, stream);
-  }
+  if (C >= 32)
+    return append_attention_tc(q, k_new, v_new, k_ring, v_ring, out, lse, pos0, B, C, H, Hkv, D,
+                               W, scale, stream);
   RowParams p;
   std::memset(&p, 0, sizeof(p));
   if (encode_kv(&p.tmK, k_ring, D, Hkv, W, B) != SWA_OK ||

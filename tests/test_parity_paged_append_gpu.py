@@ -149,6 +149,15 @@ def test_append_configs(swa, name):
     (1, 48, 16, 2, 128, 2048, [3000]),
     (2, 50, 8, 2, 128, 1024, [1500, 20]),
     (2, 64, 8, 2, 64, 512, [600, 511]),
+    # two-part key walks merged in pairs (clusters of two CTAs): the chunk
+    # stored from inside the launch (GQA 2 at D = 128, GQA 4 stacked at
+    # D = 64, MHA at D = 64 with two CTAs per SM) or by the store kernel
+    # (GQA 8: a kv head's heads span two items); small positions leave the
+    # second part empty
+    (16, 100, 8, 4, 128, 512, [5, 3000, 700, 511, 512, 513, 9000, 64] * 2),
+    (16, 64, 16, 4, 64, 256, [300, 2, 255, 256, 1000, 77, 63, 4000] * 2),
+    (8, 40, 16, 16, 64, 256, [1, 260, 5000, 255, 128, 129, 64, 700]),
+    (8, 64, 32, 4, 128, 512, [600, 3, 511, 512, 2000, 100, 64, 65]),
 ])
 def test_append_shapes(swa, B, C, H, Hkv, D, W, pos0):
     q = inputs.normal((B, C, H, D), C + W, 0)
