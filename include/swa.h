@@ -362,11 +362,16 @@ SWA_API int swa_paged_window(int64_t pos, int W, int page_size, int64_t* first_p
  * it was before the call.  W must be a positive multiple of 64; 1 <= C <=
  * 65535; D in {64, 128}; H % Hkv == 0, H / Hkv <= 8; scale <= 0 means
  * 1/sqrt(D).  Launches on `stream`: for C >= 32 the tensor-core attention
- * reading ring and chunk in place (when its work items do not fill the
- * SMs, each key walk is split over several CTAs whose partial results go
- * to a library workspace and are merged by a second kernel), then the ring
- * update; for shorter chunks the row-kernel attention and the ring update.
- * Workspace, streams and graphs as for swa_decode.
+ * reading ring and chunk in place.  When its work items do not fill the
+ * SMs each key walk is split over several CTAs: two parts run as a
+ * cluster of two CTAs that merge each other's results on chip and, when
+ * the cluster holds every reader of its kv head's ring rows (one query
+ * tile, all the kv head's query heads in one item), also store the chunk
+ * into the ring, all in one launch; more parts write partial results to a
+ * library workspace, merged (with the ring update) by a second kernel.
+ * Without a split the ring update is a second kernel.  For shorter chunks:
+ * the row-kernel attention, then the ring update.  Workspace, streams and
+ * graphs as for swa_decode.
  */
 SWA_API int swa_append(const void* q, const void* k_new, const void* v_new, void* k_ring,
                        void* v_ring, void* out, float* lse, const int64_t* pos0, int B, int C,
