@@ -1061,6 +1061,9 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
       const float inv = l > 0.f ? 1.f / l : 0.f;
       const size_t orow_i = qwin ? (size_t)b * Mq + m_row : (size_t)b * p.N + i_phys;
       uint16_t* orow = p.out + (orow_i * p.H + h) * D;
+      // rows start on 128-byte multiples from out: 32-byte stores when out
+      // itself is 32-byte aligned
+      const bool out_v8 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
       // 64 columns of O per TMEM round trip (two loads, one wait)
 #pragma unroll
       for (int j2 = 0; j2 < D / 64; ++j2) {
@@ -1089,10 +1092,16 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
             pk[e] = pack_bf16x2(__uint_as_float(v[jj][2 * e]) * inv,
                                 __uint_as_float(v[jj][2 * e + 1]) * inv);
           if (row_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + j2 * 64 + jj * 32);
+            if (out_v8) {
+              // two full 32-byte sectors per lane
+              st_global_v8(orow + j2 * 64 + jj * 32, pk);
+              st_global_v8(orow + j2 * 64 + jj * 32 + 16, pk + 8);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(orow + j2 * 64 + jj * 32);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+              for (int e = 0; e < 4; ++e)
+                dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            }
           }
         }
       }
