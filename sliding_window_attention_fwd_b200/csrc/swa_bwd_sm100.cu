@@ -472,8 +472,9 @@ __global__ void __launch_bounds__(kThreadsB, 1)
   uint64_t* empty = full + S_;        // [S_]
   uint64_t* st_full = empty + S_;     // S^T of the step in TMEM
   uint64_t* dpt_full = st_full + 1;   // dP^T of the step in TMEM
-  uint64_t* pt_full = dpt_full + 1;   // P^T, dS^T written (128 arrivals per group)
+  uint64_t* pt_full = dpt_full + 1;   // dS^T written (128 arrivals per group)
   uint64_t* done = pt_full + 1;
+  uint64_t* p_full = done + 1;        // P^T written (128 arrivals per group)
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMisc + 4);
   float* vec = reinterpret_cast<float*>(smem + C::kVec);  // [S_][2][128]
@@ -508,6 +509,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
     mbar_init(dpt_full, 1);
     mbar_init(pt_full, 128 * kGroupsB);
     mbar_init(done, 1);
+    mbar_init(p_full, 128 * kGroupsB);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -587,10 +589,11 @@ __global__ void __launch_bounds__(kThreadsB, 1)
       const uint64_t ddomn0 = sdesc_sw128(ring_addr + C::kTile, kChunkB, 1024);
       constexpr uint64_t kStageStep = C::kStageBytes >> 4;
       const uint32_t t_dv = tmem + 256u, t_dk = tmem + 256u + (uint32_t)D;
-      // order: S^T(0), dP^T(0), then per step dV(s), S^T(s + 1), dK(s),
-      // dP^T(s + 1): each of S^T(s + 1) / dP^T(s + 1) right after the MMA that
-      // reads the columns it overwrites (P^T(s) / dS^T(s)), so the compute
-      // warps get the next S^T one MMA group sooner
+      // order: S^T(0), dP^T(0), then per step dV(s) once P^T(s) is written,
+      // S^T(s + 1), dK(s) once dS^T(s) is written, dP^T(s + 1): each of
+      // S^T(s + 1) / dP^T(s + 1) right after the MMA that reads the columns
+      // it overwrites (P^T(s) / dS^T(s)), so S^T(s + 1) is computed while the
+      // compute warps form dS^T(s)
       auto issue_st = [&](int s) -> bool {
         const int st = s % S_;
         if (!mbar_wait(&full[st], (uint32_t)(s / S_) & 1u, p.err, abort_flag)) return false;
@@ -616,7 +619,7 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         const int st = s % S_;
         const uint64_t sq = (uint64_t)st * kStageStep;
         // dV += P^T dO, dK += dS^T Q
-        if (!mbar_wait(pt_full, (uint32_t)s & 1u, p.err, abort_flag)) break;
+        if (!mbar_wait(p_full, (uint32_t)s & 1u, p.err, abort_flag)) break;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kTileM / 16; ++k)
@@ -624,6 +627,8 @@ __global__ void __launch_bounds__(kThreadsB, 1)
                  (s > 0 || k > 0) ? 1u : 0u);
         const bool next = s + 1 < n_steps;
         if (next && !issue_st(s + 1)) break;
+        if (!mbar_wait(pt_full, (uint32_t)s & 1u, p.err, abort_flag)) break;
+        tc_fence_after();
 #pragma unroll
         for (int k = 0; k < kTileM / 16; ++k)
           mma_ts(t_dk, tmem + 128u + pcol(k), dqmn0 + sq + (uint64_t)((k * 2048) >> 4), idesc_o,
@@ -695,6 +700,10 @@ __global__ void __launch_bounds__(kThreadsB, 1)
         // columns of S^T
         tmem_st16(tS + 32 * kCpg * cg + 16 * i, pp);
       }
+      // P^T is complete: dV(s), then S^T(s + 1), may go while dS^T is formed
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
       // then dS^T = P^T (dP^T - Delta)
       w = mbar_wait(dpt_full, (uint32_t)s & 1u, p.err, abort_flag);
       if (!__all_sync(0xffffffffu, w)) {
