@@ -422,7 +422,8 @@ def run_ours(args, rank, world, local_rank):
     a_flops = 4.0 * acfg.D * a_pairs
     a_bytes = (acfg.B * min(acfg.W, acfg.C + acfg.W) * acfg.Hkv * acfg.D * 2 * 2
                + (aq.numel() + aout.numel() + 2 * akn.numel()) * 2)
-    # chunks of >= 32 tokens run on the tcgen05 forward (after a staging copy)
+    # chunks of >= 32 tokens run on the tcgen05 forward, reading ring and
+    # chunk in place; the two parts of each split key walk merge on chip
     append = {"workload": acfg.name, "ms": a_ms, "tflops": a_flops / a_ms / 1e9,
               "gbs": a_bytes / a_ms / 1e6,
               "roofline": {"bound": "tensor", "achieved": a_flops / a_ms / 1e9,
