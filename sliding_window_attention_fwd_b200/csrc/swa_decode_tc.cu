@@ -139,6 +139,41 @@ __global__ void __launch_bounds__(DecCfg::kThreads, 2)
   const int ntiles = s1 > s0 ? (s1 - s0 + kTK - 1) / kTK : 0;
   const int nq = p.grp;
 
+  // load j of the walk: K of tile j / 2 (j even) or its V (j odd), into
+  // ring slot j % 3 (one thread)
+  auto load_j = [&](int j) {
+    const int st = j % kRingSlots;
+    const int kv = j & 1, t = j >> 1;
+#ifdef SWA_TEST_WITHHOLD_TILE
+    // failure-detection test build only: this K tile is never loaded, so
+    // the issuer's bounded wait for it runs out
+    if (kv == 0 && t == SWA_TEST_WITHHOLD_TILE) return;
+#endif
+    const CUtensorMap* m = kv ? &p.tmV : &p.tmK;
+    uint8_t* dst = smem + C::kRing + st * C::kTile;
+    mbar_arrive_expect_tx(&full[st], C::kTile);
+    for (int hh = 0; hh < 2; ++hh) {
+      // source row of the 64 keys from index idx0: a ring slot, or a row of
+      // the page pool (a page id past the table reads as zeros, masked
+      // below)
+      const int idx0 = s0 + t * kTK + hh * 64;
+      int row = idx0, bc = b;
+      if (p.paged) {
+        const long long t0 = a64 + idx0;
+        const long long lp = t0 / p.page_size;
+        const long long page = lp < p.max_pages ? p.table[(long)b * p.max_pages + lp] : -1;
+        row = page < 0 ? -64 : (int)(page * p.page_size + t0 % p.page_size);
+        bc = 0;
+      }
+      for (int cc = 0; cc < D / 64; ++cc)
+        tma_load_4d(dst + cc * kDecChunk + hh * (kDecChunk / 2), m, &full[st], cc * 64, g, row,
+                    bc);
+    }
+  };
+  // the first ring pass is issued by thread 0 as soon as the barriers
+  // exist, so its latency overlaps TMEM allocation and the Q gather
+  const int n_early = min(kRingSlots, 2 * ntiles);
+
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     for (int s = 0; s < kRingSlots; ++s) {
@@ -152,6 +187,11 @@ __global__ void __launch_bounds__(DecCfg::kThreads, 2)
     }
     mbar_init(o_final, 1);
     fence_mbar_init();
+    if (ntiles > 0) {
+      prefetch_tensormap(&p.tmK);
+      prefetch_tensormap(&p.tmV);
+      for (int j = 0; j < n_early; ++j) load_j(j);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::kTmemCols);
@@ -181,44 +221,16 @@ __global__ void __launch_bounds__(DecCfg::kThreads, 2)
 
   if (warp == 0) {
     // =========================== producer ===========================
-    // load j of the walk: K of tile j / 2 (j even) or its V (j odd), into
-    // ring slot j % 3
-    int last = -1;
+    // the rest of the walk (the first ring pass is already issued)
+    int last = n_early - 1;
     if (lane == 0 && ntiles > 0) {
-      prefetch_tensormap(&p.tmK);
-      prefetch_tensormap(&p.tmV);
-      for (int j = 0; j < 2 * ntiles; ++j) {
+      for (int j = n_early; j < 2 * ntiles; ++j) {
         const int st = j % kRingSlots;
         if (j >= kRingSlots &&
             !mbar_wait(&empty[st], (uint32_t)((j / kRingSlots) - 1) & 1u, p.err, abort_flag))
           break;
         last = j;
-        const int kv = j & 1, t = j >> 1;
-#ifdef SWA_TEST_WITHHOLD_TILE
-        // failure-detection test build only: this K tile is never loaded, so
-        // the issuer's bounded wait for it runs out
-        if (kv == 0 && t == SWA_TEST_WITHHOLD_TILE) continue;
-#endif
-        const CUtensorMap* m = kv ? &p.tmV : &p.tmK;
-        uint8_t* dst = smem + C::kRing + st * C::kTile;
-        mbar_arrive_expect_tx(&full[st], C::kTile);
-        for (int hh = 0; hh < 2; ++hh) {
-          // source row of the 64 keys from index idx0: a ring slot, or a row
-          // of the page pool (a page id past the table reads as zeros,
-          // masked below)
-          const int idx0 = s0 + t * kTK + hh * 64;
-          int row = idx0, bc = b;
-          if (p.paged) {
-            const long long t0 = a64 + idx0;
-            const long long lp = t0 / p.page_size;
-            const long long page = lp < p.max_pages ? p.table[(long)b * p.max_pages + lp] : -1;
-            row = page < 0 ? -64 : (int)(page * p.page_size + t0 % p.page_size);
-            bc = 0;
-          }
-          for (int cc = 0; cc < D / 64; ++cc)
-            tma_load_4d(dst + cc * kDecChunk + hh * (kDecChunk / 2), m, &full[st], cc * 64, g,
-                        row, bc);
-        }
+        load_j(j);
       }
 #ifdef SWA_TEST_WITHHOLD_TILE
       const int skip = 2 * SWA_TEST_WITHHOLD_TILE;
