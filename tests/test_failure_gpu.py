@@ -5,11 +5,13 @@
   usable afterwards.
 * The same inside the production kernels: a test-only build of the library
   (SWA_TEST_WITHHOLD_TILE) never loads one K/V tile, and lowers the bound on
-  every wait to 5 ms.  The fused forward, the tensor-core decode and the
-  split-KV row kernel must then time out, leave their abort path (in-flight copies drained, TMEM
-  released) and return; a problem that needs no withheld tile still gives
-  the oracle's result with the same library, so the context and the SM
-  resources (TMEM) are intact.
+  every wait to 5 ms.  The fused forward, the tensor-core decode, the
+  split-KV row kernel and the append's two-part clusters (whose CTAs also
+  wait on each other) must then time out, leave their abort path
+  (in-flight copies drained, TMEM released, both CTAs of a cluster meeting
+  before they exit) and return; a problem that needs no withheld tile still
+  gives the oracle's result, so the context and the SM resources (TMEM) are
+  intact.
 * A workspace allocation that fails (injected through the caller-allocator
   hook, on the host) is reported as SWA_ERR_NOMEM before any launch, and a
   counting allocator shows which calls allocate at all.
@@ -60,6 +62,7 @@ def withheld_lib(tmp_path_factory, swa):
     P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
     lib.swa_forward.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, P, I, F, P]
     lib.swa_decode.argtypes = [P, P, P, P, P, I, I, I, I, I, P]
+    lib.swa_append.argtypes = [P] * 8 + [I] * 6 + [F, P]
     lib.swa_device_error.argtypes = [P]
     return lib
 
@@ -122,6 +125,40 @@ def test_decode_abort_path(withheld_lib, D):
     assert lib.swa_device_error(_stream()) == 0
     ref, _ = oracle.decode(q.cpu(), kr2.cpu(), vr2.cpu(), pos.cpu())
     compare(out2.float().cpu().numpy(), ref, BF16_MAX_ABS, BF16_MEAN_ABS)
+
+
+def test_append_pair_abort_path(withheld_lib, swa):
+    """A chunked append whose key walks are split in two parts merged on chip
+    (64 work items: clusters of two CTAs): every part waits for its withheld
+    second K tile, gives up, and both CTAs of each cluster still meet and
+    exit.  Then the regular library's append on the same shapes equals the
+    oracle."""
+    lib = withheld_lib
+    B, C, H, Hkv, D, W = 8, 64, 32, 8, 128, 1024  # four heads per CTA, 2 parts of ~5 tiles
+    q = inputs.normal((B, C, H, D), 47, 0).cuda()
+    kn = inputs.normal((B, C, Hkv, D), 47, 1).cuda()
+    vn = inputs.normal((B, C, Hkv, D), 47, 2).cuda()
+    kr = inputs.normal((B, W, Hkv, D), 47, 3)
+    vr = inputs.normal((B, W, Hkv, D), 47, 4)
+    pos0 = torch.tensor([5000, 1024, 2000, 3000, 4000, 6000, 7000, 1100], dtype=torch.int64)
+    krd, vrd, posd = kr.cuda(), vr.cuda(), pos0.cuda()
+    out = torch.empty_like(q)
+    lse = torch.empty(B, H, C, device="cuda")
+    rc = lib.swa_append(q.data_ptr(), kn.data_ptr(), vn.data_ptr(), krd.data_ptr(),
+                        vrd.data_ptr(), out.data_ptr(), lse.data_ptr(), posd.data_ptr(), B, C, H,
+                        Hkv, D, W, 0.0, _stream())
+    assert rc == 0
+    assert lib.swa_device_error(_stream()) == TIMEOUT
+    assert lib.swa_device_error(_stream()) == 0
+    # the context and the SMs are intact: the regular library's append
+    krd, vrd = kr.cuda(), vr.cuda()
+    lse2 = torch.empty(B, H, C, device="cuda")
+    out2 = swa.swa_append(q, kn, vn, krd, vrd, posd, lse=lse2)
+    torch.cuda.synchronize()
+    assert swa.swa_device_error() == 0
+    ro, rl = oracle.append(q.cpu(), kr, vr, kn.cpu(), vn.cpu(), pos0)
+    compare(out2.float().cpu().numpy(), ro, BF16_MAX_ABS, BF16_MEAN_ABS)
+    compare(lse2.cpu().numpy(), rl, LSE_ABS, what="lse")
 
 
 def test_allocation_failure_reports_nomem(swa):
