@@ -323,9 +323,10 @@ __global__ void __launch_bounds__(DecCfg::kThreads, 2)
         if (lane == 0) red[wi * kNQ + n] = v;
       }
       // every softmax thread passes this barrier on every tile (a failed
-      // wait above only leaves garbage scores; the abort flag is read after)
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (!w_ok || *abort_flag) ok = false;
+      // wait above only leaves garbage scores); the barrier also ANDs the
+      // threads' verdicts, so all four warps leave the loop on the same tile
+      // and meet at the same named barriers after it
+      ok = bar_red_and(1, 128, ok && w_ok && !*abort_flag);
       float m_tile[kNQ];
 #pragma unroll
       for (int n = 0; n < kNQ; ++n)
@@ -388,7 +389,7 @@ __global__ void __launch_bounds__(DecCfg::kThreads, 2)
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       if (lane == 0) red[wi * kNQ + n] = v;
     }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
+    ok = bar_red_and(1, 128, ok);
 #pragma unroll
     for (int n = 0; n < kNQ; ++n)
       l_tot[n] = red[n] + red[kNQ + n] + red[2 * kNQ + n] + red[3 * kNQ + n];
@@ -396,7 +397,7 @@ __global__ void __launch_bounds__(DecCfg::kThreads, 2)
     if (ntiles == 0) {
       // an empty part (slots past the filled ones): contributes nothing
       if (r < nq) p.part_lse[rowbase + r] = -INFINITY;
-    } else if (ok && mbar_wait(o_final, 0, p.err, abort_flag)) {
+    } else if (__all_sync(0xffffffffu, ok && mbar_wait(o_final, 0, p.err, abort_flag))) {
       tc_fence_after();
       uint32_t ov[16];
       tmem_ld16(tmem + 32u + lane_off, ov);

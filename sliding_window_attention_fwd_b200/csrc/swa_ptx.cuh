@@ -121,6 +121,21 @@ __device__ __forceinline__ void drain_copies(uint64_t* bars, int stages, int fir
                 kDrainLimitNs);
 }
 
+// Named barrier `id` over `count` threads that also ANDs a predicate over
+// them: every participant gets the same result.
+__device__ __forceinline__ bool bar_red_and(int id, int count, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
 // ------------------------------------------------------------------ clusters
 // Thread-block clusters: the cluster barrier (every thread of every CTA of
 // the cluster arrives, then waits) and distributed shared memory (another
