@@ -740,6 +740,9 @@ __global__ void __launch_bounds__(256) split_merge_kernel(const float* __restric
       rs.v_ring[dst] = __ldg(rs.v_new + src);
     }
   }
+  // launched as a programmatic dependent of the kernel that wrote the
+  // partials: wait here until that grid has completed (a no-op otherwise)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const long long row = (long long)blockIdx.x * 8 + threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const long long rows = (long long)B * H * C;
@@ -915,12 +918,25 @@ int merge_parts(const float* part, void* out, float* lse, int nsplit, int B, int
   const float* part_lse = part + (size_t)nsplit * rows * D;
   const long long blocks = (rows + 7) / 8;
   if (blocks > 0x7fffffffLL) return SWA_ERR_UNSUPPORTED;
+  // a programmatic dependent launch: its launch overlaps the tail of the
+  // kernel before it, and griddepcontrol.wait orders the reads
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   if (D == 128)
-    split_merge_kernel<128><<<(unsigned)blocks, 256, 0, stream>>>(
-        part, part_lse, static_cast<uint16_t*>(out), lse, nsplit, B, C, H, rs);
+    e = cudaLaunchKernelEx(&cfg, split_merge_kernel<128>, (const float*)part, part_lse,
+                           static_cast<uint16_t*>(out), lse, nsplit, B, C, H, rs);
   else
-    split_merge_kernel<64><<<(unsigned)blocks, 256, 0, stream>>>(
-        part, part_lse, static_cast<uint16_t*>(out), lse, nsplit, B, C, H, rs);
+    e = cudaLaunchKernelEx(&cfg, split_merge_kernel<64>, (const float*)part, part_lse,
+                           static_cast<uint16_t*>(out), lse, nsplit, B, C, H, rs);
+  if (e != cudaSuccess) return SWA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? SWA_OK : SWA_ERR_CUDA;
 }
 
