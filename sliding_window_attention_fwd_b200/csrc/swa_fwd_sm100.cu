@@ -347,9 +347,15 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
 #else
   auto withheld = [](int, int) { return false; };
 #endif
-  // band tiles of the first ring pass, loaded by thread 0 as soon as the
-  // barriers exist (before TMEM allocation and the block barrier)
-  const int n_early = gitem ? 0 : min(kStages, n_band);
+  // Thread 0 loads Q and the first K tile as soon as the barriers exist
+  // (before TMEM allocation and the block barrier), the producer warp the
+  // rest of the first ring pass after the block barrier: with every CTA of
+  // a wave starting at once, a smaller first burst lands Q and K(0) sooner
+  // (measured: append 57.3 -> 55.4 us, token / block dilation 152 -> 148 /
+  // 154 -> 150 us, prefill within noise).  With global tokens the whole
+  // first ring pass goes early (there one K tile only measured 2 % slower).
+  const int n_early_k = gitem ? 0 : min(KIND == 2 ? kStages : 1, n_band);
+  const int n_early_v = gitem ? 0 : min(KIND == 2 ? kStages : 0, n_band);
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -386,9 +392,9 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
         prefetch_tensormap(&p.tmVf);
       }
       load_q();
-      for (int it = 0; it < n_early; ++it)
+      for (int it = 0; it < n_early_k || it < n_early_v; ++it)
         for (int kv = 0; kv < 2; ++kv)
-          if (!withheld(it, kv)) load_kv(it, kv);
+          if (it < (kv ? n_early_v : n_early_k) && !withheld(it, kv)) load_kv(it, kv);
     }
   }
   if (warp == 1) {
@@ -442,12 +448,14 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
         __syncwarp();
         if (lane == 0) mbar_arrive(full_q);
       }
-      // last tiles whose loads were issued (the first n_early already are)
-      int last_k = n_early - 1, last_v = n_early - 1;
-      for (int it = n_early; it < n_tiles; ++it) {
+      // last tiles whose loads were issued (the first n_early_k / n_early_v
+      // already are)
+      int last_k = n_early_k - 1, last_v = n_early_v - 1;
+      for (int it = min(n_early_k, n_early_v); it < n_tiles; ++it) {
         const int st = it % kStages;
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         for (int kv = 0; kv < 2; ++kv) {  // 0: K, 1: V
+          if (it < (kv ? n_early_v : n_early_k)) continue;
           uint64_t* emp = kv ? &empty_v[st] : &empty_k[st];
           uint64_t* ful = kv ? &full_v[st] : &full_k[st];
           uint8_t* dst = smem + C::kRing + st * C::kStageBytes + kv * NSTREAM * C::kTile;
