@@ -2,8 +2,8 @@
 // memory: host -> device copies, the fused kernel and device -> host copies
 // of one call, overlapped chunk by chunk.
 //
-// The query rows are cut into chunks of kChunkRows (whole 128-row query
-// tiles).  Chunk c needs its own q rows and the k / v rows of its windows;
+// The query rows are cut into chunks (whole 128-row query tiles): short
+// first and last chunks, long ones between.  Chunk c needs its own q rows and the k / v rows of its windows;
 // with a window bounded on the right (causal, or win_right >= 0) those are
 // rows below the chunk's end + win_right, most of them already copied for
 // the chunks before.  Three streams: copies in (library-owned), the kernel
@@ -26,8 +26,9 @@
 namespace swa {
 namespace {
 
-constexpr int kChunkRows = 1024;
-constexpr int kMaxChunks = 64;  // events per device; longer inputs use longer chunks
+constexpr int kEdgeRows = 512;   // first and last chunk
+constexpr int kMidRows = 2048;   // the chunks between (longer for long inputs)
+constexpr int kMaxChunks = 64;   // events per device
 constexpr int kMaxDevH = 64;
 
 struct HostPipe {
@@ -82,10 +83,27 @@ int forward_host(const void* qh, const void* kh, const void* vh, void* oh, float
   if (!hp) return SWA_ERR_CUDA;
   const size_t qrow = (size_t)H * D * 2, kvrow = (size_t)Hkv * D * 2;
   const bool chunked = d == 1 && bs <= 1 && ng == 0 && R >= 0;
-  int chunk = kChunkRows;
-  while (chunked && (N + chunk - 1) / chunk > kMaxChunks) chunk *= 2;
-  const int nchunks = chunked ? (N + chunk - 1) / chunk : 1;
-  if (!chunked) chunk = N;
+  // chunk boundaries (multiples of 128 rows): a short first chunk (its copy
+  // in is the one nothing overlaps), long middle chunks (fewer copies), a
+  // short last chunk (its kernel and copy out are the ones nothing
+  // overlaps)
+  int bounds[kMaxChunks + 1];
+  int nchunks = 0;
+  bounds[0] = 0;
+  const int last0 = (N - kEdgeRows) / kTileM * kTileM;  // start of the last chunk
+  if (!chunked || last0 <= kEdgeRows) {
+    bounds[++nchunks] = N;
+  } else {
+    int mid = kMidRows;
+    while ((last0 - kEdgeRows + mid - 1) / mid > kMaxChunks - 2) mid *= 2;
+    int r = kEdgeRows;
+    bounds[++nchunks] = r;
+    while (r < last0) {
+      r = r + mid < last0 ? r + mid : last0;
+      bounds[++nchunks] = r;
+    }
+    bounds[++nchunks] = N;
+  }
 
   // everything below runs after the work already queued on `stream`
   if (cudaEventRecord(hp->start, stream) != cudaSuccess ||
@@ -94,7 +112,7 @@ int forward_host(const void* qh, const void* kh, const void* vh, void* oh, float
     return SWA_ERR_CUDA;
   int kv_done = 0;
   for (int c = 0; c < nchunks; ++c) {
-    const int n0 = c * chunk, n1 = n0 + chunk < N ? n0 + chunk : N;
+    const int n0 = bounds[c], n1 = bounds[c + 1];
     // k / v rows the chunk's windows reach (all of them when not chunked)
     const int kv_end = !chunked ? N : (n1 + R < N ? n1 + R : N);
     if (copy_rows(qd, qh, B, N, qrow, n0, n1, cudaMemcpyHostToDevice, hp->s_in) != cudaSuccess ||

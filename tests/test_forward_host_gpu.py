@@ -27,6 +27,7 @@ def swa():
     (1, 3000, 8, 2, 128, 700, 0, 1, 0, None, True),     # causal, 3 chunks, ragged
     (2, 2500, 4, 4, 64, 300, 100, 1, 0, None, True),    # right-bounded band, B = 2
     (1, 4096, 4, 1, 128, 4095, 0, 1, 0, None, False),   # 4 chunks, no lse
+    (1, 9000, 4, 1, 64, 1500, 0, 1, 0, None, True),     # 6 chunks: short, 2048s, ragged
     (1, 1500, 2, 2, 64, 40, 40, 1, 0, [0, 700], True),  # globals: one chunk
     (1, 1200, 2, 1, 128, 30, 30, 3, 0, None, True),     # dilation: one chunk
     (1, 1100, 2, 2, 64, 128, 0, 2, 64, None, True),     # block dilation: one chunk
