@@ -289,7 +289,22 @@ __global__ void __launch_bounds__(Cfg<D, NSLOT, NSTREAM>::kThreads,
   // in place: the masked rows between the history and the chunk
   const int gap_lo = inplace ? ip_hs + p.win - 1 : 0, gap_hi = inplace ? ip_cs : 0;
   const int n_band = tr.kv_end - tr.kv_begin;
-  const int n_gtiles = (!glob || gitem) ? 0 : (p.n_global + kTileN - 1) / kTileN;
+  int n_gtiles = (!glob || gitem) ? 0 : (p.n_global + kTileN - 1) / kTileN;
+  if (n_gtiles > 0 && p.d == 1 && p.bs <= 1 && p.L >= 0) {
+    // token-level band: a global key g joins row i unless i - L <= g <= i +
+    // R (in the band) or, causal, g > i.  If no row of the tile [qm0, qm1]
+    // takes any global key (the smallest one lies inside or right of every
+    // row's band, the largest inside or left of it), the global-key tiles
+    // would be fully masked: skip them (attention sinks near the start of
+    // the sequence, seen by the first W rows through the band anyway).
+    const int qr0 = qt * kTileM, qr1 = min(qt * kTileM + kTileM - 1, Mv - 1);
+    int g_first = __ldg(p.G), g_last = __ldg(p.G + p.n_global - 1);
+    g_first = g_first < 0 ? 0 : (g_first >= p.N ? p.N - 1 : g_first);
+    g_last = g_last < 0 ? 0 : (g_last >= p.N ? p.N - 1 : g_last);
+    const bool left = g_first < qr1 - p.L;
+    const bool right = p.R > 0 && g_last > qr0 + p.R;  // causal (R == 0) takes none right
+    if (!left && !right) n_gtiles = 0;
+  }
   const int n_tiles = n_band + n_gtiles;
   const bool block_mode = p.bs > 1;
   const int map_idx = block_mode ? 0 : cl;

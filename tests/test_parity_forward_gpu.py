@@ -115,6 +115,12 @@ SMALL_BF16 = [
     (2, 900, 2, 2, 64, 16, 16, 4, 0, [1, 2, 450, 899]),       # token dilation + globals
     (1, 96, 2, 1, 128, 3, 3, 1, 0, list(range(96))),          # every row global = full attention
     (1, 260, 3, 3, 128, 10, 0, 1, 0, [129, 130, 259]),        # odd head count, causal
+    # query tiles whose rows take no global key skip the global-key tiles:
+    # causal sinks inside the first tiles' bands, and globals inside the
+    # band on both sides of a bidirectional window
+    (1, 1200, 4, 2, 128, 300, 0, 1, 0, [0, 1, 2, 3]),          # sinks: tiles 0-2 skip
+    (1, 1100, 4, 4, 64, 300, 0, 1, 0, [0, 2, 130, 131]),        # sinks + a later global
+    (1, 900, 2, 2, 128, 400, 400, 1, 0, [300, 350]),            # in every band of tiles 0-4
 ]
 
 
